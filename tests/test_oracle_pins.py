@@ -1,0 +1,335 @@
+"""Pins of the CPU oracle against facts other than itself: published tables,
+closed forms, invariants, library routines and brute force on tiny inputs.
+Each test would fail on a plausible slip in the oracle (a dropped term, a
+wrong sign, a transposed operand, a wrong tie rule)."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import gen
+import oracle
+from conftest import read_golden
+from oracle import inputs as oin
+
+F64 = torch.float64
+
+
+# ---------------------------------------------------------------- number formats
+def test_bf16_round_matches_torch_on_fp32_values():
+    a = torch.randn(100_000, generator=torch.Generator().manual_seed(1), dtype=torch.float32) * 37.0
+    want = a.to(torch.bfloat16).to(F64)
+    got = oracle.bf16_round(a.to(F64))
+    assert torch.equal(got, want)
+
+
+def test_bf16_round_is_nearest_even_on_fp64_values():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(20_000) * 10.0 ** rng.integers(-5, 5, 20_000)
+    # include exact midpoints between bf16 neighbours
+    mid = np.array([1.0 + 2.0**-8, 1.0 + 3 * 2.0**-8, -(2.0 + 2.0**-7)])
+    x = np.concatenate([x, mid])
+    r = oracle.bf16_round(torch.from_numpy(x)).numpy()
+    for xi, ri in zip(x, r):
+        e = math.frexp(abs(xi))[1]  # |x| in [2^(e-1), 2^e)
+        ulp = 2.0 ** (e - 1 - 7)
+        lo = math.floor(abs(xi) / ulp) * ulp
+        hi = lo + ulp
+        d_lo, d_hi = abs(xi) - lo, hi - abs(xi)
+        if d_lo < d_hi:
+            want = lo
+        elif d_hi < d_lo:
+            want = hi
+        else:
+            want = lo if (round(lo / ulp) % 2 == 0) else hi
+        assert abs(ri) == want and (ri == 0 or np.sign(ri) == np.sign(xi))
+
+
+def test_e2m1_dequant_matches_ocp_table():
+    tab = {int(r[0]): float(r[1]) for r in read_golden("e2m1_ocp_mx.txt")}
+    for s in (1, 100, 120, 127, 130, 200):
+        codes = np.array([[c | (d << 4) for c, d in zip(range(0, 16, 2), range(1, 16, 2))] * 4], np.uint8)
+        scales = np.full((1, 2), s, np.uint8)
+        v = oracle.mxfp4_dequant(codes, scales)[0].numpy()
+        for k in range(32):
+            assert v[k] == tab[k % 16] * 2.0 ** (s - 127)
+    nan = oracle.mxfp4_dequant(np.zeros((1, 16), np.uint8), np.full((1, 1), 255, np.uint8))
+    assert torch.isnan(nan).all()
+
+
+def test_mxfp4_dequant_of_generator_output_is_bf16_exact():
+    # E2M1 x 2^e needs at most 2 significant bits: exact in bfloat16.
+    c, s = gen.fill_host_mxfp4(0, 7, 0, 8, 512, 512**-0.5)
+    v = oracle.mxfp4_dequant(c, s)
+    assert torch.equal(oracle.bf16_round(v), v)
+
+
+# ---------------------------------------------------------------- router
+def test_sigmoid_matches_scipy():
+    x = torch.linspace(-30, 30, 2001, dtype=F64)
+    assert torch.allclose(oracle.sigmoid(x), torch.from_numpy(scipy.special.expit(x.numpy())), rtol=1e-15, atol=0)
+
+
+def test_router_orientation():
+    # W_r = a row permutation: logit e = x[perm[e]]
+    H = 7
+    perm = [3, 0, 6, 1, 5, 2, 4]
+    Wr = torch.zeros(H, H, dtype=F64)
+    for e, h in enumerate(perm):
+        Wr[e, h] = 1.0
+    x = torch.randn(5, H, dtype=F64, generator=torch.Generator().manual_seed(0))
+    s = oracle.router_scores(x, Wr)
+    want = torch.from_numpy(scipy.special.expit(x[:, perm].numpy()))
+    assert torch.allclose(s, want, rtol=1e-15, atol=0)
+
+
+def _brute_force_topk(key, k):
+    """Best k-subset by total key; among equal totals the lexicographically
+    smallest sorted index tuple.  Slots then in (key desc, index asc)."""
+    E = len(key)
+    best, best_set = None, None
+    for sub in itertools.combinations(range(E), k):
+        tot = sum(key[i] for i in sub)
+        if best is None or tot > best or (tot == best and sub < best_set):
+            best, best_set = tot, sub
+    return sorted(best_set, key=lambda i: (-key[i], i))
+
+
+@pytest.mark.parametrize("E,k", [(6, 1), (6, 3), (8, 4), (10, 2), (12, 4)])
+def test_select_experts_brute_force(E, k):
+    rng = np.random.default_rng(E * 100 + k)
+    for trial in range(40):
+        # quantised values produce exact ties in s + b
+        s = rng.integers(1, 8, size=E) / 8.0
+        b = rng.integers(-2, 3, size=E) / 8.0
+        key = s + b
+        idx, p, margin = oracle.select_experts(torch.tensor(s[None]), torch.tensor(b), k)
+        want = _brute_force_topk(list(key), k)
+        assert idx[0].tolist() == want
+        # mixture weights: unbiased scores renormalised over the chosen set
+        assert torch.allclose(p[0], torch.tensor(s[want] / s[want].sum()), rtol=0, atol=1e-15)
+        srt = sorted(key, reverse=True)
+        assert margin[0].item() == pytest.approx(srt[k - 1] - srt[k]) if k < E else True
+
+
+def test_mixture_weights_use_unbiased_scores():
+    s = torch.tensor([[0.9, 0.2, 0.3, 0.1]], dtype=F64)
+    b = torch.tensor([-1.0, 0.5, 0.0, 0.0], dtype=F64)  # the bias reorders the selection
+    idx, p, _ = oracle.select_experts(s, b, 2)
+    assert idx[0].tolist() == [1, 2]  # keys 0.7, 0.3 beat -0.1 and 0.1
+    assert torch.allclose(p[0], torch.tensor([0.2 / 0.5, 0.3 / 0.5], dtype=F64))
+    assert abs(p.sum().item() - 1.0) < 1e-15
+
+
+def test_select_from_f32_scores_uses_fp32_key():
+    # 0.5 + 2^-30 rounds to 0.5 in fp32: the keys tie there and the lower
+    # index wins, although in fp64 the tiny bias decides.
+    s2 = np.array([[0.5, 0.5]], np.float32)
+    b2 = np.array([0.0, np.float32(2.0**-30)], np.float32)
+    idx2, _ = oracle.select_experts_from_f32_scores(s2, b2, 1)
+    assert idx2[0, 0].item() == 0
+    idx3, _, _ = oracle.select_experts(torch.tensor(s2, dtype=F64), torch.tensor(b2, dtype=F64), 1)
+    assert idx3[0, 0].item() == 1  # in fp64 the tiny bias decides
+
+
+def test_permute_invariants_and_library_sort():
+    rng = np.random.default_rng(5)
+    T, E, k = 300, 17, 4
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
+    counts, offsets, perm_token, inv_perm = oracle.permute(idx, E)
+    assert counts.sum() == T * k and np.all(np.diff(offsets) >= 0) and offsets[-1] == T * k
+    assert np.array_equal(np.bincount(idx.ravel(), minlength=E), counts)
+    # stable library sort of the flattened expert ids gives the same order
+    order = np.argsort(idx.ravel(), kind="stable")
+    assert np.array_equal(perm_token, order // k)
+    inv = np.empty(T * k, np.int64)
+    inv[order] = np.arange(T * k)
+    assert np.array_equal(inv_perm, inv)
+    for e in range(E):
+        seg = perm_token[offsets[e] : offsets[e + 1]]
+        assert np.all(np.diff(seg) > 0)
+        assert all(e in idx[t] for t in seg)
+    # inv_perm o perm = identity on the pairs
+    for t in range(T):
+        for j in range(k):
+            assert perm_token[inv_perm[t * k + j]] == t
+
+
+# ---------------------------------------------------------------- experts
+def test_situ_glu_properties():
+    g = torch.linspace(-40, 40, 801, dtype=F64)[:, None]
+    v = torch.linspace(-40, 40, 161, dtype=F64)[None, :]
+    c = 10.0
+    h = oracle.situ_glu(g, v, c)
+    assert torch.allclose(oracle.situ_glu(g, -v, c), -h, rtol=0, atol=0)  # odd in v
+    assert h.abs().max() <= c * c
+    # c -> infinity gives SwiGLU (library silu)
+    big = oracle.situ_glu(g, v, 1e6)
+    sw = torch.nn.functional.silu(g) * v
+    assert torch.allclose(big, sw, rtol=1e-8, atol=1e-12)
+    # small arguments: 0 <= 1 - h/swiglu <= (g^2 + v^2) / (3 c^2)
+    gs = torch.linspace(-2, 2, 41, dtype=F64)[:, None]
+    vs = torch.linspace(-2, 2, 41, dtype=F64)[None, :]
+    hs = oracle.situ_glu(gs, vs, c)
+    sws = torch.nn.functional.silu(gs) * vs
+    mask = sws.abs() > 1e-12
+    rel = 1.0 - hs[mask] / sws[mask]
+    bound = ((gs**2 + vs**2) / (3 * c * c)).expand_as(hs)[mask]
+    assert (rel >= -1e-15).all() and (rel <= bound + 1e-15).all()
+    # the cap binds: large positive g, v -> c^2
+    assert abs(oracle.situ_glu(torch.tensor(1e3, dtype=F64), torch.tensor(1e3, dtype=F64), c).item() - c * c) < 1e-9
+
+
+def test_expert_forward_orientation():
+    # permutation weights: g = z[pg], v = z[pv], y = h[po]
+    L = I = 6
+    rng = np.random.default_rng(0)
+    pg, pv, po = rng.permutation(L), rng.permutation(L), rng.permutation(I)
+
+    def P(p):
+        m = torch.zeros(len(p), len(p), dtype=F64)
+        m[torch.arange(len(p)), torch.as_tensor(p)] = 1.0
+        return m
+
+    z = torch.randn(3, L, dtype=F64, generator=torch.Generator().manual_seed(2))
+    y = oracle.expert_forward(z, P(pg), P(pv), P(po), 10.0, lambda t: t)
+    h = oracle.situ_glu(z[:, pg], z[:, pv], 10.0)
+    assert torch.equal(y, h[:, po])
+    # the stored h is rounded before the down projection
+    yb = oracle.expert_forward(z, P(pg), P(pv), P(po), 10.0, oracle.bf16_round)
+    assert torch.equal(yb, oracle.bf16_round(h)[:, po])
+
+
+def test_shared_experts_orientation():
+    # two shared experts with permutation weights on a square hidden size
+    H = 5
+    rng = np.random.default_rng(9)
+    ps = [(rng.permutation(H), rng.permutation(H), rng.permutation(H)) for _ in range(2)]
+
+    def P(p):
+        m = torch.zeros(len(p), len(p), dtype=F64)
+        m[torch.arange(len(p)), torch.as_tensor(p)] = 1.0
+        return m
+
+    Wsg = torch.stack([P(a) for a, _, _ in ps])
+    Wsv = torch.stack([P(b) for _, b, _ in ps])
+    Wso = torch.stack([P(c) for _, _, c in ps])
+    x = torch.randn(4, H, dtype=F64, generator=torch.Generator().manual_seed(3))
+    y = oracle.shared_experts(x, Wsg, Wsv, Wso, 10.0, lambda t: t)
+    want = sum(oracle.situ_glu(x[:, a], x[:, b], 10.0)[:, c] for a, b, c in ps)
+    assert torch.allclose(y, want, rtol=1e-15, atol=1e-15)
+
+
+def test_combine_one_hot_and_linear():
+    y = torch.randn(4, 3, 5, dtype=F64, generator=torch.Generator().manual_seed(4))
+    for j in range(3):
+        p = torch.zeros(4, 3, dtype=F64)
+        p[:, j] = 1.0
+        assert torch.equal(oracle.combine(y, p), y[:, j])
+    p = torch.rand(4, 3, dtype=F64, generator=torch.Generator().manual_seed(5))
+    want = torch.einsum("tj,tjl->tl", p, y)
+    assert torch.allclose(oracle.combine(y, p), want, rtol=1e-14, atol=1e-15)
+
+
+def test_rms_norm_closed_forms():
+    gam = torch.ones(8, dtype=F64)
+    for a in (1e-3, 0.5, 7.0, -3.0):
+        u = torch.full((1, 8), a, dtype=F64)
+        n = oracle.rms_norm(u, gam, 1e-6)
+        assert torch.allclose(n, torch.full((1, 8), a / math.sqrt(a * a + 1e-6), dtype=F64), rtol=1e-15)
+    u = torch.randn(6, 64, dtype=F64, generator=torch.Generator().manual_seed(7))
+    n = oracle.rms_norm(u, torch.ones(64, dtype=F64), 0.0)
+    assert torch.allclose(n, oracle.rms_norm(u * 123.0, torch.ones(64, dtype=F64), 0.0), rtol=1e-14)
+    assert torch.allclose((n * n).mean(dim=1), torch.ones(6, dtype=F64), rtol=1e-14)
+    g = torch.randn(64, dtype=F64, generator=torch.Generator().manual_seed(8))
+    assert torch.allclose(oracle.rms_norm(u, g, 0.0), g[None] * n, rtol=1e-14)
+    ms = (u * u).mean(dim=1)
+    n1 = oracle.rms_norm(u, torch.ones(64, dtype=F64), 0.25)
+    assert torch.allclose((n1 * n1).mean(dim=1), ms / (ms + 0.25), rtol=1e-14)
+
+
+# ---------------------------------------------------------------- whole layer
+def _tiny_weights(cfg):
+    return oin.all_weights(cfg)
+
+
+def test_identical_experts_reduce_to_dense_glu():
+    """Zero bias and identical experts: the routed mixture is one dense GLU
+    (the renormalised weights sum to one), for any routing."""
+    cfg = gen.CONFIGS["tiny"]
+    w = _tiny_weights(cfg)
+    w["bias"] = torch.zeros(cfg.E, dtype=F64)
+    for name in ("Wg", "Wv", "Wo"):
+        w[name] = w[name][:1].expand_as(w[name]).clone()
+    x = oin.x_rows(cfg, range(cfg.T))
+    out = oracle.layer_forward(cfg, w, x)
+    rnd = oracle.storage_round(cfg.act)
+    z = rnd(x @ w["Wdown"].T)
+    u_dense = oracle.expert_forward(z, w["Wg"][0], w["Wv"][0], w["Wo"][0], cfg.situ_c, rnd)
+    assert torch.allclose(out["u"], u_dense, rtol=1e-12, atol=1e-13)
+    n = rnd(oracle.rms_norm(u_dense, w["gamma"], cfg.rms_eps))
+    y = oracle.shared_experts(x, w["Wsg"], w["Wsv"], w["Wso"], cfg.situ_c, rnd) + n @ w["Wup"].T
+    assert torch.allclose(out["y"], y, rtol=1e-12, atol=1e-12)
+
+
+def test_latent_projection_orientation():
+    """W_down = [I | 0] selects the first L hidden coordinates of x."""
+    cfg = gen.CONFIGS["tiny"]
+    w = _tiny_weights(cfg)
+    w["Wdown"] = torch.zeros(cfg.L, cfg.H, dtype=F64)
+    w["Wdown"][torch.arange(cfg.L), torch.arange(cfg.L)] = 1.0
+    x = oin.x_rows(cfg, range(8))
+    out = oracle.layer_forward(cfg, w, x)
+    assert torch.equal(out["z"], x[:, : cfg.L])
+
+
+def test_top1_routing_uses_the_selected_expert_only():
+    """k = 1: p = 1 and u is the chosen expert's output."""
+    cfg = gen.CONFIGS["tiny"].with_(k=1)
+    w = _tiny_weights(cfg)
+    x = oin.x_rows(cfg, range(16))
+    out = oracle.layer_forward(cfg, w, x)
+    assert torch.equal(out["p"], torch.ones(16, 1, dtype=F64))
+    rnd = oracle.storage_round(cfg.act)
+    for t in range(16):
+        e = out["idx"][t, 0].item()
+        ye = oracle.expert_forward(out["z"][t : t + 1], w["Wg"][e], w["Wv"][e], w["Wo"][e], cfg.situ_c, rnd)
+        assert torch.allclose(out["u"][t : t + 1], ye, rtol=1e-14, atol=1e-15)
+
+
+def test_streamed_forward_equals_in_memory_forward():
+    cfg = gen.CONFIGS["tiny"]
+    w = _tiny_weights(cfg)
+    x = oin.x_rows(cfg, range(cfg.T))
+    a = oracle.layer_forward(cfg, w, x)
+    b = oracle.layer_forward_streamed(cfg, w, x, lambda e: (w["Wg"][e], w["Wv"][e], w["Wo"][e]))
+    assert torch.equal(a["idx"], b["idx"]) and torch.allclose(a["y"], b["y"], rtol=1e-14, atol=1e-14)
+
+
+def test_storage_rounding_points():
+    """bf16 workloads: z, n (and h, shared h) are bf16 values; u, y are not."""
+    cfg = gen.CONFIGS["mid"].with_(T=16)
+    w = oin.dense_weights(cfg)
+    x = oin.x_rows(cfg, range(16))
+    out = oracle.layer_forward_streamed(cfg, w, x, lambda e: oin.expert_weights(cfg, e))
+    assert torch.equal(oracle.bf16_round(out["z"]), out["z"])
+    assert torch.equal(oracle.bf16_round(out["n"]), out["n"])
+    assert not torch.equal(oracle.bf16_round(out["u"]), out["u"])
+    assert not torch.equal(oracle.bf16_round(out["y"]), out["y"])
+
+
+def test_k3_parameter_count_matches_the_published_total():
+    """3-matrix GLU experts in the latent space, shared intermediate 3072 and
+    93 MoE layers give 2.770T parameters, within 0.5% of the printed 2.78T."""
+    t = {r[0]: float(r[1]) for r in read_golden("k3_model_table.txt")}
+    cfg = gen.CONFIGS["prefill"]
+    assert (cfg.H, cfg.L, cfg.E, cfg.k, cfg.I, cfg.S) == (
+        t["hidden"], t["latent"], t["routed_experts"], t["top_k"], t["expert_intermediate"], t["shared_experts"])
+    per_layer = cfg.E * 3 * cfg.L * cfg.I + cfg.S * 3 * cfg.H * cfg.Is + 2 * cfg.H * cfg.L + cfg.E * cfg.H
+    total = per_layer * t["layers"]
+    assert abs(total / t["total_params"] - 1.0) < 0.005
+    active = (cfg.k * 3 * cfg.L * cfg.I + cfg.S * 3 * cfg.H * cfg.Is + 2 * cfg.H * cfg.L + cfg.E * cfg.H) * t["layers"]
+    assert active < t["active_params"]  # the rest is attention and embeddings
