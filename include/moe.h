@@ -1,0 +1,195 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) Stable LatentMoE layer forward pass.
+ *
+ * The layer (web page "Kimi K3の896エキスパートを「896人の専門家」と呼ぶと何が
+ * ズレるか、ルーターは何を選んでいるのか", section "K3のエキスパートは896個の
+ * 小型LLMではない", the three layer equations; section "ルーターは計算の割当器",
+ * the router equation):
+ *
+ *   s   = Sigmoid(W_r x)                          router scores, one per routed expert
+ *   S   = the k experts with the largest s + b    b: frozen per-expert balancing bias
+ *   p_j = s_{S_j} / sum_{j'} s_{S_j'}             mixture weights from the UNBIASED scores
+ *   z   = W_down x                                latent projection (H -> L)
+ *   u   = sum_j p_j E_{S_j}(z)                    routed GLU experts on the latent
+ *   y   = E1_shared(x) + ... + ES_shared(x) + W_up RMSNorm(u)
+ *
+ * with every expert E(a) = W_o SiTU-GLU(W_g a, W_v a) and
+ *   SiTU-GLU(g, v) = sigmoid(g) * c*tanh(g/c) * c*tanh(v/c)        (c = situ_c)
+ * (tech-report summary "幅のスケーリング：Stable LatentMoE" describes SiTU-GLU only
+ * as SwiGLU with smooth caps on the linear and up branches; this closed form is
+ * the library's reading), and RMSNorm(u) = gamma * u / sqrt(mean(u^2) + eps).
+ * Inference uses the fixed bias with plain top-k selection (page "Kimi K3の
+ * 二軸スケーリング戦略とは何か", section "Stable LatentMoE：条件付きの大容量を
+ * 安定させる").  Routing is dropless: every token gets its k experts.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc / PyTorch CUDA memory)
+ *    on the current device, row-major and contiguous in the stated shape,
+ *    16-byte aligned.  The caller allocates and owns every buffer, including
+ *    the workspace; the library never allocates, frees or synchronises (except
+ *    moe_device_error, which says so).
+ *  - Arguments are validated on the host before anything is launched; a bad
+ *    argument returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a
+ *    combination this build does not implement) and launches nothing.
+ *  - A failed launch returns MOE_ERR_CUDA.  No C++ exception crosses the ABI.
+ *  - Work is enqueued on `stream` in order; results are ready when the stream
+ *    reaches that point.  Identical inputs give bitwise-identical outputs.
+ *  - Device-side faults the host cannot see beforehand (an expert index out of
+ *    range in a caller-supplied topk_idx, a pipeline wait that ran out of time)
+ *    are recorded in a device flag read by moe_device_error; kernels then skip
+ *    the offending access, so memory stays in bounds.
+ *
+ * Supported type combinations (moe_dims.act / routed):
+ *  - MOE_F32 / MOE_F32     fp32 everywhere (CUDA-core path, small layers);
+ *  - MOE_BF16 / MOE_BF16   bf16 operands, fp32 accumulation (tcgen05 path);
+ *    H, L, I and Is must be multiples of 64, S <= 3, E <= 1024, k <= 32.
+ * Stored activations (z, expert h, shared h, n) are held in the activation type;
+ * y_perm, u and the router scores are fp32.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream); NULL means the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null / misaligned pointer, inconsistent sizes, workspace too small */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but not implemented in this build (type combination, dims) */
+  MOE_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+  MOE_ERR_DEVICE = 4       /* moe_device_error only: a kernel recorded a device-side fault */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP4 = 2 } moe_dtype;
+
+/* Layer shape and numerics.  K3 values: H=7168, L=3584, E=896, k=16, I=3072,
+ * S=2, Is=3072 (dimension table of the page cited above). */
+typedef struct {
+  int64_t T;         /* tokens in this call (>= 0; 0 is a no-op) */
+  int32_t H;         /* hidden size */
+  int32_t L;         /* latent size */
+  int32_t E;         /* routed experts */
+  int32_t k;         /* experts per token, 1 <= k <= min(E, 32) */
+  int32_t I;         /* routed-expert intermediate size */
+  int32_t S;         /* shared experts (>= 0) */
+  int32_t Is;        /* shared-expert intermediate size */
+  float situ_c;      /* SiTU-GLU cap c (> 0); 10 in the measured configurations */
+  float rms_eps;     /* RMSNorm epsilon (>= 0); 1e-6 */
+  moe_dtype act;     /* x, dense weights and stored activations: MOE_F32 or MOE_BF16 */
+  moe_dtype routed;  /* routed-expert weights: equal to act */
+  moe_dtype y_out;   /* y: MOE_F32, or equal to act */
+} moe_dims;
+
+/* Layer weights (device pointers, type `act` unless stated). */
+typedef struct {
+  const void* Wr;      /* [E, H]    router projection */
+  const float* bias;   /* [E]       fp32 selection bias (frozen) */
+  const void* Wdown;   /* [L, H]    latent down-projection */
+  const void* Wup;     /* [H, L]    latent up-projection */
+  const float* gamma;  /* [L]       fp32 RMSNorm gain */
+  const void* Wg;      /* [E, I, L] routed gate projections (type `routed`) */
+  const void* Wv;      /* [E, I, L] routed up projections */
+  const void* Wo;      /* [E, L, I] routed down projections */
+  const uint8_t* Sg;   /* reserved for block-scaled routed weights; must be NULL */
+  const uint8_t* Sv;   /* reserved; must be NULL */
+  const uint8_t* So;   /* reserved; must be NULL */
+  const void* Wsg;     /* [S, Is, H] shared gate projections */
+  const void* Wsv;     /* [S, Is, H] shared up projections */
+  const void* Wso;     /* [S, H, Is] shared down projections */
+} moe_weights;
+
+/* Optional extra outputs of moe_layer_forward; every field may be NULL.
+ * Given buffers receive the intermediate directly (no extra pass). */
+typedef struct {
+  float* scores;            /* [T, E]  fp32 router scores s = sigmoid(W_r x) */
+  int32_t* topk_idx;        /* [T, k]  selected experts, descending key, ties to lower index */
+  float* topk_w;            /* [T, k]  mixture weights p (fp32, sum to 1 per token) */
+  int32_t* expert_offsets;  /* [E+1]   CSR offsets of the expert-contiguous pair order */
+  float* u;                 /* [T, L]  fp32 mixture before RMSNorm */
+  void* n;                  /* [T, L]  RMSNorm(u) in the activation type */
+  void* z;                  /* [T, L]  W_down x in the activation type */
+} moe_aux;
+
+/* Bytes of workspace moe_layer_forward needs for these dims (also enough for
+ * moe_permute and moe_expert_ffn).  0 for invalid dims.  The workspace must be
+ * 256-byte aligned; its contents need not be initialised and are clobbered. */
+MOE_API size_t moe_workspace_size(const moe_dims* d);
+
+/* Router and selection ("ルーターは計算の割当器": s = Sigmoid(W_r x); bias added
+ * for the choice only; mixture weights = original scores normalised over the
+ * chosen experts).
+ *   from_scores == 0: scores[T,E] (fp32, written) = sigmoid(x[T,H] . Wr[E,H]^T),
+ *                     accumulated in fp32; then selection from those scores.
+ *   from_scores != 0: scores[T,E] is INPUT; x and Wr are not read (may be NULL).
+ * Selection: key_e = fl32(scores[t,e] + bias[e]); the k largest keys, listed
+ * in descending key order, equal keys to the lower expert index;
+ * topk_w[t,j] = scores[t,idx_j] / sum_j' scores[t,idx_j'] (fp32, summed in slot
+ * order).  Outputs topk_idx[T,k] int32, topk_w[T,k] fp32. */
+MOE_API moe_status moe_router_topk(const moe_dims* d, const void* x, const void* Wr, const float* bias, float* scores,
+                           int from_scores, int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* Dispatch: stable counting sort of the T*k (token, slot) pairs by expert.
+ * Pairs of expert e occupy positions expert_offsets[e] .. expert_offsets[e+1]-1
+ * in ascending token order; perm_token[pos] = token of the pair at pos;
+ * inv_perm[t*k + j] = position of pair (t, j).  If z ([T,L], act) and z_perm
+ * ([T*k, L], act) are both non-NULL, z_perm[pos] = z[perm_token[pos]].
+ * topk_idx rows must hold k distinct experts in [0, E).
+ * Workspace: at least moe_workspace_size(d) bytes. */
+MOE_API moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, const void* z, int32_t* expert_offsets,
+                       int32_t* perm_token, int32_t* inv_perm, void* z_perm, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Routed experts on expert-contiguous latent rows ("K3のエキスパートは896個の小型
+ * LLMではない": the selected experts run on z).  For every expert e and every row
+ * r in expert_offsets[e] .. expert_offsets[e+1]-1:
+ *   h = SiTU-GLU(z_perm[r] . Wg[e]^T, z_perm[r] . Wv[e]^T)   (stored in act type)
+ *   y_perm[r] = h . Wo[e]^T                                    (fp32 [T*k, L])
+ * Only w->Wg, w->Wv, w->Wo are read.  Workspace: moe_workspace_size(d) bytes. */
+MOE_API moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z_perm,
+                          const int32_t* expert_offsets, float* y_perm, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* Weighted combine and RMSNorm ("K3のエキスパートは896個の小型LLMではない":
+ * u = sum p_i E_i(z); y = ... + W_up RMSNorm(u)).
+ *   u[t]   = sum_{j=0}^{k-1} topk_w[t,j] * y_perm[inv_perm[t*k+j]]   (fp32, j ascending)
+ *   n_out[t] = gamma * u[t] / sqrt(mean(u[t]^2) + rms_eps)           (act type [T, L])
+ * u_out ([T, L] fp32) may be NULL. */
+MOE_API moe_status moe_combine(const moe_dims* d, const float* y_perm, const int32_t* inv_perm, const float* topk_w,
+                       const float* gamma, float* u_out, void* n_out, moe_stream_t stream);
+
+/* The whole layer: y[T, H] (type y_out) for x[T, H] (type act).  aux may be
+ * NULL.  Workspace: at least moe_workspace_size(d) bytes. */
+MOE_API moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void* x, void* y, const moe_aux* aux,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Human-readable name of a status. */
+MOE_API const char* moe_status_str(moe_status s);
+
+/* SYNCHRONISING diagnostic: waits for `stream`, then reports and clears the
+ * device-side fault flag of the current device.  *code = 0 when no kernel
+ * recorded a fault; otherwise a nonzero site code, and MOE_ERR_DEVICE is
+ * returned. */
+MOE_API moe_status moe_device_error(int* code, moe_stream_t stream);
+
+/* Number of kernels the last successful moe_layer_forward call on this thread
+ * enqueued (for launch accounting). */
+MOE_API int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -94,10 +94,12 @@ def storage_round(act: str):
 
 
 def bf16_bits_to_f64(a) -> torch.Tensor:
-    """Raw bfloat16 bit patterns (uint16) -> fp64 values (exact)."""
-    a = np.asarray(a)
+    """Raw bfloat16 bit patterns (uint16) -> fp64 values (exact): the 16 bits
+    are the top half of the fp32 with the same value."""
+    a = np.ascontiguousarray(np.asarray(a))
     assert a.dtype == np.uint16
-    return torch.from_numpy((a.astype(np.uint32) << 16).view(np.float32)).to(F64)
+    w = torch.from_numpy(a.view(np.int16)).to(torch.int32).bitwise_left_shift(16)
+    return w.view(torch.float32).to(F64)
 
 
 def f32_to_f64(a) -> torch.Tensor:
@@ -153,11 +155,13 @@ def select_experts(s: torch.Tensor, b: torch.Tensor, k: int):
     """Selection with the frozen bias: key = s + b (fp64); the top k keys are
     chosen; p_j = s_{e_j} / sum_{j'} s_{e_j'} with the UNBIASED scores.
 
+    b is [E] (one bias for all tokens) or [T, E].
     Returns (idx [T,k] int64, p [T,k] fp64, margin [T] fp64) where margin is
     key_(k) - key_(k+1), the gap between the k-th and (k+1)-th largest key
     (+inf when k == E)."""
     s = s.to(F64)
-    key = s + b.to(F64)[None, :]
+    b = b.to(F64)
+    key = s + (b[None, :] if b.dim() == 1 else b)
     idx, sorted_key = _top_k_by_key(key, k)
     s_sel = torch.gather(s, 1, idx)
     p = s_sel / s_sel.sum(dim=1, keepdim=True)

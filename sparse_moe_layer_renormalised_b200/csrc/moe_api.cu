@@ -1,0 +1,617 @@
+// C-ABI entry points of the Stable LatentMoE layer library (see include/moe.h):
+// host-side validation, workspace layout, TMA descriptor encoding and the
+// launch sequence.  Every step of the layer runs in the kernels included here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "combine.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+#include "routing.cuh"
+#include "../../include/moe.h"
+
+namespace moe {
+namespace {
+
+thread_local int g_last_launches = 0;
+
+constexpr size_t kAlign = 256;
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------------------ validation
+bool dims_ok(const moe_dims* d) {
+  if (d == nullptr) return false;
+  if (d->T < 0 || d->H <= 0 || d->L <= 0 || d->E <= 0 || d->k <= 0 || d->I <= 0 || d->S < 0) return false;
+  if (d->S > 0 && d->Is <= 0) return false;
+  if (d->k > d->E || d->k > 32 || d->E > 1024) return false;
+  if (!(d->situ_c > 0.f) || !std::isfinite(d->situ_c) || !(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps))
+    return false;
+  if (d->act != MOE_F32 && d->act != MOE_BF16) return false;
+  if (d->routed != MOE_F32 && d->routed != MOE_BF16 && d->routed != MOE_MXFP4) return false;
+  if (d->y_out != MOE_F32 && d->y_out != d->act) return false;
+  if (d->L % 8 != 0 || d->H % 8 != 0 || d->I % 8 != 0) return false;
+  if (d->S > 0 && d->Is % 8 != 0) return false;
+  if (d->T * static_cast<long long>(d->k) > 0x7fffffffLL) return false;
+  return true;
+}
+
+// Valid dims that this build does not implement.
+bool dims_supported(const moe_dims* d) {
+  if (d->routed != d->act) return false;  // block-scaled routed weights: not in this build
+  if (d->L > 4 * COMBINE_THREADS * 16) return false;
+  if (d->act == MOE_BF16) {
+    if (d->H % 64 || d->L % 64 || d->I % 64) return false;
+    if (d->S > 0 && d->Is % 64) return false;
+    if (d->S > TC_MAX_SEG - 1) return false;
+  } else {
+    if (d->S > SIMT_MAX_SEG - 1) return false;
+  }
+  return true;
+}
+
+moe_status check_dims(const moe_dims* d) {
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  if (!dims_supported(d)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+inline size_t act_bytes(const moe_dims& d) { return d.act == MOE_F32 ? 4 : 2; }
+
+// ------------------------------------------------------------------------------ workspace
+struct WsLayout {
+  size_t scores, topk_idx, topk_w, rank, tile_base, counts, offsets, tile_table, num_m_tiles, perm_token,
+      inv_perm, z, z_perm, h_perm, y_perm, n, h_s, total;
+};
+
+WsLayout ws_layout(const moe_dims& d) {
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, kAlign);
+    return o;
+  };
+  const size_t T = static_cast<size_t>(d.T), R = T * d.k, es = act_bytes(d);
+  const size_t ntok_tiles = cdiv(static_cast<long long>(T), PERM_TILE);
+  const size_t max_m_tiles = cdiv(static_cast<long long>(R), TC_BM) + d.E;
+  w.scores = take(T * d.E * 4);
+  w.topk_idx = take(R * 4);
+  w.topk_w = take(R * 4);
+  w.rank = take(R * 4);
+  w.tile_base = take(ntok_tiles * d.E * 4);
+  w.counts = take(static_cast<size_t>(d.E) * 4);
+  w.offsets = take(static_cast<size_t>(d.E + 1) * 4);
+  w.tile_table = take(max_m_tiles * 16);
+  w.num_m_tiles = take(16);
+  w.perm_token = take(R * 4);
+  w.inv_perm = take(R * 4);
+  w.z = take(T * d.L * es);
+  w.z_perm = take(R * d.L * es);
+  w.h_perm = take(R * d.I * es);
+  w.y_perm = take(R * d.L * 4);
+  w.n = take(T * d.L * es);
+  w.h_s = take(T * static_cast<size_t>(d.S) * d.Is * es);
+  w.total = off;
+  return w;
+}
+
+template <typename P>
+inline P* at(void* base, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(base) + off);
+}
+
+// ------------------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 matrix [rows, cols] with `ld` elements between rows, box 128 rows x 64
+// columns, 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(TC_BK), static_cast<cuuint32_t>(TC_BM)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ------------------------------------------------------------------------------ GEMM launch helpers
+struct Seg {
+  const void* a;  // A segment base (bf16 / f32)
+  long long a_ld;
+  const void* b;  // B segment base
+  long long b_ld;
+  long long b_rows;  // rows of the B view
+  int K;
+};
+
+struct GemmDesc {
+  int epi;
+  bool paired;
+  long long M;  // dense rows, or rows of the permuted buffer when grouped
+  const int4* tile_table;
+  const int* num_m_tiles_dev;
+  int max_m_tiles;  // grouped: upper bound of the table length
+  int N;
+  int b_rows_per_expert;
+  int nseg;
+  Seg seg[TC_MAX_SEG];
+  const void* b_up;  // PAIRED: B rows of the up projection (same view as seg[0].b)
+  void* out;
+  long long ldo;
+  float situ_c;
+  int fault_site;
+};
+
+template <int EPI, bool PAIRED>
+cudaError_t launch_tc_inst(const TcMaps& maps, const TcParams& p, int grid, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<EPI, PAIRED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(TC_SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  tc_gemm_kernel<EPI, PAIRED><<<grid, TC_THREADS, TC_SMEM_BYTES, s>>>(maps, p);
+  return cudaGetLastError();
+}
+
+moe_status run_gemm_tc(const GemmDesc& g, cudaStream_t s) {
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof maps);
+  TcParams p;
+  std::memset(&p, 0, sizeof p);
+  int kb = 0;
+  for (int i = 0; i < g.nseg; ++i) {
+    const Seg& sg = g.seg[i];
+    if (!make_map(&maps.a[i], sg.a, static_cast<uint64_t>(g.M), static_cast<uint64_t>(sg.K),
+                  static_cast<uint64_t>(sg.a_ld)))
+      return MOE_ERR_CUDA;
+    if (!make_map(&maps.b[i], sg.b, static_cast<uint64_t>(sg.b_rows), static_cast<uint64_t>(sg.K),
+                  static_cast<uint64_t>(sg.b_ld)))
+      return MOE_ERR_CUDA;
+    kb += static_cast<int>(cdiv(sg.K, TC_BK));
+    p.seg_end[i] = kb;
+  }
+  if (g.paired) {
+    if (!make_map(&maps.b[1], g.b_up, static_cast<uint64_t>(g.seg[0].b_rows), static_cast<uint64_t>(g.seg[0].K),
+                  static_cast<uint64_t>(g.seg[0].b_ld)))
+      return MOE_ERR_CUDA;
+  }
+  for (int i = g.nseg; i < TC_MAX_SEG; ++i) p.seg_end[i] = kb;
+  p.num_k_blocks = kb;
+  p.M = static_cast<int>(g.M);
+  p.num_m_tiles = static_cast<int>(cdiv(g.M, TC_BM));
+  p.tile_table = g.tile_table;
+  p.num_m_tiles_dev = g.num_m_tiles_dev;
+  p.N = g.N;
+  p.n_tiles = static_cast<int>(cdiv(g.N, g.paired ? TC_BN / 2 : TC_BN));
+  p.b_rows_per_expert = g.b_rows_per_expert;
+  p.out = g.out;
+  p.ldo = g.ldo;
+  p.situ_c = g.situ_c;
+  p.fault_site = g.fault_site;
+  const long long m_tiles = g.tile_table ? g.max_m_tiles : p.num_m_tiles;
+  long long work = m_tiles * p.n_tiles;
+  const int sms = num_sms();
+  const int grid = static_cast<int>(work < sms ? (work > 0 ? work : 1) : sms);
+  cudaError_t e;
+  if (g.paired)
+    e = launch_tc_inst<kEpiSituBF16, true>(maps, p, grid, s);
+  else if (g.epi == kEpiF32)
+    e = launch_tc_inst<kEpiF32, false>(maps, p, grid, s);
+  else if (g.epi == kEpiBF16)
+    e = launch_tc_inst<kEpiBF16, false>(maps, p, grid, s);
+  else
+    e = launch_tc_inst<kEpiSigmoidF32, false>(maps, p, grid, s);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status run_gemm_simt(const GemmDesc& g, cudaStream_t s) {
+  SimtParams p;
+  std::memset(&p, 0, sizeof p);
+  for (int i = 0; i < g.nseg; ++i) {
+    p.A[i] = static_cast<const float*>(g.seg[i].a);
+    p.lda[i] = g.seg[i].a_ld;
+    p.B[i] = static_cast<const float*>(g.seg[i].b);
+    p.ldb[i] = g.seg[i].b_ld;
+    p.seg_k[i] = g.seg[i].K;
+  }
+  p.nseg = g.nseg;
+  if (g.paired) {
+    p.B[1] = static_cast<const float*>(g.b_up);
+    p.ldb[1] = g.seg[0].b_ld;
+  }
+  p.M = static_cast<int>(g.M);
+  p.tile_table = g.tile_table;
+  p.num_m_tiles_dev = g.num_m_tiles_dev;
+  p.N = g.N;
+  p.b_rows_per_expert = g.b_rows_per_expert;
+  p.out = g.out;
+  p.ldo = g.ldo;
+  p.situ_c = g.situ_c;
+  const long long rows = g.tile_table ? static_cast<long long>(g.max_m_tiles) * 4 : cdiv(g.M, 32);
+  dim3 grid(static_cast<unsigned>(cdiv(g.N, 32)), static_cast<unsigned>(rows));
+  if (g.paired)
+    simt_gemm_kernel<kEpiSituBF16, true><<<grid, 256, 0, s>>>(p);
+  else if (g.epi == kEpiSigmoidF32)
+    simt_gemm_kernel<kEpiSigmoidF32, false><<<grid, 256, 0, s>>>(p);
+  else
+    simt_gemm_kernel<kEpiF32, false><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status run_gemm(const moe_dims& d, const GemmDesc& g, cudaStream_t s) {
+  ++g_last_launches;
+  return d.act == MOE_BF16 ? run_gemm_tc(g, s) : run_gemm_simt(g, s);
+}
+
+// ------------------------------------------------------------------------------ stages
+moe_status stage_router(const moe_dims& d, const void* x, const void* Wr, float* scores, cudaStream_t s) {
+  GemmDesc g{};
+  g.epi = kEpiSigmoidF32;
+  g.M = d.T;
+  g.N = d.E;
+  g.nseg = 1;
+  g.seg[0] = Seg{x, d.H, Wr, d.H, d.E, d.H};
+  g.out = scores;
+  g.ldo = d.E;
+  g.situ_c = d.situ_c;
+  g.fault_site = 100;
+  return run_gemm(d, g, s);
+}
+
+moe_status stage_topk(const moe_dims& d, const float* scores, const float* bias, int32_t* idx, float* w,
+                      cudaStream_t s) {
+  const unsigned blocks = static_cast<unsigned>(cdiv(d.T, TOPK_WARPS));
+  topk_renorm_kernel<<<blocks, TOPK_WARPS * 32, 0, s>>>(scores, bias, d.T, d.E, d.k, idx, w);
+  ++g_last_launches;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status stage_dense(const moe_dims& d, int epi, const void* A, long long lda, const void* B, long long N,
+                       int K, void* out, long long ldo, int site, cudaStream_t s) {
+  GemmDesc g{};
+  g.epi = epi;
+  g.M = d.T;
+  g.N = static_cast<int>(N);
+  g.nseg = 1;
+  g.seg[0] = Seg{A, lda, B, K, N, K};
+  g.out = out;
+  g.ldo = ldo;
+  g.situ_c = d.situ_c;
+  g.fault_site = site;
+  return run_gemm(d, g, s);
+}
+
+moe_status stage_shared_gate_up(const moe_dims& d, const moe_weights& w, const void* x, void* h_s, cudaStream_t s) {
+  GemmDesc g{};
+  g.epi = kEpiSituBF16;
+  g.paired = true;
+  g.M = d.T;
+  g.N = d.S * d.Is;
+  g.nseg = 1;
+  g.seg[0] = Seg{x, d.H, w.Wsg, d.H, static_cast<long long>(d.S) * d.Is, d.H};
+  g.b_up = w.Wsv;
+  g.out = h_s;
+  g.ldo = static_cast<long long>(d.S) * d.Is;
+  g.situ_c = d.situ_c;
+  g.fault_site = 130;
+  return run_gemm(d, g, s);
+}
+
+moe_status stage_permute(const moe_dims& d, const int32_t* idx, const WsLayout& L, void* ws, int32_t* offsets,
+                         int32_t* counts_out, int32_t* perm_token, int32_t* inv_perm, cudaStream_t s) {
+  const long long ntiles = cdiv(d.T, PERM_TILE);
+  int32_t* tile_base = at<int32_t>(ws, L.tile_base);
+  int32_t* rank = at<int32_t>(ws, L.rank);
+  perm_rank_kernel<<<static_cast<unsigned>(ntiles), PERM_TILE, static_cast<size_t>(d.E) * 16, s>>>(
+      idx, d.T, d.E, d.k, tile_base, rank);
+  perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d.E, counts_out, offsets,
+                                      at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles));
+  const long long pairs = d.T * d.k;
+  perm_scatter_kernel<<<static_cast<unsigned>(cdiv(pairs, 256)), 256, 0, s>>>(idx, d.T, d.E, d.k, tile_base, rank,
+                                                                              offsets, perm_token, inv_perm);
+  g_last_launches += 3;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status stage_gather(const moe_dims& d, const void* z, void* z_perm, const int32_t* perm_token,
+                        const int32_t* n_rows, cudaStream_t s) {
+  const long long R = d.T * d.k;
+  const int row_vecs = static_cast<int>(static_cast<size_t>(d.L) * act_bytes(d) / 16);
+  gather_rows_kernel<<<static_cast<unsigned>(cdiv(R, GATHER_WARPS)), GATHER_WARPS * 32, 0, s>>>(
+      static_cast<const uint4*>(z), static_cast<uint4*>(z_perm), perm_token, n_rows, d.T, row_vecs);
+  ++g_last_launches;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status stage_experts(const moe_dims& d, const moe_weights& w, const void* z_perm, const int4* tile_table,
+                         const int32_t* num_m_tiles, void* h_perm, float* y_perm, cudaStream_t s) {
+  const long long R = d.T * d.k;
+  const int max_m_tiles = static_cast<int>(cdiv(R, TC_BM) + d.E);
+  GemmDesc g{};
+  g.epi = kEpiSituBF16;
+  g.paired = true;
+  g.M = R;
+  g.tile_table = tile_table;
+  g.num_m_tiles_dev = num_m_tiles;
+  g.max_m_tiles = max_m_tiles;
+  g.N = d.I;
+  g.b_rows_per_expert = d.I;
+  g.nseg = 1;
+  g.seg[0] = Seg{z_perm, d.L, w.Wg, d.L, static_cast<long long>(d.E) * d.I, d.L};
+  g.b_up = w.Wv;
+  g.out = h_perm;
+  g.ldo = d.I;
+  g.situ_c = d.situ_c;
+  g.fault_site = 140;
+  moe_status st = run_gemm(d, g, s);
+  if (st != MOE_OK) return st;
+  GemmDesc g2{};
+  g2.epi = kEpiF32;
+  g2.M = R;
+  g2.tile_table = tile_table;
+  g2.num_m_tiles_dev = num_m_tiles;
+  g2.max_m_tiles = max_m_tiles;
+  g2.N = d.L;
+  g2.b_rows_per_expert = d.L;
+  g2.nseg = 1;
+  g2.seg[0] = Seg{h_perm, d.I, w.Wo, d.I, static_cast<long long>(d.E) * d.L, d.I};
+  g2.out = y_perm;
+  g2.ldo = d.L;
+  g2.situ_c = d.situ_c;
+  g2.fault_site = 150;
+  return run_gemm(d, g2, s);
+}
+
+template <typename OutT>
+cudaError_t launch_combine_t(const moe_dims& d, const float* y_perm, const int32_t* inv_perm, const float* w,
+                             const float* gamma, float* u, OutT* n, cudaStream_t s) {
+  const int nv = d.L / 4;
+  const unsigned grid = static_cast<unsigned>(d.T);
+  const float eps = d.rms_eps;
+  if (nv <= COMBINE_THREADS * 1)
+    combine_rmsnorm_kernel<OutT, 1><<<grid, COMBINE_THREADS, 0, s>>>(y_perm, inv_perm, w, gamma, d.k, d.L, eps, u, n);
+  else if (nv <= COMBINE_THREADS * 2)
+    combine_rmsnorm_kernel<OutT, 2><<<grid, COMBINE_THREADS, 0, s>>>(y_perm, inv_perm, w, gamma, d.k, d.L, eps, u, n);
+  else if (nv <= COMBINE_THREADS * 4)
+    combine_rmsnorm_kernel<OutT, 4><<<grid, COMBINE_THREADS, 0, s>>>(y_perm, inv_perm, w, gamma, d.k, d.L, eps, u, n);
+  else if (nv <= COMBINE_THREADS * 7)
+    combine_rmsnorm_kernel<OutT, 7><<<grid, COMBINE_THREADS, 0, s>>>(y_perm, inv_perm, w, gamma, d.k, d.L, eps, u, n);
+  else if (nv <= COMBINE_THREADS * 8)
+    combine_rmsnorm_kernel<OutT, 8><<<grid, COMBINE_THREADS, 0, s>>>(y_perm, inv_perm, w, gamma, d.k, d.L, eps, u, n);
+  else
+    combine_rmsnorm_kernel<OutT, 16><<<grid, COMBINE_THREADS, 0, s>>>(y_perm, inv_perm, w, gamma, d.k, d.L, eps, u, n);
+  return cudaGetLastError();
+}
+
+moe_status stage_combine(const moe_dims& d, const float* y_perm, const int32_t* inv_perm, const float* w,
+                         const float* gamma, float* u, void* n, cudaStream_t s) {
+  ++g_last_launches;
+  cudaError_t e = d.act == MOE_BF16
+                      ? launch_combine_t<__nv_bfloat16>(d, y_perm, inv_perm, w, gamma, u, static_cast<__nv_bfloat16*>(n), s)
+                      : launch_combine_t<float>(d, y_perm, inv_perm, w, gamma, u, static_cast<float*>(n), s);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status stage_output(const moe_dims& d, const moe_weights& w, const void* h_s, const void* n, void* y,
+                        cudaStream_t s) {
+  const size_t es = act_bytes(d);
+  GemmDesc g{};
+  g.epi = (d.y_out == MOE_F32) ? kEpiF32 : kEpiBF16;
+  g.M = d.T;
+  g.N = d.H;
+  g.nseg = d.S + 1;
+  for (int i = 0; i < d.S; ++i) {
+    const uint8_t* a = static_cast<const uint8_t*>(h_s) + static_cast<size_t>(i) * d.Is * es;
+    const uint8_t* b = static_cast<const uint8_t*>(w.Wso) + static_cast<size_t>(i) * d.H * d.Is * es;
+    g.seg[i] = Seg{a, static_cast<long long>(d.S) * d.Is, b, d.Is, d.H, d.Is};
+  }
+  g.seg[d.S] = Seg{n, d.L, w.Wup, d.L, d.H, d.L};
+  g.out = y;
+  g.ldo = d.H;
+  g.situ_c = d.situ_c;
+  g.fault_site = 160;
+  return run_gemm(d, g, s);
+}
+
+bool ws_ok(const moe_dims& d, const void* ws, size_t ws_bytes) {
+  return ws != nullptr && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0 && ws_bytes >= ws_layout(d).total;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims* d) {
+  if (!dims_ok(d)) return 0;
+  return ws_layout(*d).total;
+}
+
+const char* moe_status_str(moe_status s) {
+  switch (s) {
+    case MOE_OK:
+      return "MOE_OK";
+    case MOE_ERR_INVALID_ARG:
+      return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED:
+      return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA:
+      return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE:
+      return "MOE_ERR_DEVICE";
+  }
+  return "unknown moe_status";
+}
+
+int moe_last_launch_count(void) { return g_last_launches; }
+
+moe_status moe_router_topk(const moe_dims* d, const void* x, const void* Wr, const float* bias, float* scores,
+                           int from_scores, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (!aligned16(scores) || scores == nullptr || bias == nullptr || topk_idx == nullptr || topk_w == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!from_scores && (x == nullptr || Wr == nullptr || !aligned16(x) || !aligned16(Wr))) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!from_scores) {
+    st = stage_router(*d, x, Wr, scores, s);
+    if (st != MOE_OK) return st;
+  }
+  return stage_topk(*d, scores, bias, topk_idx, topk_w, s);
+}
+
+moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, const void* z, int32_t* expert_offsets,
+                       int32_t* perm_token, int32_t* inv_perm, void* z_perm, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (topk_idx == nullptr || expert_offsets == nullptr || perm_token == nullptr || inv_perm == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((z == nullptr) != (z_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (z != nullptr && (!aligned16(z) || !aligned16(z_perm))) return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(*d, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*d);
+  st = stage_permute(*d, topk_idx, L, ws, expert_offsets, nullptr, perm_token, inv_perm, s);
+  if (st != MOE_OK) return st;
+  if (z != nullptr) st = stage_gather(*d, z, z_perm, perm_token, expert_offsets + d->E, s);
+  return st;
+}
+
+moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z_perm,
+                          const int32_t* expert_offsets, float* y_perm, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (w == nullptr || z_perm == nullptr || expert_offsets == nullptr || y_perm == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->Wg) || !aligned16(w->Wv) || !aligned16(w->Wo) || w->Wg == nullptr || w->Wv == nullptr ||
+      w->Wo == nullptr || !aligned16(z_perm) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(*d, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*d);
+  tile_table_kernel<<<1, 1024, 0, s>>>(expert_offsets, d->E, d->T * d->k, at<int4>(ws, L.tile_table),
+                                       at<int32_t>(ws, L.num_m_tiles));
+  ++g_last_launches;
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  return stage_experts(*d, *w, z_perm, at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles),
+                       at<void>(ws, L.h_perm), y_perm, s);
+}
+
+moe_status moe_combine(const moe_dims* d, const float* y_perm, const int32_t* inv_perm, const float* topk_w,
+                       const float* gamma, float* u_out, void* n_out, moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (y_perm == nullptr || inv_perm == nullptr || topk_w == nullptr || gamma == nullptr || n_out == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(gamma) || !aligned16(n_out) || !aligned16(u_out)) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  return stage_combine(*d, y_perm, inv_perm, topk_w, gamma, u_out, n_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void* x, void* y, const moe_aux* aux,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (w == nullptr || x == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* need[] = {w->Wr, w->bias, w->Wdown, w->Wup, w->gamma, w->Wg, w->Wv, w->Wo, x, y};
+  for (const void* p : need)
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (d->S > 0 && (w->Wsg == nullptr || w->Wsv == nullptr || w->Wso == nullptr || !aligned16(w->Wsg) ||
+                   !aligned16(w->Wsv) || !aligned16(w->Wso)))
+    return MOE_ERR_INVALID_ARG;
+  if (w->Sg != nullptr || w->Sv != nullptr || w->So != nullptr) return MOE_ERR_UNSUPPORTED;
+  moe_aux a{};
+  if (aux != nullptr) a = *aux;
+  const void* auxp[] = {a.scores, a.topk_idx, a.topk_w, a.expert_offsets, a.u, a.n, a.z};
+  for (const void* p : auxp)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(*d, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*d);
+  float* scores = a.scores ? a.scores : at<float>(ws, L.scores);
+  int32_t* idx = a.topk_idx ? a.topk_idx : at<int32_t>(ws, L.topk_idx);
+  float* tw = a.topk_w ? a.topk_w : at<float>(ws, L.topk_w);
+  int32_t* offsets = a.expert_offsets ? a.expert_offsets : at<int32_t>(ws, L.offsets);
+  void* z = a.z ? a.z : at<void>(ws, L.z);
+  void* n = a.n ? a.n : at<void>(ws, L.n);
+  void* h_s = at<void>(ws, L.h_s);
+  int32_t* perm_token = at<int32_t>(ws, L.perm_token);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+
+  // x-side: router scores, latent projection, shared experts' gate/up
+  if ((st = stage_router(*d, x, w->Wr, scores, s)) != MOE_OK) return st;
+  if ((st = stage_topk(*d, scores, w->bias, idx, tw, s)) != MOE_OK) return st;
+  if ((st = stage_dense(*d, d->act == MOE_BF16 ? kEpiBF16 : kEpiF32, x, d->H, w->Wdown, d->L, d->H, z, d->L, 120,
+                        s)) != MOE_OK)
+    return st;
+  if (d->S > 0 && (st = stage_shared_gate_up(*d, *w, x, h_s, s)) != MOE_OK) return st;
+  // dispatch
+  if ((st = stage_permute(*d, idx, L, ws, offsets, nullptr, perm_token, inv_perm, s)) != MOE_OK) return st;
+  if ((st = stage_gather(*d, z, at<void>(ws, L.z_perm), perm_token, offsets + d->E, s)) != MOE_OK) return st;
+  // routed experts
+  if ((st = stage_experts(*d, *w, at<void>(ws, L.z_perm), at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles),
+                          at<void>(ws, L.h_perm), at<float>(ws, L.y_perm), s)) != MOE_OK)
+    return st;
+  // combine + RMSNorm, then [shared | W_up] output projection
+  if ((st = stage_combine(*d, at<float>(ws, L.y_perm), inv_perm, tw, w->gamma, a.u, n, s)) != MOE_OK) return st;
+  return stage_output(*d, *w, h_s, n, y, s);
+}
+
+moe_status moe_device_error(int* code, moe_stream_t stream) {
+  if (code == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_moe_fault, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  *code = v;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_moe_fault, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_DEVICE;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -10,7 +10,19 @@ if ROOT not in sys.path:
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+def _build_libraries():
+    """Build the CUDA library and the generator library in-tree if missing or
+    stale (nvcc cross-compiles for sm_100a without a GPU)."""
+    import gen.build
+    import sparse_moe_layer_renormalised_b200.build as b
+
+    b.build()
+    if not os.path.exists(os.path.join(ROOT, "gen", "libmoegen.so")):
+        gen.build.build()
+
+
 def pytest_configure(config):
+    _build_libraries()
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (sm_100a); run with -m gpu")
     config.addinivalue_line("markers", "slow: long-running check at the full K3 sizes")
 

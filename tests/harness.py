@@ -1,0 +1,166 @@
+"""Helpers shared by the GPU parity tests, smoke() and bench.py: device layers
+from the seeded generator, oracle references, and the parity metrics."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import gen
+import oracle
+import sparse_moe_layer_renormalised_b200 as moe
+from oracle import inputs as oin
+
+F64 = torch.float64
+
+# Tolerances (max|y - y_ref| / rms(y_ref)) stated for the layer output.
+TOL_BF16 = 1e-2
+TOL_MXFP4 = 3e-2
+TOL_F32 = 1e-4
+NEAR_TIE = 1e-4  # key margin below which an index-set difference is allowed
+
+
+def dims_for(cfg, T=None, y_out="f32") -> moe.Dims:
+    return moe.Dims(T=cfg.T if T is None else T, H=cfg.H, L=cfg.L, E=cfg.E, k=cfg.k, I=cfg.I, S=cfg.S, Is=cfg.Is,
+                    act=cfg.act, routed=cfg.routed, y_out=y_out if cfg.act == "bf16" else "f32",
+                    situ_c=cfg.situ_c, rms_eps=cfg.rms_eps)
+
+
+def make_device_layer(cfg, y_out="f32", max_tokens=None, weights=None):
+    """(MoeLayer, input tensors dict) with every input generated on the device."""
+    w = gen.device_layer(cfg, "cuda") if weights is None else weights
+    layer = moe.MoeLayer(dims_for(cfg, y_out=y_out), {k: v for k, v in w.items() if k != "x"}, max_tokens=max_tokens)
+    return layer, w
+
+
+def run_layer(layer, x, want_aux=True):
+    T = x.shape[0]
+    d = layer.dims
+    dev = x.device
+    act_dt = torch.bfloat16 if d.act == "bf16" else torch.float32
+    aux = None
+    if want_aux:
+        aux = {
+            "scores": torch.empty(T, d.E, dtype=torch.float32, device=dev),
+            "topk_idx": torch.empty(T, d.k, dtype=torch.int32, device=dev),
+            "topk_w": torch.empty(T, d.k, dtype=torch.float32, device=dev),
+            "expert_offsets": torch.empty(d.E + 1, dtype=torch.int32, device=dev),
+            "u": torch.empty(T, d.L, dtype=torch.float32, device=dev),
+            "n": torch.empty(T, d.L, dtype=act_dt, device=dev),
+            "z": torch.empty(T, d.L, dtype=act_dt, device=dev),
+        }
+    y = layer.forward(x, aux=aux)
+    torch.cuda.synchronize()
+    st, code = moe.moe_device_error()
+    assert st == moe.MOE_OK and code == 0, f"device fault {code}"
+    return y, aux
+
+
+def parity(a: torch.Tensor, ref: torch.Tensor) -> float:
+    a = a.to(F64).cpu()
+    ref = ref.to(F64).cpu()
+    rms = torch.sqrt((ref * ref).mean()).item()
+    return (a - ref).abs().max().item() / rms
+
+
+_WCACHE: dict = {}
+
+
+def _dense(cfg):
+    key = (cfg.name, cfg.H, cfg.L, cfg.E, cfg.I, cfg.S, cfg.Is, cfg.act, cfg.bias, cfg.gamma, cfg.seed)
+    if key not in _WCACHE:
+        _WCACHE.clear()
+        _WCACHE[key] = oin.dense_weights(cfg)
+    return _WCACHE[key]
+
+
+def small_enough_for_memory(cfg) -> bool:
+    return cfg.E * cfg.I * cfg.L * 3 <= 200_000_000
+
+
+def oracle_forward(cfg, tokens, forced_idx=None) -> dict:
+    """Oracle outputs for the given token rows of cfg's synthetic input."""
+    tokens = np.asarray(tokens)
+    x = oin.x_rows(cfg, tokens)
+    if small_enough_for_memory(cfg):
+        key = ("all", cfg)
+        if key not in _WCACHE:
+            _WCACHE.clear()
+            _WCACHE[key] = oin.all_weights(cfg)
+        return oracle.layer_forward(cfg, _WCACHE[key], x, forced_idx=forced_idx)
+    dense = _dense(cfg)
+    return oracle.layer_forward_streamed(cfg, dense, x, lambda e: oin.expert_weights(cfg, e), forced_idx=forced_idx)
+
+
+def compare_layer(cfg, tokens, y_gpu, aux, tol, ref=None) -> dict:
+    """Parity of the device layer on the sampled tokens against the oracle.
+
+    Index sets must match except for tokens whose oracle key margin (k-th
+    minus (k+1)-th largest key) is below NEAR_TIE; those are counted and
+    their outputs are checked against the oracle forced to the device's
+    choice.  Returns the metrics; asserts the bars."""
+    tokens = np.asarray(tokens)
+    ref = oracle_forward(cfg, tokens) if ref is None else ref
+    idx_gpu = aux["topk_idx"].cpu().to(torch.int64)[torch.as_tensor(tokens)]
+    set_gpu = torch.sort(idx_gpu, dim=1).values
+    set_ref = torch.sort(ref["idx"], dim=1).values
+    differ = (set_gpu != set_ref).any(dim=1)
+    n_diff = int(differ.sum())
+    near = ref["margin"] < NEAR_TIE
+    assert bool((~differ | near).all()), (
+        f"{int((differ & ~near).sum())} tokens choose different experts with margin >= {NEAR_TIE}")
+    y_ref = ref["y"].clone()
+    u_ref, n_ref = ref["u"].clone(), ref["n"].clone()
+    if n_diff:
+        forced = ref["idx"].clone()
+        forced[differ] = idx_gpu[differ]
+        rf = oracle_forward(cfg, tokens, forced_idx=forced)
+        y_ref, u_ref, n_ref = rf["y"], rf["u"], rf["n"]
+    sel = torch.as_tensor(tokens)
+    m = {
+        "tokens_checked": len(tokens),
+        "index_set_differences": n_diff,
+        "near_tie_tokens": int(near.sum()),
+        "y": parity(y_gpu.cpu()[sel], y_ref),
+        "u": parity(aux["u"].cpu()[sel], u_ref),
+        "n": parity(aux["n"].cpu()[sel], n_ref),
+    }
+    # mixture weights: unbiased scores renormalised over the chosen experts
+    p_gpu = aux["topk_w"].cpu().to(F64)[sel]
+    assert torch.allclose(p_gpu.sum(dim=1), torch.ones(len(tokens), dtype=F64), atol=1e-5)
+    same = ~differ
+    if same.any():
+        m["p"] = (p_gpu[same] - ref["p"][same]).abs().max().item()
+    for key in ("y", "u"):
+        assert m[key] <= tol, f"{key}: max|d|/rms = {m[key]:.3g} > {tol}"
+    # The RMSNorm step: n must be RMSNorm of the device's own u, rounded to the
+    # activation type, to within one rounding step of that type.  (Against the
+    # oracle's n, per-token normalisation magnifies u's error in tokens whose
+    # u is small, so that comparison is reported, not gated.)
+    u_dev = aux["u"].cpu().to(F64)[sel]
+    gamma = torch.from_numpy(gen.gamma(cfg)).to(F64)
+    n_from_u = oracle.storage_round(cfg.act)(oracle.rms_norm(u_dev, gamma, cfg.rms_eps))
+    m["n_steps"] = storage_steps(aux["n"].cpu()[sel], n_from_u, cfg.act)
+    assert m["n_steps"] <= 1.0 + 1e-6, f"n differs from RMSNorm(u) by {m['n_steps']:.3g} storage steps"
+    return m
+
+
+def storage_steps(a: torch.Tensor, ref: torch.Tensor, act: str) -> float:
+    """Largest |a - ref| in units of the spacing of the storage type at |ref|
+    (bf16: 2^-7 |ref| bounds one step; fp32: 2^-23 |ref|), with a floor of
+    1e-3 rms(ref) for values near zero."""
+    a = a.to(F64)
+    ref = ref.to(F64)
+    rel = 2.0**-7 if act == "bf16" else 2.0**-23
+    rms = torch.sqrt((ref * ref).mean())
+    step = torch.clamp(ref.abs() * rel, min=float(1e-3 * rms))
+    return float(((a - ref).abs() / step).max())
+
+
+def moe_inputs_rows(cfg, tokens, device="cuda"):
+    """x rows as a device tensor in the activation type (for sub-batch calls)."""
+    a = gen.host_rows(cfg, "x", np.asarray(tokens))
+    if cfg.act == "bf16":
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(a).to(device)

@@ -1,0 +1,112 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_moe_layer_renormalised_b200 as moe
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)
+
+
+def _dims(**kw):
+    base = dict(T=128, H=2048, L=1024, E=128, k=8, I=768, S=2, Is=1024)
+    base.update(kw)
+    return moe.Dims(**base)
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) == 9
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(moe.EXPORTED)
+
+
+def test_status_strings():
+    assert moe.moe_status_str(0) == "MOE_OK"
+    assert moe.moe_status_str(2) == "MOE_ERR_UNSUPPORTED"
+
+
+def test_workspace_size():
+    assert moe.moe_workspace_size(_dims(k=200)) == 0
+    a = moe.moe_workspace_size(_dims(T=100))
+    b = moe.moe_workspace_size(_dims(T=1000))
+    assert 0 < a < b
+    k3 = moe.moe_workspace_size(_dims(T=16384, H=7168, L=3584, E=896, k=16, I=3072, S=2, Is=3072))
+    # dominated by the permuted latent rows (bf16), expert h (bf16) and y_perm (fp32)
+    R = 16384 * 16
+    assert k3 >= R * (3584 * 2 + 3072 * 2 + 3584 * 4)
+
+
+FAKE = 1 << 20  # an aligned address; never dereferenced because validation fails first
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=129, E=128), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=33, E=128), moe.MOE_ERR_INVALID_ARG),
+    (dict(E=1025), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(L=1020), moe.MOE_ERR_INVALID_ARG),
+    (dict(situ_c=0.0), moe.MOE_ERR_INVALID_ARG),
+    (dict(y_out="mxfp4"), moe.MOE_ERR_INVALID_ARG),
+    (dict(routed="mxfp4"), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=2056), moe.MOE_ERR_UNSUPPORTED),
+    (dict(S=4), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_invalid_dims_rejected(kw, status):
+    d = _dims(**kw)
+    w = moe.make_weights(**{f: FAKE for f in ("Wr", "bias", "Wdown", "Wup", "gamma", "Wg", "Wv", "Wo", "Wsg", "Wsv",
+                                                "Wso")})
+    assert moe.moe_layer_forward(d, w, FAKE, FAKE, None, FAKE, 1 << 40, 0) == status
+
+
+def test_bad_pointers_rejected():
+    d = _dims()
+    full = {f: FAKE for f in ("Wr", "bias", "Wdown", "Wup", "gamma", "Wg", "Wv", "Wo", "Wsg", "Wsv", "Wso")}
+    ws = moe.moe_workspace_size(d)
+    for f in full:
+        w = moe.make_weights(**{**full, f: None})
+        assert moe.moe_layer_forward(d, w, FAKE, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG, f
+        w = moe.make_weights(**{**full, f: FAKE + 8})
+        assert moe.moe_layer_forward(d, w, FAKE, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG, f
+    w = moe.make_weights(**full)
+    assert moe.moe_layer_forward(d, w, None, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_layer_forward(d, w, FAKE, FAKE, None, FAKE + 16, ws, 0) == moe.MOE_ERR_INVALID_ARG  # ws alignment
+    assert moe.moe_layer_forward(d, w, FAKE, FAKE, None, FAKE, ws - 1, 0) == moe.MOE_ERR_INVALID_ARG  # ws size
+    aux = moe.make_aux(u=FAKE + 4)
+    assert moe.moe_layer_forward(d, w, FAKE, FAKE, aux, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
+    w_scaled = moe.make_weights(**{**full, "Sg": FAKE})
+    assert moe.moe_layer_forward(d, w_scaled, FAKE, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_stage_entry_points_validate():
+    d = _dims()
+    ws = moe.moe_workspace_size(d)
+    assert moe.moe_router_topk(d, None, None, FAKE, FAKE, 0, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_router_topk(d, None, None, None, FAKE, 1, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_permute(d, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_permute(d, FAKE, None, FAKE, FAKE, FAKE, None, FAKE, 10, 0) == moe.MOE_ERR_INVALID_ARG
+    w = moe.make_weights(Wg=FAKE, Wv=FAKE)
+    assert moe.moe_expert_ffn(d, w, FAKE, FAKE, FAKE, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_combine(d, FAKE, FAKE, FAKE, None, None, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_combine(d, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import sparse_moe_layer_renormalised_b200._binding as b
+
+    monkeypatch.setattr(b, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(b, "_lib", None)
+    with pytest.raises(moe.MoeLibraryMissing):
+        b.lib()
