@@ -111,6 +111,19 @@ typedef struct {
   const void* Wso;     /* [S, H, Is] shared down projections */
 } moe_weights;
 
+/* Stages of moe_layer_forward, in launch order (for moe_aux.stage_events). */
+#define MOE_STAGE_ROUTER 0         /* router GEMM + sigmoid -> scores */
+#define MOE_STAGE_TOPK 1           /* bias + top-k + renormalisation */
+#define MOE_STAGE_LATENT_DOWN 2    /* z = W_down x */
+#define MOE_STAGE_SHARED_GATE_UP 3 /* shared experts' SiTU-GLU(W_sg x, W_sv x) */
+#define MOE_STAGE_PERMUTE 4        /* expert-major order of the (token, slot) pairs */
+#define MOE_STAGE_GATHER 5         /* z rows into expert-major order */
+#define MOE_STAGE_EXPERT_GATE_UP 6 /* routed experts' SiTU-GLU(W_g z, W_v z) */
+#define MOE_STAGE_EXPERT_DOWN 7    /* routed experts' W_o h */
+#define MOE_STAGE_COMBINE 8        /* weighted combine + RMSNorm */
+#define MOE_STAGE_OUTPUT 9         /* y = [h_shared | n] . [W_so | W_up]^T */
+#define MOE_NUM_STAGES 10
+
 /* Optional extra outputs of moe_layer_forward; every field may be NULL.
  * Given buffers receive the intermediate directly (no extra pass). */
 typedef struct {
@@ -121,6 +134,10 @@ typedef struct {
   float* u;                 /* [T, L]  fp32 mixture before RMSNorm */
   void* n;                  /* [T, L]  RMSNorm(u) in the activation type */
   void* z;                  /* [T, L]  W_down x in the activation type */
+  /* Host array of 2 * MOE_NUM_STAGES caller-created CUDA events (cudaEvent_t),
+   * or NULL.  Event 2i is recorded on `stream` before stage i and event 2i+1
+   * after it, so cudaEventElapsedTime gives each stage's device time. */
+  void* const* stage_events;
 } moe_aux;
 
 /* Bytes of workspace moe_layer_forward needs for these dims (also enough for

@@ -13,6 +13,8 @@ from ._binding import (  # noqa: F401
     MOE_ERR_UNSUPPORTED,
     MOE_F32,
     MOE_MXFP4,
+    MOE_NUM_STAGES,
+    STAGE_NAMES,
     MOE_OK,
     Dims,
     MoeLibraryMissing,

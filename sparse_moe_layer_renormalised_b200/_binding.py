@@ -59,8 +59,13 @@ class moe_weights(ctypes.Structure):
     _fields_ = [(f, ctypes.c_void_p) for f in _WEIGHT_FIELDS]
 
 
+MOE_NUM_STAGES = 10
+STAGE_NAMES = ("router", "topk", "latent_down", "shared_gate_up", "permute", "gather", "expert_gate_up",
+               "expert_down", "combine", "output")
+
+
 class moe_aux(ctypes.Structure):
-    _fields_ = [(f, ctypes.c_void_p) for f in _AUX_FIELDS]
+    _fields_ = [(f, ctypes.c_void_p) for f in _AUX_FIELDS] + [("stage_events", ctypes.POINTER(ctypes.c_void_p))]
 
 
 class MoeLibraryMissing(RuntimeError):
@@ -151,11 +156,22 @@ def make_weights(**tensors) -> moe_weights:
     return moe_weights(*[_ptr(tensors.get(f)) for f in _WEIGHT_FIELDS])
 
 
-def make_aux(**tensors) -> moe_aux:
+def make_aux(stage_events=None, **tensors) -> moe_aux:
+    """moe_aux from keyword tensors; stage_events: 2 * MOE_NUM_STAGES CUDA
+    events (torch.cuda.Event, already recorded once so they exist, or raw
+    handles)."""
     unknown = set(tensors) - set(_AUX_FIELDS)
     if unknown:
         raise KeyError(f"unknown aux fields {sorted(unknown)}")
-    return moe_aux(*[_ptr(tensors.get(f)) for f in _AUX_FIELDS])
+    a = moe_aux(*[_ptr(tensors.get(f)) for f in _AUX_FIELDS])
+    if stage_events is not None:
+        if len(stage_events) != 2 * MOE_NUM_STAGES:
+            raise ValueError("need 2 * MOE_NUM_STAGES events")
+        arr = (ctypes.c_void_p * len(stage_events))(
+            *[e if isinstance(e, int) else e.cuda_event for e in stage_events])
+        a._events_keepalive = arr
+        a.stage_events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    return a
 
 
 # ------------------------------------------------------------------------------------ the ABI

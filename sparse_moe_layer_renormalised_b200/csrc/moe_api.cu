@@ -353,17 +353,16 @@ moe_status stage_gather(const moe_dims& d, const void* z, void* z_perm, const in
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status stage_experts(const moe_dims& d, const moe_weights& w, const void* z_perm, const int4* tile_table,
-                         const int32_t* num_m_tiles, void* h_perm, float* y_perm, cudaStream_t s) {
+moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const void* z_perm,
+                                const int4* tile_table, const int32_t* num_m_tiles, void* h_perm, cudaStream_t s) {
   const long long R = d.T * d.k;
-  const int max_m_tiles = static_cast<int>(cdiv(R, TC_BM) + d.E);
   GemmDesc g{};
   g.epi = kEpiSituBF16;
   g.paired = true;
   g.M = R;
   g.tile_table = tile_table;
   g.num_m_tiles_dev = num_m_tiles;
-  g.max_m_tiles = max_m_tiles;
+  g.max_m_tiles = static_cast<int>(cdiv(R, TC_BM) + d.E);
   g.N = d.I;
   g.b_rows_per_expert = d.I;
   g.nseg = 1;
@@ -373,23 +372,27 @@ moe_status stage_experts(const moe_dims& d, const moe_weights& w, const void* z_
   g.ldo = d.I;
   g.situ_c = d.situ_c;
   g.fault_site = 140;
-  moe_status st = run_gemm(d, g, s);
-  if (st != MOE_OK) return st;
-  GemmDesc g2{};
-  g2.epi = kEpiF32;
-  g2.M = R;
-  g2.tile_table = tile_table;
-  g2.num_m_tiles_dev = num_m_tiles;
-  g2.max_m_tiles = max_m_tiles;
-  g2.N = d.L;
-  g2.b_rows_per_expert = d.L;
-  g2.nseg = 1;
-  g2.seg[0] = Seg{h_perm, d.I, w.Wo, d.I, static_cast<long long>(d.E) * d.L, d.I};
-  g2.out = y_perm;
-  g2.ldo = d.L;
-  g2.situ_c = d.situ_c;
-  g2.fault_site = 150;
-  return run_gemm(d, g2, s);
+  return run_gemm(d, g, s);
+}
+
+moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void* h_perm, const int4* tile_table,
+                             const int32_t* num_m_tiles, float* y_perm, cudaStream_t s) {
+  const long long R = d.T * d.k;
+  GemmDesc g{};
+  g.epi = kEpiF32;
+  g.M = R;
+  g.tile_table = tile_table;
+  g.num_m_tiles_dev = num_m_tiles;
+  g.max_m_tiles = static_cast<int>(cdiv(R, TC_BM) + d.E);
+  g.N = d.L;
+  g.b_rows_per_expert = d.L;
+  g.nseg = 1;
+  g.seg[0] = Seg{h_perm, d.I, w.Wo, d.I, static_cast<long long>(d.E) * d.L, d.I};
+  g.out = y_perm;
+  g.ldo = d.L;
+  g.situ_c = d.situ_c;
+  g.fault_site = 150;
+  return run_gemm(d, g, s);
 }
 
 template <typename OutT>
@@ -532,8 +535,11 @@ moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z
                                        at<int32_t>(ws, L.num_m_tiles));
   ++g_last_launches;
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-  return stage_experts(*d, *w, z_perm, at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles),
-                       at<void>(ws, L.h_perm), y_perm, s);
+  const int4* table = at<int4>(ws, L.tile_table);
+  const int32_t* n_tiles = at<int32_t>(ws, L.num_m_tiles);
+  st = stage_expert_gate_up(*d, *w, z_perm, table, n_tiles, at<void>(ws, L.h_perm), s);
+  if (st != MOE_OK) return st;
+  return stage_expert_down(*d, *w, at<void>(ws, L.h_perm), table, n_tiles, y_perm, s);
 }
 
 moe_status moe_combine(const moe_dims* d, const float* y_perm, const int32_t* inv_perm, const float* topk_w,
@@ -563,6 +569,9 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
   moe_aux a{};
   if (aux != nullptr) a = *aux;
   const void* auxp[] = {a.scores, a.topk_idx, a.topk_w, a.expert_offsets, a.u, a.n, a.z};
+  if (a.stage_events != nullptr)
+    for (int i = 0; i < 2 * MOE_NUM_STAGES; ++i)
+      if (a.stage_events[i] == nullptr) return MOE_ERR_INVALID_ARG;
   for (const void* p : auxp)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (!ws_ok(*d, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
@@ -581,23 +590,52 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
   int32_t* perm_token = at<int32_t>(ws, L.perm_token);
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
 
+  // Records event 2*stage (+1 after) when the caller asked for stage timing.
+  auto mark = [&](int stage, int after) {
+    if (a.stage_events != nullptr)
+      cudaEventRecord(static_cast<cudaEvent_t>(a.stage_events[2 * stage + after]), s);
+  };
   // x-side: router scores, latent projection, shared experts' gate/up
+  mark(MOE_STAGE_ROUTER, 0);
   if ((st = stage_router(*d, x, w->Wr, scores, s)) != MOE_OK) return st;
+  mark(MOE_STAGE_ROUTER, 1);
+  mark(MOE_STAGE_TOPK, 0);
   if ((st = stage_topk(*d, scores, w->bias, idx, tw, s)) != MOE_OK) return st;
+  mark(MOE_STAGE_TOPK, 1);
+  mark(MOE_STAGE_LATENT_DOWN, 0);
   if ((st = stage_dense(*d, d->act == MOE_BF16 ? kEpiBF16 : kEpiF32, x, d->H, w->Wdown, d->L, d->H, z, d->L, 120,
                         s)) != MOE_OK)
     return st;
+  mark(MOE_STAGE_LATENT_DOWN, 1);
+  mark(MOE_STAGE_SHARED_GATE_UP, 0);
   if (d->S > 0 && (st = stage_shared_gate_up(*d, *w, x, h_s, s)) != MOE_OK) return st;
+  mark(MOE_STAGE_SHARED_GATE_UP, 1);
   // dispatch
+  mark(MOE_STAGE_PERMUTE, 0);
   if ((st = stage_permute(*d, idx, L, ws, offsets, nullptr, perm_token, inv_perm, s)) != MOE_OK) return st;
+  mark(MOE_STAGE_PERMUTE, 1);
+  mark(MOE_STAGE_GATHER, 0);
   if ((st = stage_gather(*d, z, at<void>(ws, L.z_perm), perm_token, offsets + d->E, s)) != MOE_OK) return st;
+  mark(MOE_STAGE_GATHER, 1);
   // routed experts
-  if ((st = stage_experts(*d, *w, at<void>(ws, L.z_perm), at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles),
-                          at<void>(ws, L.h_perm), at<float>(ws, L.y_perm), s)) != MOE_OK)
+  const int4* table = at<int4>(ws, L.tile_table);
+  const int32_t* n_tiles = at<int32_t>(ws, L.num_m_tiles);
+  mark(MOE_STAGE_EXPERT_GATE_UP, 0);
+  if ((st = stage_expert_gate_up(*d, *w, at<void>(ws, L.z_perm), table, n_tiles, at<void>(ws, L.h_perm), s)) != MOE_OK)
     return st;
+  mark(MOE_STAGE_EXPERT_GATE_UP, 1);
+  mark(MOE_STAGE_EXPERT_DOWN, 0);
+  if ((st = stage_expert_down(*d, *w, at<void>(ws, L.h_perm), table, n_tiles, at<float>(ws, L.y_perm), s)) != MOE_OK)
+    return st;
+  mark(MOE_STAGE_EXPERT_DOWN, 1);
   // combine + RMSNorm, then [shared | W_up] output projection
+  mark(MOE_STAGE_COMBINE, 0);
   if ((st = stage_combine(*d, at<float>(ws, L.y_perm), inv_perm, tw, w->gamma, a.u, n, s)) != MOE_OK) return st;
-  return stage_output(*d, *w, h_s, n, y, s);
+  mark(MOE_STAGE_COMBINE, 1);
+  mark(MOE_STAGE_OUTPUT, 0);
+  st = stage_output(*d, *w, h_s, n, y, s);
+  mark(MOE_STAGE_OUTPUT, 1);
+  return st;
 }
 
 moe_status moe_device_error(int* code, moe_stream_t stream) {
