@@ -107,6 +107,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------------- ranks
+def max_over_ranks(ms: float, device) -> float:
+    """Slowest rank's elapsed time: every rank contributes its device-timed
+    milliseconds; all ranks get the maximum (the job's time)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (max_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------------- roofline
 def dominant_stage(cfg) -> str:
     return "expert_gate_up"
@@ -167,11 +183,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
     ms_per_step = ms / args.steps
 
     # per-stage device time inside the timed region
@@ -201,11 +213,8 @@ def run_ours(args, rank, world, local_rank):
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         torch.distributed.barrier()
 
     st, code = moe.moe_device_error()
@@ -215,8 +224,7 @@ def run_ours(args, rank, world, local_rank):
         return None
 
     peaks = load_peaks()
-    tokens_total = cfg.T * args.steps * world
-    value = tokens_total / (ms / 1e3)
+    value = job_throughput(cfg.T, args.steps, world, ms)
     off = offsets.cpu().numpy()
     work = stage_work(cfg, off, cfg.T)
     dom = dominant_stage(cfg)
@@ -277,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
             "algorithmic": {"flops": work["flops"], "bytes": work["bytes"]},
         },
         "e2e": {
-            "value": round(tokens_total / (e2e_ms / 1e3), 1),
+            "value": round(job_throughput(cfg.T, args.steps, world, e2e_ms), 1),
             "unit": "tokens/s",
             "h2d_bytes_per_step": x.numel() * x.element_size(),
             "d2h_bytes_per_step": y.numel() * y.element_size(),
