@@ -192,6 +192,30 @@ MOE_API moe_status moe_combine(const moe_dims* d, const float* y_perm, const int
 MOE_API moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void* x, void* y, const moe_aux* aux,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Allocation-free variant of moe_permute (the pages have no counterpart; this
+ * is a library facility).  For callers that cannot allocate device memory when
+ * they route tokens -- code running inside an allocator or memory-pool
+ * callback, runtimes that forbid cudaMalloc after start-up to keep a fixed
+ * footprint, hosts that own no allocator -- it takes no workspace: its scratch
+ * (per-tile expert counts, in-tile ranks, tile table) lives in a fixed device
+ * array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES inside the library, which every
+ * GPU that loads the library keeps until the process exits.  The call itself
+ * allocates nothing.  Arguments and outputs are those of moe_permute.
+ *  - Scratch needed: 256-byte-rounded sum of 4*ceil(T/128)*E, 4*T*k,
+ *    16*(ceil(T*k/128) + E) and 16 bytes; larger dims return
+ *    MOE_ERR_INVALID_ARG (K3 shape: up to about 40k tokens).
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture.
+ *  - All calls share the one array: calls whose work overlaps on the GPU
+ *    (different streams, or different host threads without ordering) race and
+ *    give wrong results.  Successive calls on one stream are safe; nothing in
+ *    the array needs clearing between them. */
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+MOE_API moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk_idx, const void* z,
+                                       int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
+                                       void* z_perm, moe_stream_t stream);
+
 /* Human-readable name of a status. */
 MOE_API const char* moe_status_str(moe_status s);
 

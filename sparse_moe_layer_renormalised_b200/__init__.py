@@ -30,6 +30,8 @@ from ._binding import (  # noqa: F401
     moe_last_launch_count,
     moe_layer_forward,
     moe_permute,
+    moe_permute_noalloc,
+    MOE_PERMUTE_NOALLOC_SCRATCH_BYTES,
     moe_router_topk,
     moe_status_str,
     moe_weights,

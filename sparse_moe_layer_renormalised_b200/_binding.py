@@ -30,7 +30,10 @@ EXPORTED = (
     "moe_status_str",
     "moe_device_error",
     "moe_last_launch_count",
+    "moe_permute_noalloc",
 )
+
+MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class moe_dims(ctypes.Structure):
@@ -96,6 +99,7 @@ def lib() -> ctypes.CDLL:
         L.moe_status_str.restype = ctypes.c_char_p
         L.moe_device_error.argtypes = [ctypes.POINTER(i32), vp]
         L.moe_last_launch_count.argtypes = []
+        L.moe_permute_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp]
         for f in EXPORTED:
             if f not in ("moe_workspace_size", "moe_status_str"):
                 getattr(L, f).restype = i32
@@ -206,6 +210,13 @@ def moe_layer_forward(d, weights: moe_weights, x, y, aux: moe_aux | None, ws, ws
     return lib().moe_layer_forward(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(x), _ptr(y),
                                    ctypes.byref(aux) if aux is not None else None, _ptr(ws), ws_bytes,
                                    _stream(stream))
+
+
+def moe_permute_noalloc(d, topk_idx, z, expert_offsets, perm_token, inv_perm, z_perm, stream=None) -> int:
+    """moe_permute without a workspace, for callers that cannot allocate: its
+    scratch is a fixed array inside the library (see include/moe.h)."""
+    return lib().moe_permute_noalloc(ctypes.byref(_dims(d)), _ptr(topk_idx), _ptr(z), _ptr(expert_offsets),
+                                     _ptr(perm_token), _ptr(inv_perm), _ptr(z_perm), _stream(stream))
 
 
 def moe_status_str(status: int) -> str:

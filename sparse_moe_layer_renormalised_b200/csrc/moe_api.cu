@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "combine.cuh"
 #include "gemm_simt.cuh"
@@ -653,3 +654,97 @@ moe_status moe_device_error(int* code, moe_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------
+// Allocation-free dispatch: moe_permute_noalloc.
+//
+// Some callers cannot allocate device memory at the point where they route
+// tokens: code running inside a custom allocator or memory-pool callback, a
+// runtime that forbids cudaMalloc after start-up so its memory footprint stays
+// fixed, or a host that hands this library its inputs and outputs but owns no
+// allocator of its own.  This variant keeps its scratch (per-tile expert
+// counts, in-tile ranks, tile table) in a file-scope device array instead of a
+// caller workspace.  The array is part of the library image: every GPU that
+// loads the library holds it until the process exits.
+namespace moe {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(MOE_PERMUTE_NOALLOC_SCRATCH_BYTES);
+static __device__ __align__(256) uint8_t g_permute_scratch[kNoAllocScratchBytes];
+
+struct NoAllocLayout {
+  size_t tile_base, rank, tile_table, num_m_tiles, total;
+};
+
+NoAllocLayout noalloc_layout(const moe_dims& d) {
+  NoAllocLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, kAlign);
+    return o;
+  };
+  const size_t T = static_cast<size_t>(d.T), R = T * d.k;
+  l.tile_base = take(static_cast<size_t>(cdiv(d.T, PERM_TILE)) * d.E * 4);
+  l.rank = take(R * 4);
+  l.tile_table = take((static_cast<size_t>(cdiv(static_cast<long long>(R), TC_BM)) + d.E) * 16);
+  l.num_m_tiles = take(16);
+  l.total = off;
+  return l;
+}
+
+// Device address of g_permute_scratch on the current device.  The host-side
+// name of a __device__ array is only a stand-in, so the address is asked for
+// once per device (with that device current) and cached.
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[128] = {};
+
+moe_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk_idx, const void* z,
+                                          int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
+                                          void* z_perm, moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (topk_idx == nullptr || expert_offsets == nullptr || perm_token == nullptr || inv_perm == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((z == nullptr) != (z_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (z != nullptr && (!aligned16(z) || !aligned16(z_perm))) return MOE_ERR_INVALID_ARG;
+  const NoAllocLayout L = noalloc_layout(*d);
+  if (L.total > kNoAllocScratchBytes) return MOE_ERR_INVALID_ARG;  // more scratch than the fixed array holds
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // Every scratch word the kernels read is written earlier in the same call,
+  // so nothing has to be cleared between calls.
+  const long long ntiles = cdiv(d->T, PERM_TILE);
+  int32_t* tile_base = at<int32_t>(scratch, L.tile_base);
+  int32_t* rank = at<int32_t>(scratch, L.rank);
+  perm_rank_kernel<<<static_cast<unsigned>(ntiles), PERM_TILE, static_cast<size_t>(d->E) * 16, s>>>(
+      topk_idx, d->T, d->E, d->k, tile_base, rank);
+  perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d->E, nullptr, expert_offsets,
+                                      at<int4>(scratch, L.tile_table), at<int32_t>(scratch, L.num_m_tiles));
+  const long long pairs = d->T * d->k;
+  perm_scatter_kernel<<<static_cast<unsigned>(cdiv(pairs, 256)), 256, 0, s>>>(
+      topk_idx, d->T, d->E, d->k, tile_base, rank, expert_offsets, perm_token, inv_perm);
+  g_last_launches = 3;
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (z != nullptr) st = stage_gather(*d, z, z_perm, perm_token, expert_offsets + d->E, s);
+  return st;
+}
