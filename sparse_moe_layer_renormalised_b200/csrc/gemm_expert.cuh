@@ -1,0 +1,424 @@
+// Grouped routed-expert GEMM for sm_100a, operands swapped so that expert
+// WEIGHT rows are the MMA's M dimension and TOKENS its N dimension:
+//
+//   D[w, t] = sum_k W_e[w, k] * X[row0 + t, k]      (accumulated in TMEM, fp32)
+//
+// One work item = (token tile, weight tile).  A token tile is at most 256
+// consecutive rows of the expert-major activation buffer that belong to one
+// expert; its MMA N is the row count rounded up to 16, so a tile wastes at
+// most 15 rows (against up to 127 for 128-row M tiles over tokens).
+//
+// CG = 2 runs each item on a CTA pair (a 2-CTA cluster) with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA stages 128 weight rows and
+// half of the token rows, so per SM the shared-memory traffic per MMA is two
+// thirds of the 1-CTA 128x256 tile's.  Only the even CTA issues MMAs; TMA loads
+// of both CTAs complete on its barrier; tcgen05.commit multicasts to both.
+// CG = 1 is the same kernel on single CTAs (M = 128).
+//
+// PAIRED (gate/up): each CTA's 128 weight rows are 64 rows of W_g followed by
+// the same 64 rows of W_v (two 64-row TMA boxes), so epilogue warps 0/1 hold g
+// and warps 2/3 hold v for the same intermediate columns; per 32-token chunk
+// the g and v warps of a column range swap half their values through shared
+// memory and each forms SiTU-GLU for 16 of the tokens.  Otherwise (down
+// projection) the 128 rows are consecutive rows of W_o and each lane stores
+// one output column.
+//
+// Warp roles as in gemm_tc.cuh: warp 0 TMA producer, warp 1 TMEM owner and (on
+// the even CTA) MMA issuer, warps 2-5 epilogue.  Every wait is bounded.
+#pragma once
+
+#include "activations.cuh"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int EX_BK = 64;
+constexpr int EX_STAGES = 6;
+constexpr int EX_THREADS = 192;
+constexpr int EX_MAX_TOK = 256;                       // tokens per tile (MMA N <= 256)
+constexpr uint32_t EX_A_BYTES = 128 * EX_BK * 2;      // 128 weight rows
+constexpr uint32_t EX_B_BYTES = 128 * EX_BK * 2;      // up to 128 token rows per CTA
+constexpr uint32_t EX_STAGE_BYTES = EX_A_BYTES + EX_B_BYTES;
+constexpr uint32_t EX_BOX16_BYTES = 16 * EX_BK * 2;   // one 16-row TMA box
+constexpr uint32_t EX_ACC_COLS = 256;
+constexpr uint32_t EX_XCH_FLOATS = 2 * 2 * 16 * 32;        // [pair][direction][token][lane]
+constexpr uint32_t EX_XCH_BYTES = 2 * EX_XCH_FLOATS * 4;    // double-buffered, 16 KB
+constexpr size_t EX_SMEM_BYTES = 1024 + static_cast<size_t>(EX_STAGES) * EX_STAGE_BYTES + EX_XCH_BYTES + 512;
+
+struct ExMaps {
+  CUtensorMap a0;  // PAIRED: W_g as [E*I, L], 64-row boxes; else W_o as [E*L, I], 128-row boxes
+  CUtensorMap a1;  // PAIRED: W_v as [E*I, L], 64-row boxes
+  CUtensorMap b;   // activations [R, K], 16-row boxes
+};
+
+struct ExParams {
+  const int4* tile_table;     // {expert, row0, ntok, 0} per token tile
+  const int* num_tiles_dev;   // number of valid entries
+  int n_wtiles;               // weight tiles per expert
+  int w_rows_per_expert;      // I (PAIRED) or L
+  int num_k_blocks;
+  void* out;                  // PAIRED: bf16 h [R, I]; else fp32 y [R, L]
+  long long ldo;
+  int out_cols;               // I or L (output columns; bound for stores)
+  float situ_c;
+  int fault_site;
+};
+
+// ------------------------------------------------------------------------------ 2-CTA PTX
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Barrier 1 over the 128 epilogue threads (warps 2-5).
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+template <int CG>
+__device__ __forceinline__ void ex_tmem_alloc(uint32_t* holder) {
+  if (CG == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(holder)),
+                 "r"(2 * EX_ACC_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  } else {
+    tmem_alloc(holder, 2 * EX_ACC_COLS);
+    tmem_relinquish();
+  }
+}
+
+template <int CG>
+__device__ __forceinline__ void ex_tmem_dealloc(uint32_t taddr) {
+  if (CG == 2)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(2 * EX_ACC_COLS) : "memory");
+  else
+    tmem_dealloc(taddr, 2 * EX_ACC_COLS);
+}
+
+// TMA tile load that completes on the pair's even-CTA barrier (CG = 2) or the
+// local one (CG = 1).  `bar` is the local barrier; for CG = 2 the pair bit of
+// its address is cleared so both CTAs signal the even CTA's copy.
+template <int CG>
+__device__ __forceinline__ void ex_tma_load(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0, int32_t c1) {
+  if (CG == 2) {
+    const uint32_t mb = smem_u32(bar) & 0xFEFFFFFFu;
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(mb)
+        : "memory");
+  } else {
+    tma_load_2d(dst, map, bar, c0, c1);
+  }
+}
+
+template <int CG>
+__device__ __forceinline__ void ex_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  if (CG == 2) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    tc_mma_bf16(d_tmem, adesc, bdesc, idesc, accumulate);
+  }
+}
+
+// Arrive on `bar` (same offset in both CTAs of the pair for CG = 2) when the
+// MMAs issued so far have completed.
+template <int CG>
+__device__ __forceinline__ void ex_commit(uint64_t* bar) {
+  if (CG == 2) {
+    const uint16_t mask = 0x3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                     "r"(smem_u32(bar)),
+                 "h"(mask)
+                 : "memory");
+  } else {
+    tc_commit(bar);
+  }
+}
+
+struct ExTile {
+  int expert, row0, ntok, n_mma, wt;
+};
+
+__device__ __forceinline__ ExTile ex_decode(int w, const ExParams& p) {
+  const int tt = w / p.n_wtiles;
+  ExTile t;
+  t.wt = w - tt * p.n_wtiles;
+  const int4 e = p.tile_table[tt];
+  t.expert = e.x;
+  t.row0 = e.y;
+  t.ntok = e.z;
+  t.n_mma = max(16, (t.ntok + 15) & ~15);
+  return t;
+}
+
+template <int EPI, bool PAIRED, int CG>
+__global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_constant__ ExMaps maps, const ExParams p) {
+  extern __shared__ uint8_t ex_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ex_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + EX_STAGES * EX_A_BYTES;
+  float* xch = reinterpret_cast<float*>(sB + EX_STAGES * EX_B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + EX_STAGES * EX_B_BYTES + EX_XCH_BYTES);
+  uint64_t* empty = full + EX_STAGES;
+  uint64_t* acc_full = empty + EX_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_ok = abort + 1;  // accumulator-ready verdict shared by the epilogue warps
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int pair = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int npairs = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < EX_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4 * CG);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.a0);
+    if (PAIRED) tma_prefetch_desc(&maps.a1);
+    tma_prefetch_desc(&maps.b);
+  }
+  if (warp == 1) ex_tmem_alloc<CG>(tmem_holder);
+  tc_fence_before();
+  if (CG == 2)
+    cluster_sync_all();
+  else
+    __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int total = *p.num_tiles_dev * p.n_wtiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0u, issued_parity = 0u;
+      bool ok = true;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const ExTile t = ex_decode(w, p);
+        const int rows_cta = CG == 2 ? t.n_mma / 2 : t.n_mma;   // token rows this CTA stages
+        const int nbox = (rows_cta + 15) >> 4;
+        const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
+        const uint32_t bytes = static_cast<uint32_t>(CG) * (EX_A_BYTES + nbox * EX_BOX16_BYTES);
+        // weight rows of this CTA
+        const int wrow_pair = PAIRED ? t.wt * (64 * CG) : t.wt * (128 * CG);
+        const int wrow = t.expert * p.w_rows_per_expert + wrow_pair + static_cast<int>(rank) * (PAIRED ? 64 : 128);
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.fault_site + 1)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
+          const int kc = kb * EX_BK;
+          uint8_t* a_dst = sA + stage * EX_A_BYTES;
+          uint8_t* b_dst = sB + stage * EX_B_BYTES;
+          if (PAIRED) {
+            ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
+            ex_tma_load<CG>(a_dst + EX_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
+          } else {
+            ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
+          }
+          for (int bx = 0; bx < nbox; ++bx)
+            ex_tma_load<CG>(b_dst + bx * EX_BOX16_BYTES, &maps.b, &full[stage], kc, tok0 + 16 * bx);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == EX_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // The even CTA's barriers count both CTAs' bytes: it waits for every
+      // load of the pair to land before the pair may exit.
+      if (leader) {
+        volatile int never = 0;
+        for (int s = 0; s < EX_STAGES; ++s)
+          if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_parity >> s) & 1u, &never, p.fault_site + 2);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const ExTile t = ex_decode(w, p);
+        const uint32_t idesc = idesc_bf16_f32(128 * CG, t.n_mma);
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort, p.fault_site + 3)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * EX_ACC_COLS);
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort, p.fault_site + 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * EX_A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * EX_B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < EX_BK / 16; ++kk)
+            ex_mma<CG>(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                       (kb | kk) != 0 ? 1u : 0u);
+          ex_commit<CG>(&empty[stage]);
+          if (++stage == EX_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ex_commit<CG>(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      ex_commit<CG>(drain);
+    }
+    // Both CTAs: every MMA touching this CTA's shared memory or TMEM is done.
+    if (lane == 0) {
+      volatile int never = 0;
+      mbar_wait(drain, 0u, &never, p.fault_site + 5);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const uint32_t acc_empty_leader =
+        CG == 2 ? map_to_rank(smem_u32(&acc_empty[0]), 0u) : smem_u32(&acc_empty[0]);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int xbuf = 0;
+    for (int w = pair; w < total; w += npairs) {
+      const ExTile t = ex_decode(w, p);
+      bool got;
+      if constexpr (PAIRED) {
+        // One thread waits; the verdict reaches all four warps through the
+        // epilogue barrier, so they always run the same number of barriers.
+        if (threadIdx.x == 64) *epi_ok = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
+        epilogue_bar();
+        got = *epi_ok != 0;
+      } else {
+        // warp-uniform decision: tcgen05.ld below needs the whole warp
+        got = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6));
+      }
+      if (!got) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EX_ACC_COLS);
+      const int nch = (t.ntok + 31) >> 5;  // 32-token chunks (uniform over the epilogue warps)
+      if constexpr (PAIRED) {
+        // warps 0,1 hold g and warps 2,3 hold v for intermediate columns
+        // base + 32 * (q & 1) + lane; g warps form tokens 0-15 of a chunk,
+        // v warps tokens 16-31, after swapping the other half.
+        const bool is_g = q < 2;
+        const int col = t.wt * (64 * CG) + static_cast<int>(rank) * 64 + (q & 1) * 32 + lane;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+        const float c = p.situ_c;
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          float r[32];
+          tmem_ld32(tbase + ch * 32, r);
+          float* X = xch + xbuf * EX_XCH_FLOATS + (q & 1) * 1024;
+          // direction 0 region carries g (tokens 16-31), direction 1 carries v (tokens 0-15)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (is_g)
+              X[i * 32 + lane] = r[16 + i];
+            else
+              X[512 + i * 32 + lane] = r[i];
+          }
+          epilogue_bar();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g = is_g ? r[i] : X[i * 32 + lane];
+            const float v = is_g ? X[512 + i * 32 + lane] : r[16 + i];
+            const int tok = ch * 32 + (is_g ? 0 : 16) + i;
+            if (tok < t.ntok && col < p.out_cols)
+              out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = __float2bfloat16_rn(situ_glu_f32(g, v, c));
+          }
+          xbuf ^= 1;
+        }
+      } else {
+        const int col = t.wt * (128 * CG) + static_cast<int>(rank) * 128 + q * 32 + lane;
+        float* out = reinterpret_cast<float*>(p.out);
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          float r[32];
+          tmem_ld32(tbase + ch * 32, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = ch * 32 + i;
+            if (tok < t.ntok && col < p.out_cols) out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = r[i];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 2)
+          mbar_arrive_cluster(acc_empty_leader + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+        else
+          mbar_arrive(&acc_empty[acc]);
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncwarp();  // reconverge lanes that skipped the single-thread roles
+  tc_fence_before();
+  if (CG == 2)
+    cluster_sync_all();
+  else
+    __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    ex_tmem_dealloc<CG>(tmem_base);
+  }
+}
+
+}  // namespace moe

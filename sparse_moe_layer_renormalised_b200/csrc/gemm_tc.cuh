@@ -237,7 +237,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(const __grid_con
     uint32_t acc_phase = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       const TcTile t = tc_decode<PAIRED>(w, p);
-      if (!mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6)) break;
+      // warp-uniform decision: tcgen05.ld below needs the whole warp
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * TC_BN);
       const bool row_ok = r < t.nrows;

@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "combine.cuh"
+#include "gemm_expert.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -65,6 +66,14 @@ moe_status check_dims(const moe_dims* d) {
 }
 
 inline size_t act_bytes(const moe_dims& d) { return d.act == MOE_F32 ? 4 : 2; }
+
+// Expert kernel pairing: 2-CTA pairs when the weight tiles divide evenly.
+int expert_cg(const moe_dims& d) { return (d.I % 128 == 0 && d.L % 256 == 0) ? 2 : 1; }
+
+// Largest token tile of the grouped expert GEMMs (MMA N = 256 on pairs; a
+// single CTA stages at most 128 token rows; the fp32 path uses 128-row tiles).
+int expert_tile_rows(const moe_dims& d) { return d.act == MOE_BF16 ? 128 * expert_cg(d) : 128; }
+
 
 // ------------------------------------------------------------------------------ workspace
 struct WsLayout {
@@ -127,14 +136,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 matrix [rows, cols] with `ld` elements between rows, box 128 rows x 64
-// columns, 128-byte swizzle, out-of-bounds elements read as zero.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+// bf16 matrix [rows, cols] with `ld` elements between rows, box `box_rows`
+// rows x 64 columns, 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+              uint32_t box_rows = TC_BM) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr || rows == 0 || cols == 0) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(TC_BK), static_cast<cuuint32_t>(TC_BM)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(TC_BK), box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -336,7 +346,7 @@ moe_status stage_permute(const moe_dims& d, const int32_t* idx, const WsLayout& 
   perm_rank_kernel<<<static_cast<unsigned>(ntiles), PERM_TILE, static_cast<size_t>(d.E) * 16, s>>>(
       idx, d.T, d.E, d.k, tile_base, rank);
   perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d.E, counts_out, offsets,
-                                      at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles));
+                                      expert_tile_rows(d), at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles));
   const long long pairs = d.T * d.k;
   perm_scatter_kernel<<<static_cast<unsigned>(cdiv(pairs, 256)), 256, 0, s>>>(idx, d.T, d.E, d.k, tile_base, rank,
                                                                               offsets, perm_token, inv_perm);
@@ -354,46 +364,130 @@ moe_status stage_gather(const moe_dims& d, const void* z, void* z_perm, const in
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+template <int EPI, bool PAIRED, int CG>
+cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream_t s) {
+  auto kern = tc_expert_kernel<EPI, PAIRED, CG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(EX_SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(EX_THREADS);
+  cfg.dynamicSmemBytes = EX_SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // One pair per two SMs that can co-schedule a cluster (asked once per device).
+    static int pairs_cache[128] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int pairs = dev >= 0 && dev < 128 ? pairs_cache[dev] : 0;
+    if (pairs == 0) {
+      cfg.gridDim = dim3(2 * 74);
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess || nc <= 0) nc = num_sms() / 2;
+      pairs = nc;
+      if (dev >= 0 && dev < 128) pairs_cache[dev] = pairs;
+    }
+    cfg.gridDim = dim3(2 * pairs);
+  } else {
+    cfg.gridDim = dim3(num_sms());
+    cfg.numAttrs = 0;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, maps, p);
+}
+
+template <int EPI, bool PAIRED>
+cudaError_t launch_expert(int cg, const ExMaps& maps, const ExParams& p, cudaStream_t s) {
+  return cg == 2 ? launch_expert_inst<EPI, PAIRED, 2>(maps, p, s) : launch_expert_inst<EPI, PAIRED, 1>(maps, p, s);
+}
+
 moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const void* z_perm,
-                                const int4* tile_table, const int32_t* num_m_tiles, void* h_perm, cudaStream_t s) {
+                                const int4* tile_table, const int32_t* num_tiles, void* h_perm, cudaStream_t s) {
   const long long R = d.T * d.k;
-  GemmDesc g{};
-  g.epi = kEpiSituBF16;
-  g.paired = true;
-  g.M = R;
-  g.tile_table = tile_table;
-  g.num_m_tiles_dev = num_m_tiles;
-  g.max_m_tiles = static_cast<int>(cdiv(R, TC_BM) + d.E);
-  g.N = d.I;
-  g.b_rows_per_expert = d.I;
-  g.nseg = 1;
-  g.seg[0] = Seg{z_perm, d.L, w.Wg, d.L, static_cast<long long>(d.E) * d.I, d.L};
-  g.b_up = w.Wv;
-  g.out = h_perm;
-  g.ldo = d.I;
-  g.situ_c = d.situ_c;
-  g.fault_site = 140;
-  return run_gemm(d, g, s);
+  ++g_last_launches;
+  if (d.act != MOE_BF16) {
+    GemmDesc g{};
+    g.epi = kEpiSituBF16;
+    g.paired = true;
+    g.M = R;
+    g.tile_table = tile_table;
+    g.num_m_tiles_dev = num_tiles;
+    g.max_m_tiles = static_cast<int>(cdiv(R, 128) + d.E);
+    g.N = d.I;
+    g.b_rows_per_expert = d.I;
+    g.nseg = 1;
+    g.seg[0] = Seg{z_perm, d.L, w.Wg, d.L, static_cast<long long>(d.E) * d.I, d.L};
+    g.b_up = w.Wv;
+    g.out = h_perm;
+    g.ldo = d.I;
+    g.situ_c = d.situ_c;
+    return run_gemm_simt(g, s);
+  }
+  const int cg = expert_cg(d);
+  ExMaps maps;
+  std::memset(&maps, 0, sizeof maps);
+  const uint64_t wrows = static_cast<uint64_t>(d.E) * d.I;
+  if (!make_map(&maps.a0, w.Wg, wrows, d.L, d.L, 64) || !make_map(&maps.a1, w.Wv, wrows, d.L, d.L, 64) ||
+      !make_map(&maps.b, z_perm, static_cast<uint64_t>(R), d.L, d.L, 16))
+    return MOE_ERR_CUDA;
+  ExParams p{};
+  p.tile_table = tile_table;
+  p.num_tiles_dev = num_tiles;
+  p.n_wtiles = d.I / (64 * cg);
+  p.w_rows_per_expert = d.I;
+  p.num_k_blocks = d.L / EX_BK;
+  p.out = h_perm;
+  p.ldo = d.I;
+  p.out_cols = d.I;
+  p.situ_c = d.situ_c;
+  p.fault_site = 140;
+  return launch_expert<kEpiSituBF16, true>(cg, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void* h_perm, const int4* tile_table,
-                             const int32_t* num_m_tiles, float* y_perm, cudaStream_t s) {
+                             const int32_t* num_tiles, float* y_perm, cudaStream_t s) {
   const long long R = d.T * d.k;
-  GemmDesc g{};
-  g.epi = kEpiF32;
-  g.M = R;
-  g.tile_table = tile_table;
-  g.num_m_tiles_dev = num_m_tiles;
-  g.max_m_tiles = static_cast<int>(cdiv(R, TC_BM) + d.E);
-  g.N = d.L;
-  g.b_rows_per_expert = d.L;
-  g.nseg = 1;
-  g.seg[0] = Seg{h_perm, d.I, w.Wo, d.I, static_cast<long long>(d.E) * d.L, d.I};
-  g.out = y_perm;
-  g.ldo = d.L;
-  g.situ_c = d.situ_c;
-  g.fault_site = 150;
-  return run_gemm(d, g, s);
+  ++g_last_launches;
+  if (d.act != MOE_BF16) {
+    GemmDesc g{};
+    g.epi = kEpiF32;
+    g.M = R;
+    g.tile_table = tile_table;
+    g.num_m_tiles_dev = num_tiles;
+    g.max_m_tiles = static_cast<int>(cdiv(R, 128) + d.E);
+    g.N = d.L;
+    g.b_rows_per_expert = d.L;
+    g.nseg = 1;
+    g.seg[0] = Seg{h_perm, d.I, w.Wo, d.I, static_cast<long long>(d.E) * d.L, d.I};
+    g.out = y_perm;
+    g.ldo = d.L;
+    g.situ_c = d.situ_c;
+    return run_gemm_simt(g, s);
+  }
+  const int cg = expert_cg(d);
+  ExMaps maps;
+  std::memset(&maps, 0, sizeof maps);
+  if (!make_map(&maps.a0, w.Wo, static_cast<uint64_t>(d.E) * d.L, d.I, d.I, 128) ||
+      !make_map(&maps.b, h_perm, static_cast<uint64_t>(R), d.I, d.I, 16))
+    return MOE_ERR_CUDA;
+  ExParams p{};
+  p.tile_table = tile_table;
+  p.num_tiles_dev = num_tiles;
+  p.n_wtiles = d.L / (128 * cg);
+  p.w_rows_per_expert = d.L;
+  p.num_k_blocks = d.I / EX_BK;
+  p.out = y_perm;
+  p.ldo = d.L;
+  p.out_cols = d.L;
+  p.situ_c = d.situ_c;
+  p.fault_site = 150;
+  return launch_expert<kEpiF32, false>(cg, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 template <typename OutT>
@@ -532,8 +626,8 @@ moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z
   if (d->T == 0) return MOE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(*d);
-  tile_table_kernel<<<1, 1024, 0, s>>>(expert_offsets, d->E, d->T * d->k, at<int4>(ws, L.tile_table),
-                                       at<int32_t>(ws, L.num_m_tiles));
+  tile_table_kernel<<<1, 1024, 0, s>>>(expert_offsets, d->E, d->T * d->k, expert_tile_rows(*d),
+                                       at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_m_tiles));
   ++g_last_launches;
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   const int4* table = at<int4>(ws, L.tile_table);
@@ -738,7 +832,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk
   int32_t* rank = at<int32_t>(scratch, L.rank);
   perm_rank_kernel<<<static_cast<unsigned>(ntiles), PERM_TILE, static_cast<size_t>(d->E) * 16, s>>>(
       topk_idx, d->T, d->E, d->k, tile_base, rank);
-  perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d->E, nullptr, expert_offsets,
+  perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d->E, nullptr, expert_offsets, 128,
                                       at<int4>(scratch, L.tile_table), at<int32_t>(scratch, L.num_m_tiles));
   const long long pairs = d->T * d->k;
   perm_scatter_kernel<<<static_cast<unsigned>(cdiv(pairs, 256)), 256, 0, s>>>(

@@ -153,11 +153,17 @@ __device__ __forceinline__ int block_incl_scan_1024(int v, int* buf) {
   return buf[threadIdx.x];
 }
 
+// Number of grouped-GEMM tiles of expert e: ceil(n_e / max_rows).
+__device__ __forceinline__ int tiles_of(int cnt, int max_rows) { return (cnt + max_rows - 1) / max_rows; }
+
 // Writes the grouped-GEMM tile table: expert e with n_e rows starting at
-// offset o_e contributes ceil(n_e / 128) entries {e, o_e + 128 i, rows}.
-__device__ __forceinline__ void emit_tiles(int e, int off, int cnt, int first, int4* tile_table) {
-  const int mt = (cnt + 127) / 128;
-  for (int i = 0; i < mt; ++i) tile_table[first + i] = make_int4(e, off + 128 * i, min(128, cnt - 128 * i), 0);
+// offset o_e contributes ceil(n_e / max_rows) entries {e, row0, rows} of
+// near-equal height (at most max_rows).
+__device__ __forceinline__ void emit_tiles(int e, int off, int cnt, int first, int max_rows, int4* tile_table) {
+  const int nt = tiles_of(cnt, max_rows);
+  if (nt == 0) return;
+  const int size = (cnt + nt - 1) / nt;
+  for (int i = 0; i < nt; ++i) tile_table[first + i] = make_int4(e, off + size * i, min(size, cnt - size * i), 0);
 }
 
 // One block of 1024 threads, thread = expert.  Turns the per-tile counts into
@@ -165,7 +171,8 @@ __device__ __forceinline__ void emit_tiles(int e, int off, int cnt, int first, i
 // tile table and its length.
 __global__ void __launch_bounds__(1024)
     perm_scan_kernel(int32_t* __restrict__ tile_counts, int ntiles, int E, int32_t* __restrict__ counts_out,
-                     int32_t* __restrict__ offsets, int4* __restrict__ tile_table, int32_t* __restrict__ num_m_tiles) {
+                     int32_t* __restrict__ offsets, int max_tile_rows, int4* __restrict__ tile_table,
+                     int32_t* __restrict__ num_m_tiles) {
   __shared__ int buf[1024];
   const int e = threadIdx.x;
   int run = 0;
@@ -178,14 +185,14 @@ __global__ void __launch_bounds__(1024)
     }
   }
   const int cnt = e < E ? run : 0;
-  const int mt = (cnt + 127) / 128;
+  const int mt = tiles_of(cnt, max_tile_rows);
   const int incl_off = block_incl_scan_1024(cnt, buf);
   __syncthreads();
   const int incl_mt = block_incl_scan_1024(mt, buf);
   if (e < E) {
     offsets[e] = incl_off - cnt;
     if (counts_out != nullptr) counts_out[e] = cnt;
-    emit_tiles(e, incl_off - cnt, cnt, incl_mt - mt, tile_table);
+    emit_tiles(e, incl_off - cnt, cnt, incl_mt - mt, max_tile_rows, tile_table);
   }
   if (e == E - 1) {
     offsets[E] = incl_off;
@@ -197,8 +204,8 @@ __global__ void __launch_bounds__(1024)
 // are not monotone or exceed max_rows are recorded as a fault and the expert
 // is given no rows, so no tile addresses memory outside [0, max_rows).
 __global__ void __launch_bounds__(1024)
-    tile_table_kernel(const int32_t* __restrict__ offsets, int E, long long max_rows, int4* __restrict__ tile_table,
-                      int32_t* __restrict__ num_m_tiles) {
+    tile_table_kernel(const int32_t* __restrict__ offsets, int E, long long max_rows, int max_tile_rows,
+                      int4* __restrict__ tile_table, int32_t* __restrict__ num_m_tiles) {
   __shared__ int buf[1024];
   const int e = threadIdx.x;
   int off = 0, cnt = 0;
@@ -212,9 +219,9 @@ __global__ void __launch_bounds__(1024)
       cnt = end - off;
     }
   }
-  const int mt = (cnt + 127) / 128;
+  const int mt = tiles_of(cnt, max_tile_rows);
   const int incl_mt = block_incl_scan_1024(mt, buf);
-  if (e < E) emit_tiles(e, off, cnt, incl_mt - mt, tile_table);
+  if (e < E) emit_tiles(e, off, cnt, incl_mt - mt, max_tile_rows, tile_table);
   if (e == E - 1) *num_m_tiles = incl_mt;
 }
 

@@ -120,9 +120,11 @@ def test_combine_rmsnorm(T, L, k, act):
 
 
 # ------------------------------------------------------------------------------ experts
-@pytest.mark.parametrize("T", [512, 37])
-def test_expert_ffn_mid_dims(T):
-    cfg = gen.CONFIGS["mid"]
+@pytest.mark.parametrize("T,L", [(512, 1024), (37, 1024), (300, 1152)])
+def test_expert_ffn_mid_dims(T, L):
+    # L = 1024 runs the expert GEMMs on CTA pairs; L = 1152 (not a multiple of
+    # 256) on single CTAs.
+    cfg = gen.CONFIGS["mid"].with_(L=L)
     E, k, L, I = cfg.E, cfg.k, cfg.L, cfg.I
     d = dims_for(cfg, T=T)
     w = gen.device_layer(cfg.with_(T=T), "cuda", with_x=False)
