@@ -62,7 +62,7 @@ CONFIGS: dict[str, LayerConfig] = {
     # Profiling stand-in for the prefill layer: K3 matrix shapes, 64 experts
     # (4.2 GB of routed weights instead of 59 GB) so that multi-pass counter
     # captures stay small; not a measured workload.
-    "prefill-e64": LayerConfig("prefill-e64", T=2048, H=7168, L=3584, E=64, k=16, I=3072, S=2, Is=3072, bias="zipf",
+    "prefill-e64": LayerConfig("prefill-e64", T=1024, H=7168, L=3584, E=64, k=16, I=3072, S=2, Is=3072, bias="zipf",
                                oracle_tokens=64),
 }
 

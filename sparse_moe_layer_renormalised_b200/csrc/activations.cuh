@@ -12,9 +12,21 @@ __device__ __forceinline__ float sigmoid_f32(float l) { return 1.0f / (1.0f + ex
 // SiTU-GLU: SwiGLU sigmoid(g) * g * v with the linear factor g and the up
 // branch v replaced by the smooth caps c * tanh(. / c)  (tech-report summary,
 // section "幅のスケーリング：Stable LatentMoE"; closed form is this library's
-// reading of that description).
+// reading of that description).  Used by the fp32 path.
 __device__ __forceinline__ float situ_glu_f32(float g, float v, float c) {
   return sigmoid_f32(g) * (c * tanhf(g / c)) * (c * tanhf(v / c));
+}
+
+// The same SiTU-GLU for bf16-stored outputs, from CUDA's fast exponential and
+// division intrinsics: sigmoid(g) = 1 / (1 + e^-g) and
+// tanh(x) = 1 - 2 / (e^(2x) + 1).  Relative error is around 1e-6, far below
+// the 2^-9 rounding of the bf16 result; e^(2x) overflowing to +inf gives
+// tanh = 1 and underflowing to 0 gives -1, as it should.
+__device__ __forceinline__ float fast_tanh(float x) { return 1.0f - __fdividef(2.0f, __expf(2.0f * x) + 1.0f); }
+
+__device__ __forceinline__ float situ_glu_fast(float g, float v, float c, float inv_c) {
+  const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+  return sg * (c * fast_tanh(g * inv_c)) * (c * fast_tanh(v * inv_c));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -40,16 +40,15 @@ constexpr int EX_MAX_TOK = 256;                       // tokens per tile (MMA N 
 constexpr uint32_t EX_A_BYTES = 128 * EX_BK * 2;      // 128 weight rows
 constexpr uint32_t EX_B_BYTES = 128 * EX_BK * 2;      // up to 128 token rows per CTA
 constexpr uint32_t EX_STAGE_BYTES = EX_A_BYTES + EX_B_BYTES;
-constexpr uint32_t EX_BOX16_BYTES = 16 * EX_BK * 2;   // one 16-row TMA box
 constexpr uint32_t EX_ACC_COLS = 256;
 constexpr uint32_t EX_XCH_FLOATS = 2 * 2 * 16 * 32;        // [pair][direction][token][lane]
 constexpr uint32_t EX_XCH_BYTES = 2 * EX_XCH_FLOATS * 4;    // double-buffered, 16 KB
 constexpr size_t EX_SMEM_BYTES = 1024 + static_cast<size_t>(EX_STAGES) * EX_STAGE_BYTES + EX_XCH_BYTES + 512;
 
 struct ExMaps {
-  CUtensorMap a0;  // PAIRED: W_g as [E*I, L], 64-row boxes; else W_o as [E*L, I], 128-row boxes
-  CUtensorMap a1;  // PAIRED: W_v as [E*I, L], 64-row boxes
-  CUtensorMap b;   // activations [R, K], 16-row boxes
+  CUtensorMap a0;      // PAIRED: W_g as [E*I, L], 64-row boxes; else W_o as [E*L, I], 128-row boxes
+  CUtensorMap a1;      // PAIRED: W_v as [E*I, L], 64-row boxes
+  CUtensorMap b[4];    // activations [R, K] with 128-, 64-, 32- and 16-row boxes
 };
 
 struct ExParams {
@@ -162,10 +161,28 @@ struct ExTile {
   int expert, row0, ntok, n_mma, wt;
 };
 
-__device__ __forceinline__ ExTile ex_decode(int w, const ExParams& p) {
-  const int tt = w / p.n_wtiles;
+// Work order: token tiles are taken in groups of EX_GROUP consecutive tiles;
+// inside a group the weight tile is the outer index.  Consecutive work items
+// then share a weight tile (its rows stream from HBM once per group, not once
+// per token tile, when a large expert has many token tiles) while the
+// group's token rows stay in L2 across the weight tiles.
+constexpr int EX_GROUP = 8;
+
+// The producer asks L2 for this CTA's weight rows EX_PREFETCH k-blocks ahead
+// of the tile loads, so the ring's loads find them in L2 instead of waiting on
+// HBM latency (the shared-memory ring alone cannot cover it when small token
+// tiles consume a stage every few hundred cycles).
+constexpr int EX_PREFETCH = 12;
+
+__device__ __forceinline__ ExTile ex_decode(int w, int num_tiles, const ExParams& p) {
+  const int gsize = EX_GROUP * p.n_wtiles;
+  const int grp = w / gsize;
+  const int r = w - grp * gsize;
+  const int in_grp = min(EX_GROUP, num_tiles - grp * EX_GROUP);
+  const int wt = r / in_grp;
+  const int tt = grp * EX_GROUP + (r - wt * in_grp);
   ExTile t;
-  t.wt = w - tt * p.n_wtiles;
+  t.wt = wt;
   const int4 e = p.tile_table[tt];
   t.expert = e.x;
   t.row0 = e.y;
@@ -213,7 +230,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&maps.a0);
     if (PAIRED) tma_prefetch_desc(&maps.a1);
-    tma_prefetch_desc(&maps.b);
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(&maps.b[i]);
   }
   if (warp == 1) ex_tmem_alloc<CG>(tmem_holder);
   tc_fence_before();
@@ -224,7 +241,8 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int total = *p.num_tiles_dev * p.n_wtiles;
+  const int num_tiles = *p.num_tiles_dev;
+  const int total = num_tiles * p.n_wtiles;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (both CTAs)
@@ -233,16 +251,39 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
       uint32_t phase = 0;
       uint32_t issued = 0u, issued_parity = 0u;
       bool ok = true;
-      for (int w = pair; w < total && ok; w += npairs) {
-        const ExTile t = ex_decode(w, p);
-        const int rows_cta = CG == 2 ? t.n_mma / 2 : t.n_mma;   // token rows this CTA stages
-        const int nbox = (rows_cta + 15) >> 4;
-        const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
-        const uint32_t bytes = static_cast<uint32_t>(CG) * (EX_A_BYTES + nbox * EX_BOX16_BYTES);
-        // weight rows of this CTA
+      // prefetch cursor, EX_PREFETCH k-blocks ahead of the loads
+      int pf_w = pair, pf_kb = 0, pf_row = -1;
+      auto weight_row = [&](const ExTile& t) {
         const int wrow_pair = PAIRED ? t.wt * (64 * CG) : t.wt * (128 * CG);
-        const int wrow = t.expert * p.w_rows_per_expert + wrow_pair + static_cast<int>(rank) * (PAIRED ? 64 : 128);
+        return t.expert * p.w_rows_per_expert + wrow_pair + static_cast<int>(rank) * (PAIRED ? 64 : 128);
+      };
+      auto prefetch_next = [&]() {
+        if (pf_w >= total) return;
+        if (pf_row < 0) pf_row = weight_row(ex_decode(pf_w, num_tiles, p));
+        const int kc = pf_kb * EX_BK;
+        tma_prefetch_l2_2d(&maps.a0, kc, pf_row);
+        if (PAIRED) tma_prefetch_l2_2d(&maps.a1, kc, pf_row);
+        if (++pf_kb == p.num_k_blocks) {
+          pf_kb = 0;
+          pf_w += npairs;
+          pf_row = -1;
+        }
+      };
+      for (int i = 0; i < EX_PREFETCH; ++i) prefetch_next();
+      for (int w = pair; w < total && ok; w += npairs) {
+        const ExTile t = ex_decode(w, num_tiles, p);
+        const int rows_cta = CG == 2 ? t.n_mma / 2 : t.n_mma;   // token rows this CTA stages
+        // Staged as ONE box of 128, 64, 32 or 16 rows, the smallest that covers
+        // the tile: measured on B200, a single TMA request per operand and
+        // stage streams far better than several smaller ones, even though up
+        // to half of the box may be rows of the next tile.
+        const int bsel = rows_cta > 64 ? 0 : rows_cta > 32 ? 1 : rows_cta > 16 ? 2 : 3;
+        const int brows = 128 >> bsel;
+        const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
+        const uint32_t bytes = static_cast<uint32_t>(CG) * (EX_A_BYTES + brows * EX_BK * 2);
+        const int wrow = weight_row(t);  // first weight row of this CTA
         for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          prefetch_next();
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.fault_site + 1)) {
             ok = false;
             break;
@@ -257,8 +298,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
           } else {
             ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
           }
-          for (int bx = 0; bx < nbox; ++bx)
-            ex_tma_load<CG>(b_dst + bx * EX_BOX16_BYTES, &maps.b, &full[stage], kc, tok0 + 16 * bx);
+          ex_tma_load<CG>(b_dst, &maps.b[bsel], &full[stage], kc, tok0);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == EX_STAGES) {
@@ -284,7 +324,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int w = pair; w < total && ok; w += npairs) {
-        const ExTile t = ex_decode(w, p);
+        const ExTile t = ex_decode(w, num_tiles, p);
         const uint32_t idesc = idesc_bf16_f32(128 * CG, t.n_mma);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort, p.fault_site + 3)) break;
         tc_fence_after();
@@ -331,7 +371,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
     uint32_t acc_phase = 0;
     int xbuf = 0;
     for (int w = pair; w < total; w += npairs) {
-      const ExTile t = ex_decode(w, p);
+      const ExTile t = ex_decode(w, num_tiles, p);
       bool got;
       if constexpr (PAIRED) {
         // One thread waits; the verdict reaches all four warps through the
@@ -355,6 +395,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
         const int col = t.wt * (64 * CG) + static_cast<int>(rank) * 64 + (q & 1) * 32 + lane;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const float c = p.situ_c;
+        const float inv_c = 1.0f / c;
 #pragma unroll 1
         for (int ch = 0; ch < nch; ++ch) {
           float r[32];
@@ -375,7 +416,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
             const float v = is_g ? X[512 + i * 32 + lane] : r[16 + i];
             const int tok = ch * 32 + (is_g ? 0 : 16) + i;
             if (tok < t.ntok && col < p.out_cols)
-              out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = __float2bfloat16_rn(situ_glu_f32(g, v, c));
+              out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = __float2bfloat16_rn(situ_glu_fast(g, v, c, inv_c));
           }
           xbuf ^= 1;
         }

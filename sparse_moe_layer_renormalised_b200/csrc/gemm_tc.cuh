@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(const __grid_con
         if constexpr (PAIRED) {
           __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
           const float c = p.situ_c;
+          const float inv_c = 1.0f / c;
 #pragma unroll 1
           for (int ch = 0; ch < TC_BN / 64; ++ch) {
             const int col = t.col0 + ch * 32;
@@ -259,7 +260,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(const __grid_con
               uint32_t pk[16];
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(situ_glu_f32(g[2 * i], v[2 * i], c), situ_glu_f32(g[2 * i + 1], v[2 * i + 1], c));
+                pk[i] = pack_bf16x2(situ_glu_fast(g[2 * i], v[2 * i], c, inv_c),
+                                    situ_glu_fast(g[2 * i + 1], v[2 * i + 1], c, inv_c));
               __nv_bfloat16* dst = out + grow * p.ldo + col;
               if (col + 32 <= p.N) {
                 uint4* d4 = reinterpret_cast<uint4*>(dst);

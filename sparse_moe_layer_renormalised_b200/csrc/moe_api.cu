@@ -364,6 +364,14 @@ moe_status stage_gather(const moe_dims& d, const void* z, void* z_perm, const in
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Maps of the expert-major activation rows [R, K] with 128-, 64-, 32- and
+// 16-row boxes (token tiles are staged as a sum of these).
+bool make_token_maps(CUtensorMap* maps4, const void* base, uint64_t rows, uint64_t K) {
+  for (int i = 0; i < 4; ++i)
+    if (!make_map(&maps4[i], base, rows, K, K, 128u >> i)) return false;
+  return true;
+}
+
 template <int EPI, bool PAIRED, int CG>
 cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream_t s) {
   auto kern = tc_expert_kernel<EPI, PAIRED, CG>;
@@ -434,7 +442,7 @@ moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const v
   std::memset(&maps, 0, sizeof maps);
   const uint64_t wrows = static_cast<uint64_t>(d.E) * d.I;
   if (!make_map(&maps.a0, w.Wg, wrows, d.L, d.L, 64) || !make_map(&maps.a1, w.Wv, wrows, d.L, d.L, 64) ||
-      !make_map(&maps.b, z_perm, static_cast<uint64_t>(R), d.L, d.L, 16))
+      !make_token_maps(maps.b, z_perm, static_cast<uint64_t>(R), d.L))
     return MOE_ERR_CUDA;
   ExParams p{};
   p.tile_table = tile_table;
@@ -474,7 +482,7 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
   ExMaps maps;
   std::memset(&maps, 0, sizeof maps);
   if (!make_map(&maps.a0, w.Wo, static_cast<uint64_t>(d.E) * d.L, d.I, d.I, 128) ||
-      !make_map(&maps.b, h_perm, static_cast<uint64_t>(R), d.I, d.I, 16))
+      !make_token_maps(maps.b, h_perm, static_cast<uint64_t>(R), d.I))
     return MOE_ERR_CUDA;
   ExParams p{};
   p.tile_table = tile_table;

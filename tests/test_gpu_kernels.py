@@ -150,3 +150,32 @@ def test_expert_ffn_mid_dims(T, L):
         Wg, Wv, Wo = oin.expert_weights(cfg, e)
         ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wv, Wo, cfg.situ_c, oracle.bf16_round)
     assert parity(y, ref) <= 1e-2
+
+
+def test_expert_ffn_same_gate_and_up_weights():
+    """W_v = W_g (one buffer passed twice): h = SiTU-GLU(g, g)."""
+    cfg = gen.CONFIGS["mid"]
+    T = 256
+    E, k, L, I = cfg.E, cfg.k, cfg.L, cfg.I
+    d = dims_for(cfg, T=T)
+    w = gen.device_layer(cfg.with_(T=T), "cuda", with_x=False)
+    idx = _routing(T, E, k, True, 11)
+    _, offsets, _, _ = oracle.permute(idx.numpy(), E)
+    R = T * k
+    z_perm = torch.randn(R, L, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    y_perm = torch.full((R, L), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(moe.moe_workspace_size(d), dtype=torch.uint8, device="cuda")
+    wts = moe.make_weights(Wg=w["Wg"], Wv=w["Wg"], Wo=w["Wo"])
+    off = torch.as_tensor(offsets, dtype=torch.int32).cuda()
+    assert moe.moe_expert_ffn(d, wts, z_perm.cuda(), off, y_perm, ws) == moe.MOE_OK
+    torch.cuda.synchronize()
+    _no_fault()
+    zf = z_perm.to(F64)
+    ref = torch.empty(R, L, dtype=F64)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        Wg, _, Wo = oin.expert_weights(cfg, e)
+        ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wg, Wo, cfg.situ_c, oracle.bf16_round)
+    assert parity(y_perm.cpu().to(F64), ref) <= 1e-2
