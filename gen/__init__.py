@@ -251,7 +251,7 @@ def device_layer(cfg: LayerConfig, device="cuda", with_x: bool = True) -> dict:
             if rc != 0:
                 raise RuntimeError(f"generator launch failed: cuda error {rc}")
             out[name] = codes
-            out[name + "_scale"] = scales
+            out[{"Wg": "Sg", "Wv": "Sv", "Wo": "So"}[name]] = scales
         else:
             t = torch.empty((E, R, K), dtype=tdt[cfg.routed], device=dev)
             _dev_fill(t, cfg, name)

@@ -59,6 +59,10 @@ CONFIGS: dict[str, LayerConfig] = {
                            oracle_tokens=512),
     "mxfp4": LayerConfig("mxfp4", T=8192, H=7168, L=3584, E=896, k=16, I=3072, S=2, Is=3072, routed="mxfp4",
                          oracle_tokens=512),
+    # Small MXFP4 layer for parity tests (L and I multiples of 512 as the
+    # block-scaled path requires).
+    "mxfp4-small": LayerConfig("mxfp4-small", T=1024, H=2048, L=1024, E=64, k=8, I=1024, S=2, Is=1024,
+                               routed="mxfp4"),
     # Profiling stand-in for the prefill layer: K3 matrix shapes, 64 experts
     # (4.2 GB of routed weights instead of 59 GB) so that multi-pass counter
     # captures stay small; not a measured workload.

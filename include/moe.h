@@ -42,7 +42,12 @@
  * Supported type combinations (moe_dims.act / routed):
  *  - MOE_F32 / MOE_F32     fp32 everywhere (CUDA-core path, small layers);
  *  - MOE_BF16 / MOE_BF16   bf16 operands, fp32 accumulation (tcgen05 path);
- *    H, L, I and Is must be multiples of 64, S <= 3, E <= 1024, k <= 32.
+ *    H, L, I and Is must be multiples of 64, S <= 3, E <= 1024, k <= 32;
+ *  - MOE_BF16 / MOE_MXFP4  routed-expert weights in OCP MXFP4 (the serving
+ *    format of page "ai-tech-express.jp" on K3, section "量子化を前提とした学習
+ *    「MXFP4 Quantization-Aware Training」"), everything else bf16; the kernels
+ *    decode each weight exactly to bf16 in shared memory and multiply in bf16
+ *    with fp32 accumulation.  Additionally L and I must be multiples of 512.
  * Stored activations (z, expert h, shared h, n) are held in the activation type;
  * y_perm, u and the router scores are fp32.
  */
@@ -89,7 +94,7 @@ typedef struct {
   float situ_c;      /* SiTU-GLU cap c (> 0); 10 in the measured configurations */
   float rms_eps;     /* RMSNorm epsilon (>= 0); 1e-6 */
   moe_dtype act;     /* x, dense weights and stored activations: MOE_F32 or MOE_BF16 */
-  moe_dtype routed;  /* routed-expert weights: equal to act */
+  moe_dtype routed;  /* routed-expert weights: equal to act, or MOE_MXFP4 with act = MOE_BF16 */
   moe_dtype y_out;   /* y: MOE_F32, or equal to act */
 } moe_dims;
 
@@ -100,12 +105,15 @@ typedef struct {
   const void* Wdown;   /* [L, H]    latent down-projection */
   const void* Wup;     /* [H, L]    latent up-projection */
   const float* gamma;  /* [L]       fp32 RMSNorm gain */
-  const void* Wg;      /* [E, I, L] routed gate projections (type `routed`) */
-  const void* Wv;      /* [E, I, L] routed up projections */
-  const void* Wo;      /* [E, L, I] routed down projections */
-  const uint8_t* Sg;   /* reserved for block-scaled routed weights; must be NULL */
-  const uint8_t* Sv;   /* reserved; must be NULL */
-  const uint8_t* So;   /* reserved; must be NULL */
+  const void* Wg;      /* [E, I, L] routed gate projections (type `routed`); MXFP4: [E, I, L/2] bytes */
+  const void* Wv;      /* [E, I, L] routed up projections;                   MXFP4: [E, I, L/2] bytes */
+  const void* Wo;      /* [E, L, I] routed down projections;                 MXFP4: [E, L, I/2] bytes */
+  /* MXFP4 only (NULL otherwise): E8M0 scale bytes, one per 32 consecutive
+   * elements along K (value 2^(s-127); 255 = NaN).  Codes are E2M1, two per
+   * byte, the even-K element in the low nibble, bit 3 of a code the sign. */
+  const uint8_t* Sg;   /* [E, I, L/32] */
+  const uint8_t* Sv;   /* [E, I, L/32] */
+  const uint8_t* So;   /* [E, L, I/32] */
   const void* Wsg;     /* [S, Is, H] shared gate projections */
   const void* Wsv;     /* [S, Is, H] shared up projections */
   const void* Wso;     /* [S, H, Is] shared down projections */
@@ -174,7 +182,8 @@ MOE_API moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, const
  * r in expert_offsets[e] .. expert_offsets[e+1]-1:
  *   h = SiTU-GLU(z_perm[r] . Wg[e]^T, z_perm[r] . Wv[e]^T)   (stored in act type)
  *   y_perm[r] = h . Wo[e]^T                                    (fp32 [T*k, L])
- * Only w->Wg, w->Wv, w->Wo are read.  Workspace: moe_workspace_size(d) bytes. */
+ * Only w->Wg, w->Wv, w->Wo (and for MXFP4 w->Sg, w->Sv, w->So) are read.
+ * Workspace: moe_workspace_size(d) bytes. */
 MOE_API moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z_perm,
                           const int32_t* expert_offsets, float* y_perm, void* ws, size_t ws_bytes,
                           moe_stream_t stream);

@@ -23,8 +23,16 @@
 // projection) the 128 rows are consecutive rows of W_o and each lane stores
 // one output column.
 //
+// MX (block-scaled weights): the weights arrive as OCP MXFP4 -- E2M1 codes,
+// two per byte, and one E8M0 scale per 32 elements along K.  Each CTA loads
+// its codes and scales by TMA into a local staging slot; eight converter
+// warps decode them (E2M1 pair -> f16x2 in hardware, times 2^(scale-127) in
+// fp32, packed to bf16, all exact) into the same 128-byte-swizzled bf16 A tile
+// the tensor cores read, and the MMA is the ordinary bf16 kind::f16.
+//
 // Warp roles as in gemm_tc.cuh: warp 0 TMA producer, warp 1 TMEM owner and (on
-// the even CTA) MMA issuer, warps 2-5 epilogue.  Every wait is bounded.
+// the even CTA) MMA issuer, warps 2-5 epilogue, and with MX warps 6-13
+// converters.  Every wait is bounded.
 #pragma once
 
 #include "activations.cuh"
@@ -34,8 +42,6 @@
 namespace moe {
 
 constexpr int EX_BK = 64;
-constexpr int EX_STAGES = 6;
-constexpr int EX_THREADS = 192;
 constexpr int EX_MAX_TOK = 256;                       // tokens per tile (MMA N <= 256)
 constexpr uint32_t EX_A_BYTES = 128 * EX_BK * 2;      // 128 weight rows
 constexpr uint32_t EX_B_BYTES = 128 * EX_BK * 2;      // up to 128 token rows per CTA
@@ -43,11 +49,24 @@ constexpr uint32_t EX_STAGE_BYTES = EX_A_BYTES + EX_B_BYTES;
 constexpr uint32_t EX_ACC_COLS = 256;
 constexpr uint32_t EX_XCH_FLOATS = 2 * 2 * 16 * 32;        // [pair][direction][token][lane]
 constexpr uint32_t EX_XCH_BYTES = 2 * EX_XCH_FLOATS * 4;    // double-buffered, 16 KB
-constexpr size_t EX_SMEM_BYTES = 1024 + static_cast<size_t>(EX_STAGES) * EX_STAGE_BYTES + EX_XCH_BYTES + 512;
+constexpr uint32_t EX_CODES_BYTES = 128 * 32;               // MX: E2M1 codes of 128 rows x 64 K
+constexpr uint32_t EX_SCALES_BYTES = 128 * 16;              // MX: E8M0 scales of 128 rows x 8 k-blocks
+constexpr int EX_CONV_WARPS = 8;
+
+template <bool MX>
+struct ExCfg {
+  static constexpr int kStages = MX ? 5 : 6;
+  static constexpr int kThreads = 192 + (MX ? 32 * EX_CONV_WARPS : 0);
+  static constexpr uint32_t kStageBytes = EX_STAGE_BYTES + (MX ? EX_CODES_BYTES + EX_SCALES_BYTES : 0u);
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + EX_XCH_BYTES + 512;
+};
 
 struct ExMaps {
   CUtensorMap a0;      // PAIRED: W_g as [E*I, L], 64-row boxes; else W_o as [E*L, I], 128-row boxes
-  CUtensorMap a1;      // PAIRED: W_v as [E*I, L], 64-row boxes
+                       // (MX: the packed codes, [rows, K/2] bytes, 32-byte-wide boxes)
+  CUtensorMap a1;      // PAIRED: W_v, as a0
+  CUtensorMap s0;      // MX: E8M0 scales of a0's rows, [rows, K/32] bytes, 16-byte-wide boxes
+  CUtensorMap s1;      // MX, PAIRED: scales of W_v
   CUtensorMap b[4];    // activations [R, K] with 128-, 64-, 32- and 16-row boxes
 };
 
@@ -157,6 +176,27 @@ __device__ __forceinline__ void ex_commit(uint64_t* bar) {
   }
 }
 
+// E8M0 scale byte -> 2^(s - 127) as fp32 (s = 0: 2^-127; s = 255: NaN).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+  if (s == 0u) return __int_as_float(0x00400000);
+  if (s == 255u) return __int_as_float(0x7FC00000);
+  return __int_as_float(static_cast<int>(s << 23));
+}
+
+// Two E2M1 codes (low nibble = element 0) times `scale`, as bf16x2.
+__device__ __forceinline__ uint32_t e2m1x2_scaled_bf16x2(uint32_t byte, float scale) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\tmov.b16 {t, _}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2)
+      : "h"(static_cast<unsigned short>(byte & 0xFFu)));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  return pack_bf16x2(f.x * scale, f.y * scale);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 struct ExTile {
   int expert, row0, ntok, n_mma, wt;
 };
@@ -191,16 +231,22 @@ __device__ __forceinline__ ExTile ex_decode(int w, int num_tiles, const ExParams
   return t;
 }
 
-template <int EPI, bool PAIRED, int CG>
-__global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_constant__ ExMaps maps, const ExParams p) {
+template <int EPI, bool PAIRED, int CG, bool MX>
+__global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
+    tc_expert_kernel(const __grid_constant__ ExMaps maps, const ExParams p) {
+  constexpr int EX_STAGES = ExCfg<MX>::kStages;
   extern __shared__ uint8_t ex_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ex_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + EX_STAGES * EX_A_BYTES;
-  float* xch = reinterpret_cast<float*>(sB + EX_STAGES * EX_B_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + EX_STAGES * EX_B_BYTES + EX_XCH_BYTES);
+  uint8_t* sQ = sB + EX_STAGES * EX_B_BYTES;                       // MX codes
+  uint8_t* sS = sQ + (MX ? EX_STAGES * EX_CODES_BYTES : 0u);       // MX scales
+  float* xch = reinterpret_cast<float*>(sS + (MX ? EX_STAGES * EX_SCALES_BYTES : 0u));
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + EX_XCH_BYTES);
   uint64_t* empty = full + EX_STAGES;
-  uint64_t* acc_full = empty + EX_STAGES;
+  uint64_t* raw = empty + EX_STAGES;     // MX: local codes + scales landed
+  uint64_t* conv = raw + EX_STAGES;      // MX: both CTAs' A tiles converted (even CTA's copy counts)
+  uint64_t* acc_full = conv + EX_STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -218,6 +264,8 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
     for (int s = 0; s < EX_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&raw[s], 1);
+      mbar_init(&conv[s], CG * EX_CONV_WARPS);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
@@ -230,6 +278,10 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&maps.a0);
     if (PAIRED) tma_prefetch_desc(&maps.a1);
+    if (MX) {
+      tma_prefetch_desc(&maps.s0);
+      if (PAIRED) tma_prefetch_desc(&maps.s1);
+    }
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&maps.b[i]);
   }
   if (warp == 1) ex_tmem_alloc<CG>(tmem_holder);
@@ -260,7 +312,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
       auto prefetch_next = [&]() {
         if (pf_w >= total) return;
         if (pf_row < 0) pf_row = weight_row(ex_decode(pf_w, num_tiles, p));
-        const int kc = pf_kb * EX_BK;
+        const int kc = pf_kb * (MX ? EX_BK / 2 : EX_BK);  // MX codes: 32 bytes per row and k-block
         tma_prefetch_l2_2d(&maps.a0, kc, pf_row);
         if (PAIRED) tma_prefetch_l2_2d(&maps.a1, kc, pf_row);
         if (++pf_kb == p.num_k_blocks) {
@@ -280,7 +332,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
         const int bsel = rows_cta > 64 ? 0 : rows_cta > 32 ? 1 : rows_cta > 16 ? 2 : 3;
         const int brows = 128 >> bsel;
         const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
-        const uint32_t bytes = static_cast<uint32_t>(CG) * (EX_A_BYTES + brows * EX_BK * 2);
+        const uint32_t bytes = static_cast<uint32_t>(CG) * ((MX ? 0u : EX_A_BYTES) + brows * EX_BK * 2);
         const int wrow = weight_row(t);  // first weight row of this CTA
         for (int kb = 0; kb < p.num_k_blocks; ++kb) {
           prefetch_next();
@@ -292,7 +344,22 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
           const int kc = kb * EX_BK;
           uint8_t* a_dst = sA + stage * EX_A_BYTES;
           uint8_t* b_dst = sB + stage * EX_B_BYTES;
-          if (PAIRED) {
+          if constexpr (MX) {
+            // codes and scales of this CTA's rows, to its own staging slot
+            uint8_t* q_dst = sQ + stage * EX_CODES_BYTES;
+            uint8_t* s_dst = sS + stage * EX_SCALES_BYTES;
+            const int sc0 = (kb >> 3) * 16;  // 16 scale bytes = 8 k-blocks per box
+            mbar_arrive_expect_tx(&raw[stage], EX_CODES_BYTES + EX_SCALES_BYTES);
+            if (PAIRED) {
+              tma_load_2d(q_dst, &maps.a0, &raw[stage], kb * 32, wrow);
+              tma_load_2d(q_dst + EX_CODES_BYTES / 2, &maps.a1, &raw[stage], kb * 32, wrow);
+              tma_load_2d(s_dst, &maps.s0, &raw[stage], sc0, wrow);
+              tma_load_2d(s_dst + EX_SCALES_BYTES / 2, &maps.s1, &raw[stage], sc0, wrow);
+            } else {
+              tma_load_2d(q_dst, &maps.a0, &raw[stage], kb * 32, wrow);
+              tma_load_2d(s_dst, &maps.s0, &raw[stage], sc0, wrow);
+            }
+          } else if (PAIRED) {
             ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
             ex_tma_load<CG>(a_dst + EX_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
           } else {
@@ -309,10 +376,13 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
       }
       // The even CTA's barriers count both CTAs' bytes: it waits for every
       // load of the pair to land before the pair may exit.
-      if (leader) {
+      {
         volatile int never = 0;
-        for (int s = 0; s < EX_STAGES; ++s)
-          if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_parity >> s) & 1u, &never, p.fault_site + 2);
+        for (int s = 0; s < EX_STAGES; ++s) {
+          if (!((issued >> s) & 1u)) continue;
+          if (leader) mbar_wait(&full[s], (issued_parity >> s) & 1u, &never, p.fault_site + 2);
+          if (MX) mbar_wait(&raw[s], (issued_parity >> s) & 1u, &never, p.fault_site + 2);
+        }
       }
     }
   } else if (warp == 1) {
@@ -330,7 +400,8 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * EX_ACC_COLS);
         for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort, p.fault_site + 4)) {
+          if (!mbar_wait(&full[stage], phase, abort, p.fault_site + 4) ||
+              (MX && !mbar_wait(&conv[stage], phase, abort, p.fault_site + 7))) {
             ok = false;
             break;
           }
@@ -362,6 +433,50 @@ __global__ void __launch_bounds__(EX_THREADS, 1) tc_expert_kernel(const __grid_c
       mbar_wait(drain, 0u, &never, p.fault_site + 5);
     }
     __syncwarp();
+  } else if (MX && warp >= 6) {
+    // ------------------------------------------------------------------ MXFP4 converters (both CTAs)
+    // thread = one 32-element MX block: row r of the A tile, K half h
+    const int ct = threadIdx.x - 192;
+    const int r = ct >> 1, h = ct & 1;
+    const uint32_t conv_leader = CG == 2 ? map_to_rank(smem_u32(&conv[0]), 0u) : smem_u32(&conv[0]);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int w = pair; w < total && ok; w += npairs) {
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&raw[stage], phase, abort, p.fault_site + 8))) {
+          ok = false;
+          break;
+        }
+        const uint4 q = *reinterpret_cast<const uint4*>(sQ + stage * EX_CODES_BYTES + r * 32 + h * 16);
+        const float sc = e8m0_to_f32(sS[stage * EX_SCALES_BYTES + r * 16 + (kb & 7) * 2 + h]);
+        uint32_t o[16];
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) o[4 * i + j] = e2m1x2_scaled_bf16x2(words[i] >> (8 * j), sc);
+        // 64 bytes = chunks 4h .. 4h+3 of row r, 128-byte swizzle
+        uint8_t* arow = sA + stage * EX_A_BYTES + r * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = (4 * h + c) ^ (r & 7);
+          *reinterpret_cast<uint4*>(arow + chunk * 16) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        }
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2)
+            mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+          else
+            mbar_arrive(&conv[stage]);
+        }
+        if (++stage == EX_STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quarter of this warp

@@ -47,7 +47,13 @@ bool dims_ok(const moe_dims* d) {
 
 // Valid dims that this build does not implement.
 bool dims_supported(const moe_dims* d) {
-  if (d->routed != d->act) return false;  // block-scaled routed weights: not in this build
+  if (d->routed == MOE_MXFP4) {
+    // MXFP4 routed weights: bf16 activations; code and scale rows must suit TMA
+    // (K/2 and K/32 bytes per row, multiples of 16) for both expert GEMMs.
+    if (d->act != MOE_BF16 || d->L % 512 != 0 || d->I % 512 != 0) return false;
+  } else if (d->routed != d->act) {
+    return false;
+  }
   if (d->L > 4 * COMBINE_THREADS * 16) return false;
   if (d->act == MOE_BF16) {
     if (d->H % 64 || d->L % 64 || d->I % 64) return false;
@@ -148,6 +154,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// uint8 matrix [rows, cols] (cols in bytes), box box_rows x box_cols bytes, no
+// swizzle (MXFP4 codes and scales).
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                 uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -372,15 +393,15 @@ bool make_token_maps(CUtensorMap* maps4, const void* base, uint64_t rows, uint64
   return true;
 }
 
-template <int EPI, bool PAIRED, int CG>
+template <int EPI, bool PAIRED, int CG, bool MX>
 cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream_t s) {
-  auto kern = tc_expert_kernel<EPI, PAIRED, CG>;
+  auto kern = tc_expert_kernel<EPI, PAIRED, CG, MX>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(EX_SMEM_BYTES));
+                                       static_cast<int>(ExCfg<MX>::kSmem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(EX_THREADS);
-  cfg.dynamicSmemBytes = EX_SMEM_BYTES;
+  cfg.blockDim = dim3(ExCfg<MX>::kThreads);
+  cfg.dynamicSmemBytes = ExCfg<MX>::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   if (CG == 2) {
@@ -391,7 +412,7 @@ cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // One pair per two SMs that can co-schedule a cluster (asked once per device).
-    static int pairs_cache[128] = {};
+    static int pairs_cache[128] = {};  // per instantiation and device
     int dev = 0;
     cudaGetDevice(&dev);
     int pairs = dev >= 0 && dev < 128 ? pairs_cache[dev] : 0;
@@ -411,8 +432,12 @@ cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream
 }
 
 template <int EPI, bool PAIRED>
-cudaError_t launch_expert(int cg, const ExMaps& maps, const ExParams& p, cudaStream_t s) {
-  return cg == 2 ? launch_expert_inst<EPI, PAIRED, 2>(maps, p, s) : launch_expert_inst<EPI, PAIRED, 1>(maps, p, s);
+cudaError_t launch_expert(int cg, bool mx, const ExMaps& maps, const ExParams& p, cudaStream_t s) {
+  if (mx)
+    return cg == 2 ? launch_expert_inst<EPI, PAIRED, 2, true>(maps, p, s)
+                   : launch_expert_inst<EPI, PAIRED, 1, true>(maps, p, s);
+  return cg == 2 ? launch_expert_inst<EPI, PAIRED, 2, false>(maps, p, s)
+                 : launch_expert_inst<EPI, PAIRED, 1, false>(maps, p, s);
 }
 
 moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const void* z_perm,
@@ -438,12 +463,17 @@ moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const v
     return run_gemm_simt(g, s);
   }
   const int cg = expert_cg(d);
+  const bool mx = d.routed == MOE_MXFP4;
   ExMaps maps;
   std::memset(&maps, 0, sizeof maps);
   const uint64_t wrows = static_cast<uint64_t>(d.E) * d.I;
-  if (!make_map(&maps.a0, w.Wg, wrows, d.L, d.L, 64) || !make_map(&maps.a1, w.Wv, wrows, d.L, d.L, 64) ||
-      !make_token_maps(maps.b, z_perm, static_cast<uint64_t>(R), d.L))
-    return MOE_ERR_CUDA;
+  bool ok = make_token_maps(maps.b, z_perm, static_cast<uint64_t>(R), d.L);
+  if (mx)
+    ok = ok && make_map_u8(&maps.a0, w.Wg, wrows, d.L / 2, 32, 64) && make_map_u8(&maps.a1, w.Wv, wrows, d.L / 2, 32, 64) &&
+         make_map_u8(&maps.s0, w.Sg, wrows, d.L / 32, 16, 64) && make_map_u8(&maps.s1, w.Sv, wrows, d.L / 32, 16, 64);
+  else
+    ok = ok && make_map(&maps.a0, w.Wg, wrows, d.L, d.L, 64) && make_map(&maps.a1, w.Wv, wrows, d.L, d.L, 64);
+  if (!ok) return MOE_ERR_CUDA;
   ExParams p{};
   p.tile_table = tile_table;
   p.num_tiles_dev = num_tiles;
@@ -455,7 +485,7 @@ moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const v
   p.out_cols = d.I;
   p.situ_c = d.situ_c;
   p.fault_site = 140;
-  return launch_expert<kEpiSituBF16, true>(cg, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_expert<kEpiSituBF16, true>(cg, mx, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void* h_perm, const int4* tile_table,
@@ -479,11 +509,16 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
     return run_gemm_simt(g, s);
   }
   const int cg = expert_cg(d);
+  const bool mx = d.routed == MOE_MXFP4;
   ExMaps maps;
   std::memset(&maps, 0, sizeof maps);
-  if (!make_map(&maps.a0, w.Wo, static_cast<uint64_t>(d.E) * d.L, d.I, d.I, 128) ||
-      !make_token_maps(maps.b, h_perm, static_cast<uint64_t>(R), d.I))
-    return MOE_ERR_CUDA;
+  const uint64_t wrows = static_cast<uint64_t>(d.E) * d.L;
+  bool ok = make_token_maps(maps.b, h_perm, static_cast<uint64_t>(R), d.I);
+  if (mx)
+    ok = ok && make_map_u8(&maps.a0, w.Wo, wrows, d.I / 2, 32, 128) && make_map_u8(&maps.s0, w.So, wrows, d.I / 32, 16, 128);
+  else
+    ok = ok && make_map(&maps.a0, w.Wo, wrows, d.I, d.I, 128);
+  if (!ok) return MOE_ERR_CUDA;
   ExParams p{};
   p.tile_table = tile_table;
   p.num_tiles_dev = num_tiles;
@@ -495,7 +530,7 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
   p.out_cols = d.L;
   p.situ_c = d.situ_c;
   p.fault_site = 150;
-  return launch_expert<kEpiF32, false>(cg, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_expert<kEpiF32, false>(cg, mx, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 template <typename OutT>
@@ -547,6 +582,17 @@ moe_status stage_output(const moe_dims& d, const moe_weights& w, const void* h_s
   g.situ_c = d.situ_c;
   g.fault_site = 160;
   return run_gemm(d, g, s);
+}
+
+// MXFP4 routed weights need their E8M0 scale arrays; other types take none.
+moe_status check_scales(const moe_dims& d, const moe_weights& w) {
+  const bool mx = d.routed == MOE_MXFP4;
+  const void* sc[] = {w.Sg, w.Sv, w.So};
+  for (const void* p : sc) {
+    if (mx && (p == nullptr || !aligned16(p))) return MOE_ERR_INVALID_ARG;
+    if (!mx && p != nullptr) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
 }
 
 bool ws_ok(const moe_dims& d, const void* ws, size_t ws_bytes) {
@@ -629,6 +675,7 @@ moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z
   if (!aligned16(w->Wg) || !aligned16(w->Wv) || !aligned16(w->Wo) || w->Wg == nullptr || w->Wv == nullptr ||
       w->Wo == nullptr || !aligned16(z_perm) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
+  if ((st = check_scales(*d, *w)) != MOE_OK) return st;
   if (!ws_ok(*d, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
   g_last_launches = 0;
   if (d->T == 0) return MOE_OK;
@@ -668,7 +715,7 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
   if (d->S > 0 && (w->Wsg == nullptr || w->Wsv == nullptr || w->Wso == nullptr || !aligned16(w->Wsg) ||
                    !aligned16(w->Wsv) || !aligned16(w->Wso)))
     return MOE_ERR_INVALID_ARG;
-  if (w->Sg != nullptr || w->Sv != nullptr || w->So != nullptr) return MOE_ERR_UNSUPPORTED;
+  if ((st = check_scales(*d, *w)) != MOE_OK) return st;
   moe_aux a{};
   if (aux != nullptr) a = *aux;
   const void* auxp[] = {a.scores, a.topk_idx, a.topk_w, a.expert_offsets, a.u, a.n, a.z};

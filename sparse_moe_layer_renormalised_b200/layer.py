@@ -14,14 +14,15 @@ _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 class MoeLayer:
     """Weights: dict with Wr, bias, Wdown, Wup, gamma, Wg, Wv, Wo, Wsg, Wsv, Wso
-    (device tensors in the shapes of include/moe.h).  max_tokens sizes the
+    and, for MXFP4 routed weights, Sg, Sv, So (device tensors in the shapes of
+    include/moe.h).  max_tokens sizes the
     workspace; each call may use any T <= max_tokens."""
 
     def __init__(self, dims: Dims, weights: dict, max_tokens: int | None = None):
         self.dims = dims
         self.weights = weights
         self.max_tokens = dims.T if max_tokens is None else max_tokens
-        self._w = make_weights(**{k: v for k, v in weights.items() if not k.endswith("_scale")})
+        self._w = make_weights(**weights)
         dev = weights["Wr"].device
         nbytes = moe_workspace_size(replace(dims, T=self.max_tokens))
         if nbytes == 0:

@@ -60,7 +60,8 @@ FAKE = 1 << 20  # an aligned address; never dereferenced because validation fail
     (dict(L=1020), moe.MOE_ERR_INVALID_ARG),
     (dict(situ_c=0.0), moe.MOE_ERR_INVALID_ARG),
     (dict(y_out="mxfp4"), moe.MOE_ERR_INVALID_ARG),
-    (dict(routed="mxfp4"), moe.MOE_ERR_UNSUPPORTED),
+    (dict(routed="mxfp4"), moe.MOE_ERR_UNSUPPORTED),  # L = 1024 fine, I = 768 not a multiple of 512
+    (dict(routed="mxfp4", act="f32", y_out="f32"), moe.MOE_ERR_UNSUPPORTED),
     (dict(H=2056), moe.MOE_ERR_UNSUPPORTED),
     (dict(S=4), moe.MOE_ERR_UNSUPPORTED),
 ])
@@ -86,8 +87,13 @@ def test_bad_pointers_rejected():
     assert moe.moe_layer_forward(d, w, FAKE, FAKE, None, FAKE, ws - 1, 0) == moe.MOE_ERR_INVALID_ARG  # ws size
     aux = moe.make_aux(u=FAKE + 4)
     assert moe.moe_layer_forward(d, w, FAKE, FAKE, aux, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
-    w_scaled = moe.make_weights(**{**full, "Sg": FAKE})
-    assert moe.moe_layer_forward(d, w_scaled, FAKE, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_UNSUPPORTED
+    w_scaled = moe.make_weights(**{**full, "Sg": FAKE})  # scales with bf16 weights
+    assert moe.moe_layer_forward(d, w_scaled, FAKE, FAKE, None, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
+    dm = _dims(I=1024, routed="mxfp4")
+    wsm = moe.moe_workspace_size(dm)
+    assert moe.moe_layer_forward(dm, w, FAKE, FAKE, None, FAKE, wsm, 0) == moe.MOE_ERR_INVALID_ARG  # no scales
+    wm = moe.make_weights(**{**full, "Sg": FAKE, "Sv": FAKE, "So": FAKE + 4})
+    assert moe.moe_layer_forward(dm, wm, FAKE, FAKE, None, FAKE, wsm, 0) == moe.MOE_ERR_INVALID_ARG  # misaligned
 
 
 def test_stage_entry_points_validate():

@@ -179,3 +179,33 @@ def test_expert_ffn_same_gate_and_up_weights():
         Wg, _, Wo = oin.expert_weights(cfg, e)
         ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wg, Wo, cfg.situ_c, oracle.bf16_round)
     assert parity(y_perm.cpu().to(F64), ref) <= 1e-2
+
+
+@pytest.mark.parametrize("T", [300, 40])
+def test_expert_ffn_mxfp4(T):
+    """Routed experts with MXFP4 weights against the oracle, which decodes the
+    same bits (E2M1 codes x E8M0 scales) to fp64."""
+    cfg = gen.CONFIGS["mxfp4-small"].with_(T=T)
+    E, k, L, I = cfg.E, cfg.k, cfg.L, cfg.I
+    d = dims_for(cfg, T=T)
+    w = gen.device_layer(cfg, "cuda", with_x=False)
+    idx = _routing(T, E, k, True, 21)
+    _, offsets, _, _ = oracle.permute(idx.numpy(), E)
+    R = T * k
+    z_perm = torch.randn(R, L, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    y_perm = torch.full((R, L), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(moe.moe_workspace_size(d), dtype=torch.uint8, device="cuda")
+    wts = moe.make_weights(Wg=w["Wg"], Wv=w["Wv"], Wo=w["Wo"], Sg=w["Sg"], Sv=w["Sv"], So=w["So"])
+    off = torch.as_tensor(offsets, dtype=torch.int32).cuda()
+    assert moe.moe_expert_ffn(d, wts, z_perm.cuda(), off, y_perm, ws) == moe.MOE_OK
+    torch.cuda.synchronize()
+    _no_fault()
+    zf = z_perm.to(F64)
+    ref = torch.empty(R, L, dtype=F64)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        Wg, Wv, Wo = oin.expert_weights(cfg, e)
+        ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wv, Wo, cfg.situ_c, oracle.bf16_round)
+    assert parity(y_perm.cpu().to(F64), ref) <= 1e-2

@@ -7,7 +7,7 @@ import torch
 
 import gen
 import sparse_moe_layer_renormalised_b200 as moe
-from harness import (TOL_BF16, TOL_F32, compare_layer, make_device_layer, moe_inputs_rows, oracle_forward,
+from harness import (TOL_BF16, TOL_F32, TOL_MXFP4, compare_layer, make_device_layer, moe_inputs_rows, oracle_forward,
                      run_layer)
 
 pytestmark = pytest.mark.gpu
@@ -74,6 +74,16 @@ def test_mid_ragged_token_counts(mid_layer, T):
     _report(f"mid T={T}", m)
 
 
+def test_mxfp4_layer_all_tokens():
+    """The whole layer with MXFP4 routed weights (bar 3e-2; the oracle decodes
+    the same bits, so the error budget is that of the bf16 layer)."""
+    cfg = gen.CONFIGS["mxfp4-small"]
+    layer, w = make_device_layer(cfg)
+    y, aux = run_layer(layer, w["x"])
+    m = compare_layer(cfg, np.arange(cfg.T), y, aux, TOL_MXFP4)
+    _report("mxfp4-small", m)
+
+
 def test_zero_tokens_is_a_no_op(mid_layer):
     cfg, layer, w = mid_layer
     y = torch.full((1, cfg.H), 7.0, device="cuda")
@@ -109,3 +119,15 @@ def test_k3_decode_and_prefill_sampled():
     tokens = np.arange(min(dec.T, K3_SAMPLE))
     m = compare_layer(dec, tokens, y, aux, TOL_BF16)
     _report("decode", m)
+
+
+@pytest.mark.slow
+def test_k3_mxfp4_sampled():
+    """K3 shape with MXFP4 routed weights at the full T = 8192, seeded sample of
+    tokens checked against the oracle decoding the same bits."""
+    cfg = gen.CONFIGS["mxfp4"]
+    layer, w = make_device_layer(cfg)
+    y, aux = run_layer(layer, w["x"])
+    tokens = gen.sample_tokens(cfg, min(K3_SAMPLE, cfg.T))
+    m = compare_layer(cfg, tokens, y, aux, TOL_MXFP4)
+    _report("mxfp4", m)
