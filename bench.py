@@ -245,6 +245,8 @@ def run_ours(args, rank, world, local_rank):
     traffic = None
     prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}_{dom}.json")
     if os.path.exists(prof):
+        # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu
+        # capture of this workload (see the file for the command and kernel build)
         with open(prof) as f:
             traffic = json.load(f).get("dram_bytes_per_launch")
     out = {
@@ -274,7 +276,7 @@ def run_ours(args, rank, world, local_rank):
         "tflops": round(flops_step / (ms_per_step / 1e3) / 1e12, 2),
         "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
         "roofline": {
-            "kernel": f"tc_gemm_kernel (grouped, paired gate/up + SiTU epilogue) = stage {dom}",
+            "kernel": f"tc_expert_kernel (2-CTA grouped gate/up + SiTU epilogue) = stage {dom}",
             "bound": bound,
             "achieved": round(achieved, 1),
             "peak": peak,
