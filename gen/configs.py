@@ -68,6 +68,9 @@ CONFIGS: dict[str, LayerConfig] = {
     # captures stay small; not a measured workload.
     "prefill-e64": LayerConfig("prefill-e64", T=1024, H=7168, L=3584, E=64, k=16, I=3072, S=2, Is=3072, bias="zipf",
                                oracle_tokens=64),
+    # The same stand-in with MXFP4 routed weights (1.1 GB of codes and scales).
+    "mxfp4-e64": LayerConfig("mxfp4-e64", T=1024, H=7168, L=3584, E=64, k=16, I=3072, S=2, Is=3072, bias="zipf",
+                             routed="mxfp4", oracle_tokens=64),
 }
 
 # Tensor ids: the second half of the Philox key of each input tensor.

@@ -393,6 +393,23 @@ bool make_token_maps(CUtensorMap* maps4, const void* base, uint64_t rows, uint64
   return true;
 }
 
+// One CTA pair per two SMs that can co-schedule a cluster of `kern`, asked
+// once per device and kernel.
+template <typename K>
+int cluster_pairs(K kern, cudaLaunchConfig_t cfg, int* cache) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int pairs = dev >= 0 && dev < 128 ? cache[dev] : 0;
+  if (pairs == 0) {
+    cfg.gridDim = dim3(2 * 74);
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess || nc <= 0) nc = num_sms() / 2;
+    pairs = nc;
+    if (dev >= 0 && dev < 128) cache[dev] = pairs;
+  }
+  return pairs;
+}
+
 template <int EPI, bool PAIRED, int CG, bool MX>
 cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream_t s) {
   auto kern = tc_expert_kernel<EPI, PAIRED, CG, MX>;
@@ -411,19 +428,8 @@ cudaError_t launch_expert_inst(const ExMaps& maps, const ExParams& p, cudaStream
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // One pair per two SMs that can co-schedule a cluster (asked once per device).
     static int pairs_cache[128] = {};  // per instantiation and device
-    int dev = 0;
-    cudaGetDevice(&dev);
-    int pairs = dev >= 0 && dev < 128 ? pairs_cache[dev] : 0;
-    if (pairs == 0) {
-      cfg.gridDim = dim3(2 * 74);
-      int nc = 0;
-      if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess || nc <= 0) nc = num_sms() / 2;
-      pairs = nc;
-      if (dev >= 0 && dev < 128) pairs_cache[dev] = pairs;
-    }
-    cfg.gridDim = dim3(2 * pairs);
+    cfg.gridDim = dim3(2 * cluster_pairs(kern, cfg, pairs_cache));
   } else {
     cfg.gridDim = dim3(num_sms());
     cfg.numAttrs = 0;
