@@ -444,13 +444,25 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
           const int chunk = (4 * h + c) ^ (r & 7);
           *reinterpret_cast<uint4*>(arow + chunk * 16) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
         }
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
-        __syncwarp();
-        if (lane == 0) {
-          if (CG == 2)
-            mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(stage * sizeof(uint64_t)));
-          else
-            mbar_arrive(&conv[stage]);
+        // The proxy fence that hands these generic-proxy writes to the tensor
+        // cores is the converters' dominant stall (ncu: membar), so it is paid
+        // once per two k-blocks: after the odd one, both slots are released
+        // together.  Every item has an even number of k-blocks (K is a
+        // multiple of 512), and the slot of the odd k-block never waits on the
+        // even one's release, so the delay cannot deadlock.
+        if (kb & 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int prev = stage == 0 ? EX_STAGES - 1 : stage - 1;
+            if (CG == 2) {
+              mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(prev * sizeof(uint64_t)));
+              mbar_arrive_cluster(conv_leader + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+            } else {
+              mbar_arrive(&conv[prev]);
+              mbar_arrive(&conv[stage]);
+            }
+          }
         }
         if (++stage == EX_STAGES) {
           stage = 0;
