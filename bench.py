@@ -141,6 +141,44 @@ def stage_work(cfg, offsets: np.ndarray, T: int) -> dict:
     return {"flops": flops, "bytes": bytes_, "touched_experts": touched}
 
 
+def measure_qb(cfg, dev, stream, peaks: dict, reps: int = 10) -> dict:
+    """The Quantile Balancing bias update (the training-time step beside the
+    router) on a [T, E] score batch of this workload's shape, timed on its
+    own with CUDA events; L2 is flushed (a 256 MB write) before every call,
+    since the scores alone would fit in it.  Not part of the layer step."""
+    nb, lo, hi = 1024, -1.5, 1.5
+    s = torch.from_numpy(gen.qb_scores(cfg)).to(dev)
+    b = torch.from_numpy(gen.bias(cfg)).to(dev)
+    out = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+    hist = torch.empty(cfg.E * nb, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    d = dims_for(cfg, "f32")
+
+    def call():
+        moe.check(moe.moe_qb_bias_update(d, s, b, out, None, hist, nb, lo, hi, stream))
+
+    for _ in range(3):
+        call()
+    total = 0.0
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    ms = total / reps
+    # scores read, histogram zeroed and read back, bias in / out
+    nbytes = cfg.T * cfg.E * 4 + 2 * cfg.E * nb * 4 + 2 * cfg.E * 4
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": "qb_zero_kernel + qb_hist_kernel + qb_quantile_kernel", "ms": round(ms, 4), "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes, "bins": nb,
+            "scores": f"[{cfg.T}, {cfg.E}] fp32, uniform in [0, 1); target floor(T k / E) = {cfg.T * cfg.k // cfg.E}"}
+
+
 # ----------------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     cfg = gen.CONFIGS[args.config]
@@ -295,6 +333,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    out["qb_update"] = measure_qb(cfg, dev, stream, peaks)
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, seed_offset=0)
     return out

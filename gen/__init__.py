@@ -35,6 +35,7 @@ __all__ = [
     "bias",
     "gamma",
     "sample_tokens",
+    "qb_scores",
     "device_layer",
     "philox4x32_10",
 ]
@@ -196,6 +197,14 @@ def bias(cfg: LayerConfig) -> np.ndarray:
     if cfg.bias == "zipf":
         return zipf_bias(cfg.E, cfg.k, cfg.zipf_s, cfg.seed)
     return fill_host(cfg.seed, TID["bias"], 0, cfg.E, cfg.bias_std, 0.0, "f32")
+
+
+def qb_scores(cfg: LayerConfig) -> np.ndarray:
+    """Router-score stand-in [T, E] for the Quantile Balancing step: uniform
+    fp32 values in [0, 1) with 24 random bits each (Philox words >> 8, times
+    2^-24, exact in fp32)."""
+    words = u32_words(cfg.seed, TID["qb_scores"], 0, cfg.T * cfg.E)
+    return ((words >> 8).astype(np.float32) * np.float32(2.0 ** -24)).reshape(cfg.T, cfg.E)
 
 
 def sample_tokens(cfg: LayerConfig, n: int | None = None) -> np.ndarray:

@@ -89,6 +89,7 @@ TID = {
     "Wso": 12,
     "zipf_perm": 13,
     "sample": 14,
+    "qb_scores": 15,
 }
 
 

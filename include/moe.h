@@ -225,6 +225,32 @@ MOE_API moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk_id
                                        int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
                                        void* z_perm, moe_stream_t stream);
 
+/* Quantile Balancing bias update: the training-time step beside the router
+ * ("Kimi K3の896エキスパート…", section 「ルーター専用の独立訓練はない」: each
+ * expert's selection bias is updated from the boundary, read off quantiles of
+ * the router scores, at which it receives its target number of tokens; Kimi
+ * K3 tech-report summary, section 「幅のスケーリング：Stable LatentMoE」: the
+ * quantiles come from a histogram of the router's score margins).
+ *  - scores [T, E] fp32 (the router's sigmoid scores, e.g. moe_router_topk's
+ *    scores_out), bias_in [E] fp32: the current bias.  Uses d->T, d->E, d->k
+ *    only (2 <= E <= 1024, 0 < k < E, 1 <= floor(T*k/E) < T).
+ *  - Margin of expert e for token t: fl32(s + b_e) minus the k-th largest key
+ *    fl32(s + b) among the token's OTHER experts (ties rank the lower index
+ *    first); e is selected exactly when its margin is positive.
+ *  - hist [E, nbins] uint32: caller-owned workspace, overwritten with the
+ *    per-expert margin histogram on [lo, hi) (nbins equal bins, a multiple of
+ *    32 in [32, 65536]; margins outside go to the end bins; the bin index is
+ *    floor(fl32(fl32(m - lo) * fl32(nbins / (hi - lo))))).
+ *  - bias_out[e] = bias_in[e] - q[e], with q[e] the rank-c boundary of e's
+ *    margins, c = floor(T*k/E), read from the histogram with the margins
+ *    spread evenly within a bin; quantile_out [E] (may be NULL) receives q.
+ *    bias_out may alias bias_in.
+ *  - Errors: MOE_ERR_INVALID_ARG for bad dims, bins or range, NULL or
+ *    misaligned (4-byte) pointers; MOE_ERR_CUDA for a failed launch. */
+MOE_API moe_status moe_qb_bias_update(const moe_dims* d, const float* scores, const float* bias_in, float* bias_out,
+                                      float* quantile_out, uint32_t* hist, int32_t nbins, float lo, float hi,
+                                      moe_stream_t stream);
+
 /* Human-readable name of a status. */
 MOE_API const char* moe_status_str(moe_status s);
 

@@ -31,6 +31,7 @@ from ._binding import (  # noqa: F401
     moe_layer_forward,
     moe_permute,
     moe_permute_noalloc,
+    moe_qb_bias_update,
     MOE_PERMUTE_NOALLOC_SCRATCH_BYTES,
     moe_router_topk,
     moe_status_str,

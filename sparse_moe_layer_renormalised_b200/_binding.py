@@ -31,6 +31,7 @@ EXPORTED = (
     "moe_device_error",
     "moe_last_launch_count",
     "moe_permute_noalloc",
+    "moe_qb_bias_update",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -100,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.moe_device_error.argtypes = [ctypes.POINTER(i32), vp]
         L.moe_last_launch_count.argtypes = []
         L.moe_permute_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp]
+        f32 = ctypes.c_float
+        L.moe_qb_bias_update.argtypes = [pd, vp, vp, vp, vp, vp, i32, f32, f32, vp]
         for f in EXPORTED:
             if f not in ("moe_workspace_size", "moe_status_str"):
                 getattr(L, f).restype = i32
@@ -217,6 +220,14 @@ def moe_permute_noalloc(d, topk_idx, z, expert_offsets, perm_token, inv_perm, z_
     scratch is a fixed array inside the library (see include/moe.h)."""
     return lib().moe_permute_noalloc(ctypes.byref(_dims(d)), _ptr(topk_idx), _ptr(z), _ptr(expert_offsets),
                                      _ptr(perm_token), _ptr(inv_perm), _ptr(z_perm), _stream(stream))
+
+
+def moe_qb_bias_update(d, scores, bias_in, bias_out, quantile_out, hist, nbins: int, lo: float, hi: float,
+                       stream=None) -> int:
+    """Quantile Balancing bias update from a batch of router scores (see
+    include/moe.h); hist is an [E, nbins] uint32 workspace, overwritten."""
+    return lib().moe_qb_bias_update(ctypes.byref(_dims(d)), _ptr(scores), _ptr(bias_in), _ptr(bias_out),
+                                    _ptr(quantile_out), _ptr(hist), int(nbins), float(lo), float(hi), _stream(stream))
 
 
 def moe_status_str(status: int) -> str:

@@ -15,6 +15,7 @@
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 #include "routing.cuh"
+#include "qb.cuh"
 #include "../../include/moe.h"
 
 namespace moe {
@@ -902,4 +903,32 @@ extern "C" moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   if (z != nullptr) st = stage_gather(*d, z, z_perm, perm_token, expert_offsets + d->E, s);
   return st;
+}
+
+extern "C" moe_status moe_qb_bias_update(const moe_dims* d, const float* scores, const float* bias_in, float* bias_out,
+                                         float* quantile_out, uint32_t* hist, int32_t nbins, float lo, float hi,
+                                         moe_stream_t stream) {
+  using namespace moe;
+  if (d == nullptr || scores == nullptr || bias_in == nullptr || bias_out == nullptr || hist == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  const long long T = d->T;
+  const int E = d->E, k = d->k;
+  if (T < 1 || E < 2 || E > 1024 || k < 1 || k >= E) return MOE_ERR_INVALID_ARG;
+  const long long c = T * k / E;
+  if (c < 1 || c >= T) return MOE_ERR_INVALID_ARG;
+  if (nbins < 32 || nbins > 65536 || nbins % 32 != 0) return MOE_ERR_INVALID_ARG;
+  if (!(lo < hi) || !std::isfinite(lo) || !std::isfinite(hi) || !std::isfinite(hi - lo)) return MOE_ERR_INVALID_ARG;
+  auto al4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+  if (!al4(scores) || !al4(bias_in) || !al4(bias_out) || !al4(hist) || (quantile_out && !al4(quantile_out)))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const double span = static_cast<double>(hi) - static_cast<double>(lo);
+  const float inv_w = static_cast<float>(nbins / span);
+  const float w = static_cast<float>(span / nbins);
+  const long long n = static_cast<long long>(E) * nbins;
+  qb_zero_kernel<<<static_cast<unsigned>(std::min<long long>(cdiv(n, 256), 1184)), 256, 0, s>>>(hist, n);
+  qb_hist_kernel<<<static_cast<unsigned>(cdiv(T, QB_WARPS)), QB_WARPS * 32, 0, s>>>(scores, bias_in, T, E, k, nbins,
+                                                                                      lo, inv_w, hist);
+  qb_quantile_kernel<<<E, 32, 0, s>>>(hist, E, nbins, c, lo, w, bias_in, bias_out, quantile_out);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

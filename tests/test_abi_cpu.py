@@ -25,7 +25,7 @@ def _dims(**kw):
 
 def test_library_exports_every_declared_symbol():
     names = _declared()
-    assert len(names) == 10
+    assert len(names) == 11
     lib = ctypes.CDLL(moe.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -107,6 +107,27 @@ def test_stage_entry_points_validate():
     assert moe.moe_expert_ffn(d, w, FAKE, FAKE, FAKE, FAKE, ws, 0) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_combine(d, FAKE, FAKE, FAKE, None, None, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_combine(d, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_qb_bias_update_validates():
+    """Bad dims, bins, range and pointers are rejected on the host (the
+    pointers are never dereferenced)."""
+    ok = dict(scores=FAKE, bias_in=FAKE, bias_out=FAKE, quantile_out=None, hist=FAKE, nbins=256, lo=-1.0, hi=1.0)
+
+    def call(d=None, **kw):
+        a = {**ok, **kw}
+        return moe.moe_qb_bias_update(d or _dims(), a["scores"], a["bias_in"], a["bias_out"], a["quantile_out"],
+                                      a["hist"], a["nbins"], a["lo"], a["hi"], 0)
+
+    assert call(d=_dims(E=1, k=1)) == moe.MOE_ERR_INVALID_ARG       # k must be < E
+    assert call(d=_dims(E=2048)) == moe.MOE_ERR_INVALID_ARG         # E > 1024
+    assert call(d=_dims(T=4, E=128, k=8)) == moe.MOE_ERR_INVALID_ARG  # target floor(T k / E) = 0
+    assert call(nbins=100) == moe.MOE_ERR_INVALID_ARG                # not a multiple of 32
+    assert call(nbins=1 << 17) == moe.MOE_ERR_INVALID_ARG
+    assert call(lo=1.0, hi=1.0) == moe.MOE_ERR_INVALID_ARG
+    assert call(hi=float("inf")) == moe.MOE_ERR_INVALID_ARG
+    assert call(hist=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(scores=FAKE + 2) == moe.MOE_ERR_INVALID_ARG           # misaligned
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
