@@ -35,8 +35,10 @@ notes):
     spread evenly inside a bin: if A margins lie in the bins above bin j and
     bin j (lower edge lo + j*w) holds n_j of them with A < c <= A + n_j,
     then q = lo + w * (j + 1 - (c - A) / n_j).  The exact quantile (the
-    midpoint of the c-th and (c+1)-th largest margin) is given too; the two
-    differ by at most one bin width when the c-th margin lies inside [lo, hi).
+    midpoint of the c-th and (c+1)-th largest margin) is given too; when the
+    c-th margin lies inside [lo, hi) the two differ by at most one bin width
+    plus half the gap between the c-th and (c+1)-th margins (q lies in the
+    c-th margin's bin).
   * Binning decides an integer from floating point, so it is written as the
     device evaluates it, in fp32: bin = clamp(floor(fl32(fl32(m - lo) * inv_w)),
     0, nb - 1) with m = fl32(key_e - theta) and inv_w = fl32(nb / (hi - lo)).
@@ -45,7 +47,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["qb_keys", "qb_margins", "qb_target", "qb_quantile_exact", "qb_inv_width", "qb_histogram",
+__all__ = ["qb_keys", "qb_margins", "qb_target", "qb_quantile_exact", "qb_rank_margins", "qb_inv_width", "qb_histogram",
            "qb_quantile_from_hist", "qb_bias_update"]
 
 
@@ -87,10 +89,16 @@ def qb_target(T: int, k: int, E: int) -> int:
 
 def qb_quantile_exact(m64: np.ndarray, c: int) -> np.ndarray:
     """Per expert, the midpoint of its c-th and (c+1)-th largest margin."""
+    lo_hi = qb_rank_margins(m64, c)
+    return 0.5 * (lo_hi[0] + lo_hi[1])
+
+
+def qb_rank_margins(m64: np.ndarray, c: int):
+    """Per expert, (c-th largest margin, (c+1)-th largest margin)."""
     srt = -np.sort(-m64, axis=0)  # descending per column
     if not 1 <= c < srt.shape[0]:
         raise ValueError("target count must be in [1, T)")
-    return 0.5 * (srt[c - 1] + srt[c])
+    return srt[c - 1], srt[c]
 
 
 def qb_inv_width(nb: int, lo: float, hi: float) -> np.float32:
@@ -136,4 +144,5 @@ def qb_bias_update(s32, b32, k: int, nb: int, lo: float, hi: float) -> dict:
     counts = qb_histogram(m32, nb, lo, hi)
     q = qb_quantile_from_hist(counts, c, lo, hi)
     return {"counts": counts, "q": q, "bias": np.asarray(b32, dtype=np.float64) - q, "target": c,
-            "q_exact": qb_quantile_exact(m64, c), "selected": selected, "m64": m64}
+            "q_exact": qb_quantile_exact(m64, c), "rank_gap": np.subtract(*qb_rank_margins(m64, c)),
+            "selected": selected, "m64": m64}
