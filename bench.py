@@ -150,7 +150,7 @@ def measure_qb(cfg, dev, stream, peaks: dict, reps: int = 10) -> dict:
     s = torch.from_numpy(gen.qb_scores(cfg)).to(dev)
     b = torch.from_numpy(gen.bias(cfg)).to(dev)
     out = torch.empty(cfg.E, dtype=torch.float32, device=dev)
-    hist = torch.empty(cfg.E * nb + 3 * cfg.T, dtype=torch.int32, device=dev)
+    hist = torch.empty(cfg.E * nb, dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     d = dims_for(cfg, "f32")
 
@@ -173,8 +173,7 @@ def measure_qb(cfg, dev, stream, peaks: dict, reps: int = 10) -> dict:
     # scores read, histogram zeroed and read back, bias in / out
     nbytes = cfg.T * cfg.E * 4 + 2 * cfg.E * nb * 4 + 2 * cfg.E * 4
     achieved = nbytes / (ms / 1e3) / 1e9
-    return {"kernel": "qb_zero_kernel + qb_thresh_kernel + qb_slice_hist_kernel + qb_quantile_kernel", "ms": round(ms, 4),
-            "bound": "hbm",
+    return {"kernel": "qb_zero_kernel + qb_hist_kernel + qb_quantile_kernel", "ms": round(ms, 4), "bound": "hbm",
             "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes, "bins": nb,
             "scores": f"[{cfg.T}, {cfg.E}] fp32, uniform in [0, 1); target floor(T k / E) = {cfg.T * cfg.k // cfg.E}"}

@@ -237,12 +237,10 @@ MOE_API moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk_id
  *  - Margin of expert e for token t: fl32(s + b_e) minus the k-th largest key
  *    fl32(s + b) among the token's OTHER experts (ties rank the lower index
  *    first); e is selected exactly when its margin is positive.
- *  - hist: caller-owned workspace of E*nbins + 3*T uint32 words; on return
- *    its first E*nbins words hold the per-expert margin histogram [E, nbins]
- *    on [lo, hi) (nbins equal bins, a multiple of 32 in [32, 65536]; margins
- *    outside go to the end bins; the bin index is
- *    floor(fl32(fl32(m - lo) * fl32(nbins / (hi - lo))))); the rest is
- *    scratch (each token's k-th / (k+1)-th key and k-th winner).
+ *  - hist [E, nbins] uint32: caller-owned workspace, overwritten with the
+ *    per-expert margin histogram on [lo, hi) (nbins equal bins, a multiple of
+ *    32 in [32, 65536]; margins outside go to the end bins; the bin index is
+ *    floor(fl32(fl32(m - lo) * fl32(nbins / (hi - lo))))).
  *  - bias_out[e] = bias_in[e] - q[e], with q[e] the rank-c boundary of e's
  *    margins, c = floor(T*k/E), read from the histogram with the margins
  *    spread evenly within a bin; quantile_out [E] (may be NULL) receives q.

@@ -225,8 +225,7 @@ def moe_permute_noalloc(d, topk_idx, z, expert_offsets, perm_token, inv_perm, z_
 def moe_qb_bias_update(d, scores, bias_in, bias_out, quantile_out, hist, nbins: int, lo: float, hi: float,
                        stream=None) -> int:
     """Quantile Balancing bias update from a batch of router scores (see
-    include/moe.h); hist is a workspace of E * nbins + 3 * T uint32 words whose
-    first E * nbins hold the histogram on return."""
+    include/moe.h); hist is an [E, nbins] uint32 workspace, overwritten."""
     return lib().moe_qb_bias_update(ctypes.byref(_dims(d)), _ptr(scores), _ptr(bias_in), _ptr(bias_out),
                                     _ptr(quantile_out), _ptr(hist), int(nbins), float(lo), float(hi), _stream(stream))
 

@@ -927,23 +927,8 @@ extern "C" moe_status moe_qb_bias_update(const moe_dims* d, const float* scores,
   const float w = static_cast<float>(span / nbins);
   const long long n = static_cast<long long>(E) * nbins;
   qb_zero_kernel<<<static_cast<unsigned>(std::min<long long>(cdiv(n, 256), 1184)), 256, 0, s>>>(hist, n);
-  if (nbins <= QB_MAX_SMEM_BINS) {
-    // thresholds live after the histogram in the caller's workspace
-    float* thr_k = reinterpret_cast<float*>(hist + n);
-    float* thr_k1 = thr_k + T;
-    int* idx_k = reinterpret_cast<int*>(thr_k1 + T);
-    qb_thresh_kernel<<<static_cast<unsigned>(cdiv(T, QB_WARPS)), QB_WARPS * 32, 0, s>>>(scores, bias_in, T, E, k, thr_k,
-                                                                                          thr_k1, idx_k);
-    const size_t smem = static_cast<size_t>(QB_ES) * nbins * 4;
-    if (cudaFuncSetAttribute(qb_slice_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    qb_slice_hist_kernel<<<static_cast<unsigned>(cdiv(E, QB_ES)), QB_WARPS * 32, smem, s>>>(
-        scores, bias_in, T, E, nbins, lo, inv_w, thr_k, thr_k1, idx_k, hist);
-  } else {
-    qb_hist_kernel<<<static_cast<unsigned>(cdiv(T, QB_WARPS)), QB_WARPS * 32, 0, s>>>(scores, bias_in, T, E, k, nbins,
-                                                                                        lo, inv_w, hist);
-  }
+  qb_hist_kernel<<<static_cast<unsigned>(cdiv(T, QB_WARPS)), QB_WARPS * 32, 0, s>>>(scores, bias_in, T, E, k, nbins,
+                                                                                      lo, inv_w, hist);
   qb_quantile_kernel<<<E, 32, 0, s>>>(hist, E, nbins, c, lo, w, bias_in, bias_out, quantile_out);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

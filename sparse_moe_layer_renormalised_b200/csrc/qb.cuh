@@ -14,20 +14,11 @@
 // floor(T k / E), read from an nb-bin histogram on [lo, hi) with the margins
 // spread evenly inside a bin.
 //
-//   qb_thresh_kernel      one warp per token: keys, top-(k+1) by warp arg-max
-//                         rounds; stores the k-th and (k+1)-th key and the
-//                         k-th winner's index (12 bytes per token).
-//   qb_slice_hist_kernel  one block per QB_ES experts over all tokens: each
-//                         margin from the stored thresholds, counted in a
-//                         shared-memory histogram, merged into the global one
-//                         with one atomic per nonzero bin (nb <= 4096).
-//   qb_hist_kernel        the single-pass form for finer histograms: margins
-//                         counted with one global atomic each.
-//   qb_quantile_kernel    one warp per expert: scan its nb counts from the top
-//                         bin, locate rank c, interpolate, write q_e and b_e - q_e.
-// Expert e is among token t's top k exactly when key_e > kth or (key_e == kth
-// and e <= the k-th winner's index), which is how the second pass recovers
-// the selection from the stored thresholds.
+//   qb_hist_kernel      one warp per token: keys, top-(k+1) by warp arg-max
+//                       rounds, margins, fp32 bin index, global atomic count.
+//                       HBM-bound: T*E*4 bytes of scores read.
+//   qb_quantile_kernel  one warp per expert: scan its nb counts from the top
+//                       bin, locate rank c, interpolate, write q_e and b_e - q_e.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -109,107 +100,6 @@ __global__ void __launch_bounds__(QB_WARPS * 32)
       const int bin = min(max(static_cast<int>(floorf(u)), 0), nb - 1);
       atomicAdd(&hist[static_cast<long long>(e) * nb + bin], 1u);
     }
-  }
-}
-
-constexpr int QB_ES = 8;               // experts per block of the histogram pass
-constexpr int QB_MAX_SMEM_BINS = 4096;  // QB_ES * nb * 4 bytes of shared memory
-
-__global__ void __launch_bounds__(QB_WARPS * 32)
-    qb_thresh_kernel(const float* __restrict__ scores, const float* __restrict__ bias, long long T, int E, int k,
-                     float* __restrict__ thr_k, float* __restrict__ thr_k1, int* __restrict__ idx_k) {
-  const int lane = threadIdx.x & 31;
-  const long long t = static_cast<long long>(blockIdx.x) * QB_WARPS + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const float* srow = scores + t * E;
-  float key[32];
-  uint32_t live = 0u;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = -INFINITY;
-    if (e < E) {
-      float kk = __fadd_rn(srow[e], bias[e]);
-      if (kk != kk) kk = -INFINITY;  // a NaN key ranks below every number
-      key[i] = kk;
-      live |= 1u << i;
-    }
-  }
-  float kth = -INFINITY, k1th = -INFINITY;
-  int kidx = 0;
-  for (int j = 0; j <= k; ++j) {
-    float bk = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if ((live >> i) & 1u) {
-        const int e = lane + 32 * i;
-        if (key[i] > bk || (key[i] == bk && e < be)) {
-          bk = key[i];
-          be = e;
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ok > bk || (ok == bk && oe < be)) {
-        bk = ok;
-        be = oe;
-      }
-    }
-    if (lane == (be & 31)) live &= ~(1u << (be >> 5));  // k < E: be is a valid expert
-    if (j == k - 1) {
-      kth = bk;
-      kidx = be;
-    }
-    if (j == k) k1th = bk;
-  }
-  if (lane == 0) {
-    thr_k[t] = kth;
-    thr_k1[t] = k1th;
-    idx_k[t] = kidx;
-  }
-}
-
-// Block = QB_ES consecutive experts x all tokens; a warp takes 32 / QB_ES
-// tokens per step, lane = (token, expert) of the step.
-__global__ void __launch_bounds__(QB_WARPS * 32)
-    qb_slice_hist_kernel(const float* __restrict__ scores, const float* __restrict__ bias, long long T, int E, int nb,
-                         float lo, float inv_w, const float* __restrict__ thr_k, const float* __restrict__ thr_k1,
-                         const int* __restrict__ idx_k, uint32_t* __restrict__ hist) {
-  extern __shared__ uint32_t qb_sh[];  // [QB_ES][nb]
-  constexpr int TPS = 32 / QB_ES;      // tokens per warp step
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int e0 = blockIdx.x * QB_ES;
-  for (int i = threadIdx.x; i < QB_ES * nb; i += blockDim.x) qb_sh[i] = 0u;
-  __syncthreads();
-  const int el = lane % QB_ES;
-  const int e = e0 + el;
-  if (e < E) {
-    const float b = bias[e];
-    uint32_t* my = qb_sh + el * nb;
-    for (long long t = static_cast<long long>(warp) * TPS + lane / QB_ES; t < T; t += QB_WARPS * TPS) {
-      float key = __fadd_rn(scores[t * E + e], b);
-      if (key != key) key = -INFINITY;
-      const float kk = thr_k[t];
-      const bool selected = key > kk || (key == kk && e <= idx_k[t]);
-      const float theta = selected ? thr_k1[t] : kk;
-      const float m = __fsub_rn(key, theta);
-      float u = __fmul_rn(__fsub_rn(m, lo), inv_w);
-      if (u != u) u = 0.f;
-      u = fminf(fmaxf(u, -1.0f), static_cast<float>(nb));
-      const int bin = min(max(static_cast<int>(floorf(u)), 0), nb - 1);
-      atomicAdd(&my[bin], 1u);
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < QB_ES * nb; i += blockDim.x) {
-    const uint32_t v = qb_sh[i];
-    const int ee = e0 + i / nb;
-    if (v != 0u && ee < E) atomicAdd(&hist[static_cast<long long>(ee) * nb + (i % nb)], v);
   }
 }
 
