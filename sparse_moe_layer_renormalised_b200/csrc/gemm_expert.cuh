@@ -42,7 +42,6 @@
 namespace moe {
 
 constexpr int EX_BK = 64;
-constexpr int EX_MAX_TOK = 256;                       // tokens per tile (MMA N <= 256)
 constexpr uint32_t EX_A_BYTES = 128 * EX_BK * 2;      // 128 weight rows
 constexpr uint32_t EX_B_BYTES = 128 * EX_BK * 2;      // up to 128 token rows per CTA
 constexpr uint32_t EX_STAGE_BYTES = EX_A_BYTES + EX_B_BYTES;

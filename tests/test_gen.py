@@ -89,3 +89,21 @@ def test_sample_tokens():
     s = gen.sample_tokens(cfg)
     assert len(s) == 512 and len(np.unique(s)) == 512 and s.min() >= 0 and s.max() < cfg.T
     assert np.array_equal(s, gen.sample_tokens(cfg))
+
+
+def test_qb_scores_are_24_bit_uniforms():
+    """The Quantile Balancing input: fp32 in [0, 1) on the 2^-24 grid,
+    reproducible, and from its own Philox stream (not the x or bias words)."""
+    cfg = gen.CONFIGS["mid"].with_(T=512)
+    s = gen.qb_scores(cfg)
+    assert s.shape == (cfg.T, cfg.E) and s.dtype == np.float32
+    assert s.min() >= 0.0 and s.max() < 1.0
+    grid = s.astype(np.float64) * 2.0 ** 24
+    assert np.array_equal(grid, np.round(grid))
+    assert np.array_equal(s, gen.qb_scores(cfg))
+    words = gen.u32_words(cfg.seed, gen.TID["qb_scores"], 0, 8)
+    assert np.array_equal(s.ravel()[:8], (words >> 8).astype(np.float32) * np.float32(2.0 ** -24))
+    # mean and variance of U[0, 1) within 4 standard errors
+    n = s.size
+    assert abs(s.mean() - 0.5) < 4 * (1 / 12) ** 0.5 / n ** 0.5
+    assert abs(s.var() - 1 / 12) < 4 * (1 / 180) ** 0.5 / n ** 0.5
