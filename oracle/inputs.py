@@ -40,6 +40,13 @@ def expert_weights(cfg, e: int):
     return tuple(mats)
 
 
+def expert_weights_raw(cfg, e: int):
+    """(Wg_e, Wv_e, Wo_e) as the generator's host arrays: float32 values, bf16
+    bit patterns (uint16) or MXFP4 (codes, scales) pairs.  The C++ oracle
+    decodes these bits itself."""
+    return tuple(gen.host_expert(cfg, name, e) for name in ("Wg", "Wv", "Wo"))
+
+
 def all_weights(cfg) -> dict:
     """Every weight as fp64 (small configurations only)."""
     w = dense_weights(cfg)

@@ -14,9 +14,11 @@ def _build_libraries():
     """Build the CUDA library and the generator library in-tree if missing or
     stale (nvcc cross-compiles for sm_100a without a GPU)."""
     import gen.build
+    import oracle.build
     import sparse_moe_layer_renormalised_b200.build as b
 
     b.build()
+    oracle.build.build()
     if not os.path.exists(os.path.join(ROOT, "gen", "libmoegen.so")):
         gen.build.build()
 

@@ -18,21 +18,28 @@ from oracle import inputs as oin
 F64 = torch.float64
 
 
+@pytest.fixture(params=["cpp", "torch"])
+def O(request):
+    """Each pin runs on both restatements of the method: the fp64 C++ oracle
+    and the fp64 PyTorch one."""
+    return oracle if request.param == "cpp" else oracle.torch_ref
+
+
 # ---------------------------------------------------------------- number formats
-def test_bf16_round_matches_torch_on_fp32_values():
+def test_bf16_round_matches_torch_on_fp32_values(O):
     a = torch.randn(100_000, generator=torch.Generator().manual_seed(1), dtype=torch.float32) * 37.0
     want = a.to(torch.bfloat16).to(F64)
-    got = oracle.bf16_round(a.to(F64))
+    got = O.bf16_round(a.to(F64))
     assert torch.equal(got, want)
 
 
-def test_bf16_round_is_nearest_even_on_fp64_values():
+def test_bf16_round_is_nearest_even_on_fp64_values(O):
     rng = np.random.default_rng(3)
     x = rng.standard_normal(20_000) * 10.0 ** rng.integers(-5, 5, 20_000)
     # include exact midpoints between bf16 neighbours
     mid = np.array([1.0 + 2.0**-8, 1.0 + 3 * 2.0**-8, -(2.0 + 2.0**-7)])
     x = np.concatenate([x, mid])
-    r = oracle.bf16_round(torch.from_numpy(x)).numpy()
+    r = O.bf16_round(torch.from_numpy(x)).numpy()
     for xi, ri in zip(x, r):
         e = math.frexp(abs(xi))[1]  # |x| in [2^(e-1), 2^e)
         ulp = 2.0 ** (e - 1 - 7)
@@ -48,32 +55,32 @@ def test_bf16_round_is_nearest_even_on_fp64_values():
         assert abs(ri) == want and (ri == 0 or np.sign(ri) == np.sign(xi))
 
 
-def test_e2m1_dequant_matches_ocp_table():
+def test_e2m1_dequant_matches_ocp_table(O):
     tab = {int(r[0]): float(r[1]) for r in read_golden("e2m1_ocp_mx.txt")}
     for s in (1, 100, 120, 127, 130, 200):
         codes = np.array([[c | (d << 4) for c, d in zip(range(0, 16, 2), range(1, 16, 2))] * 4], np.uint8)
         scales = np.full((1, 2), s, np.uint8)
-        v = oracle.mxfp4_dequant(codes, scales)[0].numpy()
+        v = O.mxfp4_dequant(codes, scales)[0].numpy()
         for k in range(32):
             assert v[k] == tab[k % 16] * 2.0 ** (s - 127)
-    nan = oracle.mxfp4_dequant(np.zeros((1, 16), np.uint8), np.full((1, 1), 255, np.uint8))
+    nan = O.mxfp4_dequant(np.zeros((1, 16), np.uint8), np.full((1, 1), 255, np.uint8))
     assert torch.isnan(nan).all()
 
 
-def test_mxfp4_dequant_of_generator_output_is_bf16_exact():
+def test_mxfp4_dequant_of_generator_output_is_bf16_exact(O):
     # E2M1 x 2^e needs at most 2 significant bits: exact in bfloat16.
     c, s = gen.fill_host_mxfp4(0, 7, 0, 8, 512, 512**-0.5)
-    v = oracle.mxfp4_dequant(c, s)
-    assert torch.equal(oracle.bf16_round(v), v)
+    v = O.mxfp4_dequant(c, s)
+    assert torch.equal(O.bf16_round(v), v)
 
 
 # ---------------------------------------------------------------- router
-def test_sigmoid_matches_scipy():
+def test_sigmoid_matches_scipy(O):
     x = torch.linspace(-30, 30, 2001, dtype=F64)
-    assert torch.allclose(oracle.sigmoid(x), torch.from_numpy(scipy.special.expit(x.numpy())), rtol=1e-15, atol=0)
+    assert torch.allclose(O.sigmoid(x), torch.from_numpy(scipy.special.expit(x.numpy())), rtol=1e-15, atol=0)
 
 
-def test_router_orientation():
+def test_router_orientation(O):
     # W_r = a row permutation: logit e = x[perm[e]]
     H = 7
     perm = [3, 0, 6, 1, 5, 2, 4]
@@ -81,7 +88,7 @@ def test_router_orientation():
     for e, h in enumerate(perm):
         Wr[e, h] = 1.0
     x = torch.randn(5, H, dtype=F64, generator=torch.Generator().manual_seed(0))
-    s = oracle.router_scores(x, Wr)
+    s = O.router_scores(x, Wr)
     want = torch.from_numpy(scipy.special.expit(x[:, perm].numpy()))
     assert torch.allclose(s, want, rtol=1e-15, atol=0)
 
@@ -99,14 +106,14 @@ def _brute_force_topk(key, k):
 
 
 @pytest.mark.parametrize("E,k", [(6, 1), (6, 3), (8, 4), (10, 2), (12, 4)])
-def test_select_experts_brute_force(E, k):
+def test_select_experts_brute_force(O, E, k):
     rng = np.random.default_rng(E * 100 + k)
     for trial in range(40):
         # quantised values produce exact ties in s + b
         s = rng.integers(1, 8, size=E) / 8.0
         b = rng.integers(-2, 3, size=E) / 8.0
         key = s + b
-        idx, p, margin = oracle.select_experts(torch.tensor(s[None]), torch.tensor(b), k)
+        idx, p, margin = O.select_experts(torch.tensor(s[None]), torch.tensor(b), k)
         want = _brute_force_topk(list(key), k)
         assert idx[0].tolist() == want
         # mixture weights: unbiased scores renormalised over the chosen set
@@ -115,31 +122,31 @@ def test_select_experts_brute_force(E, k):
         assert margin[0].item() == pytest.approx(srt[k - 1] - srt[k]) if k < E else True
 
 
-def test_mixture_weights_use_unbiased_scores():
+def test_mixture_weights_use_unbiased_scores(O):
     s = torch.tensor([[0.9, 0.2, 0.3, 0.1]], dtype=F64)
     b = torch.tensor([-1.0, 0.5, 0.0, 0.0], dtype=F64)  # the bias reorders the selection
-    idx, p, _ = oracle.select_experts(s, b, 2)
+    idx, p, _ = O.select_experts(s, b, 2)
     assert idx[0].tolist() == [1, 2]  # keys 0.7, 0.3 beat -0.1 and 0.1
     assert torch.allclose(p[0], torch.tensor([0.2 / 0.5, 0.3 / 0.5], dtype=F64))
     assert abs(p.sum().item() - 1.0) < 1e-15
 
 
-def test_select_from_f32_scores_uses_fp32_key():
+def test_select_from_f32_scores_uses_fp32_key(O):
     # 0.5 + 2^-30 rounds to 0.5 in fp32: the keys tie there and the lower
     # index wins, although in fp64 the tiny bias decides.
     s2 = np.array([[0.5, 0.5]], np.float32)
     b2 = np.array([0.0, np.float32(2.0**-30)], np.float32)
-    idx2, _ = oracle.select_experts_from_f32_scores(s2, b2, 1)
+    idx2, _ = O.select_experts_from_f32_scores(s2, b2, 1)
     assert idx2[0, 0].item() == 0
-    idx3, _, _ = oracle.select_experts(torch.tensor(s2, dtype=F64), torch.tensor(b2, dtype=F64), 1)
+    idx3, _, _ = O.select_experts(torch.tensor(s2, dtype=F64), torch.tensor(b2, dtype=F64), 1)
     assert idx3[0, 0].item() == 1  # in fp64 the tiny bias decides
 
 
-def test_permute_invariants_and_library_sort():
+def test_permute_invariants_and_library_sort(O):
     rng = np.random.default_rng(5)
     T, E, k = 300, 17, 4
     idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)])
-    counts, offsets, perm_token, inv_perm = oracle.permute(idx, E)
+    counts, offsets, perm_token, inv_perm = O.permute(idx, E)
     assert counts.sum() == T * k and np.all(np.diff(offsets) >= 0) and offsets[-1] == T * k
     assert np.array_equal(np.bincount(idx.ravel(), minlength=E), counts)
     # stable library sort of the flattened expert ids gives the same order
@@ -159,31 +166,31 @@ def test_permute_invariants_and_library_sort():
 
 
 # ---------------------------------------------------------------- experts
-def test_situ_glu_properties():
+def test_situ_glu_properties(O):
     g = torch.linspace(-40, 40, 801, dtype=F64)[:, None]
     v = torch.linspace(-40, 40, 161, dtype=F64)[None, :]
     c = 10.0
-    h = oracle.situ_glu(g, v, c)
-    assert torch.allclose(oracle.situ_glu(g, -v, c), -h, rtol=0, atol=0)  # odd in v
+    h = O.situ_glu(g, v, c)
+    assert torch.allclose(O.situ_glu(g, -v, c), -h, rtol=0, atol=0)  # odd in v
     assert h.abs().max() <= c * c
     # c -> infinity gives SwiGLU (library silu)
-    big = oracle.situ_glu(g, v, 1e6)
+    big = O.situ_glu(g, v, 1e6)
     sw = torch.nn.functional.silu(g) * v
     assert torch.allclose(big, sw, rtol=1e-8, atol=1e-12)
     # small arguments: 0 <= 1 - h/swiglu <= (g^2 + v^2) / (3 c^2)
     gs = torch.linspace(-2, 2, 41, dtype=F64)[:, None]
     vs = torch.linspace(-2, 2, 41, dtype=F64)[None, :]
-    hs = oracle.situ_glu(gs, vs, c)
+    hs = O.situ_glu(gs, vs, c)
     sws = torch.nn.functional.silu(gs) * vs
     mask = sws.abs() > 1e-12
     rel = 1.0 - hs[mask] / sws[mask]
     bound = ((gs**2 + vs**2) / (3 * c * c)).expand_as(hs)[mask]
     assert (rel >= -1e-15).all() and (rel <= bound + 1e-15).all()
     # the cap binds: large positive g, v -> c^2
-    assert abs(oracle.situ_glu(torch.tensor(1e3, dtype=F64), torch.tensor(1e3, dtype=F64), c).item() - c * c) < 1e-9
+    assert abs(O.situ_glu(torch.tensor(1e3, dtype=F64), torch.tensor(1e3, dtype=F64), c).item() - c * c) < 1e-9
 
 
-def test_expert_forward_orientation():
+def test_expert_forward_orientation(O):
     # permutation weights: g = z[pg], v = z[pv], y = h[po]
     L = I = 6
     rng = np.random.default_rng(0)
@@ -195,15 +202,15 @@ def test_expert_forward_orientation():
         return m
 
     z = torch.randn(3, L, dtype=F64, generator=torch.Generator().manual_seed(2))
-    y = oracle.expert_forward(z, P(pg), P(pv), P(po), 10.0, lambda t: t)
-    h = oracle.situ_glu(z[:, pg], z[:, pv], 10.0)
+    y = O.expert_forward(z, P(pg), P(pv), P(po), 10.0, lambda t: t)
+    h = O.situ_glu(z[:, pg], z[:, pv], 10.0)
     assert torch.equal(y, h[:, po])
     # the stored h is rounded before the down projection
-    yb = oracle.expert_forward(z, P(pg), P(pv), P(po), 10.0, oracle.bf16_round)
-    assert torch.equal(yb, oracle.bf16_round(h)[:, po])
+    yb = O.expert_forward(z, P(pg), P(pv), P(po), 10.0, O.bf16_round)
+    assert torch.equal(yb, O.bf16_round(h)[:, po])
 
 
-def test_shared_experts_orientation():
+def test_shared_experts_orientation(O):
     # two shared experts with permutation weights on a square hidden size
     H = 5
     rng = np.random.default_rng(9)
@@ -218,36 +225,36 @@ def test_shared_experts_orientation():
     Wsv = torch.stack([P(b) for _, b, _ in ps])
     Wso = torch.stack([P(c) for _, _, c in ps])
     x = torch.randn(4, H, dtype=F64, generator=torch.Generator().manual_seed(3))
-    y = oracle.shared_experts(x, Wsg, Wsv, Wso, 10.0, lambda t: t)
-    want = sum(oracle.situ_glu(x[:, a], x[:, b], 10.0)[:, c] for a, b, c in ps)
+    y = O.shared_experts(x, Wsg, Wsv, Wso, 10.0, lambda t: t)
+    want = sum(O.situ_glu(x[:, a], x[:, b], 10.0)[:, c] for a, b, c in ps)
     assert torch.allclose(y, want, rtol=1e-15, atol=1e-15)
 
 
-def test_combine_one_hot_and_linear():
+def test_combine_one_hot_and_linear(O):
     y = torch.randn(4, 3, 5, dtype=F64, generator=torch.Generator().manual_seed(4))
     for j in range(3):
         p = torch.zeros(4, 3, dtype=F64)
         p[:, j] = 1.0
-        assert torch.equal(oracle.combine(y, p), y[:, j])
+        assert torch.equal(O.combine(y, p), y[:, j])
     p = torch.rand(4, 3, dtype=F64, generator=torch.Generator().manual_seed(5))
     want = torch.einsum("tj,tjl->tl", p, y)
-    assert torch.allclose(oracle.combine(y, p), want, rtol=1e-14, atol=1e-15)
+    assert torch.allclose(O.combine(y, p), want, rtol=1e-14, atol=1e-15)
 
 
-def test_rms_norm_closed_forms():
+def test_rms_norm_closed_forms(O):
     gam = torch.ones(8, dtype=F64)
     for a in (1e-3, 0.5, 7.0, -3.0):
         u = torch.full((1, 8), a, dtype=F64)
-        n = oracle.rms_norm(u, gam, 1e-6)
+        n = O.rms_norm(u, gam, 1e-6)
         assert torch.allclose(n, torch.full((1, 8), a / math.sqrt(a * a + 1e-6), dtype=F64), rtol=1e-15)
     u = torch.randn(6, 64, dtype=F64, generator=torch.Generator().manual_seed(7))
-    n = oracle.rms_norm(u, torch.ones(64, dtype=F64), 0.0)
-    assert torch.allclose(n, oracle.rms_norm(u * 123.0, torch.ones(64, dtype=F64), 0.0), rtol=1e-14)
+    n = O.rms_norm(u, torch.ones(64, dtype=F64), 0.0)
+    assert torch.allclose(n, O.rms_norm(u * 123.0, torch.ones(64, dtype=F64), 0.0), rtol=1e-14)
     assert torch.allclose((n * n).mean(dim=1), torch.ones(6, dtype=F64), rtol=1e-14)
     g = torch.randn(64, dtype=F64, generator=torch.Generator().manual_seed(8))
-    assert torch.allclose(oracle.rms_norm(u, g, 0.0), g[None] * n, rtol=1e-14)
+    assert torch.allclose(O.rms_norm(u, g, 0.0), g[None] * n, rtol=1e-14)
     ms = (u * u).mean(dim=1)
-    n1 = oracle.rms_norm(u, torch.ones(64, dtype=F64), 0.25)
+    n1 = O.rms_norm(u, torch.ones(64, dtype=F64), 0.25)
     assert torch.allclose((n1 * n1).mean(dim=1), ms / (ms + 0.25), rtol=1e-14)
 
 
@@ -256,7 +263,7 @@ def _tiny_weights(cfg):
     return oin.all_weights(cfg)
 
 
-def test_identical_experts_reduce_to_dense_glu():
+def test_identical_experts_reduce_to_dense_glu(O):
     """Zero bias and identical experts: the routed mixture is one dense GLU
     (the renormalised weights sum to one), for any routing."""
     cfg = gen.CONFIGS["tiny"]
@@ -265,60 +272,60 @@ def test_identical_experts_reduce_to_dense_glu():
     for name in ("Wg", "Wv", "Wo"):
         w[name] = w[name][:1].expand_as(w[name]).clone()
     x = oin.x_rows(cfg, range(cfg.T))
-    out = oracle.layer_forward(cfg, w, x)
-    rnd = oracle.storage_round(cfg.act)
+    out = O.layer_forward(cfg, w, x)
+    rnd = O.storage_round(cfg.act)
     z = rnd(x @ w["Wdown"].T)
-    u_dense = oracle.expert_forward(z, w["Wg"][0], w["Wv"][0], w["Wo"][0], cfg.situ_c, rnd)
+    u_dense = O.expert_forward(z, w["Wg"][0], w["Wv"][0], w["Wo"][0], cfg.situ_c, rnd)
     assert torch.allclose(out["u"], u_dense, rtol=1e-12, atol=1e-13)
-    n = rnd(oracle.rms_norm(u_dense, w["gamma"], cfg.rms_eps))
-    y = oracle.shared_experts(x, w["Wsg"], w["Wsv"], w["Wso"], cfg.situ_c, rnd) + n @ w["Wup"].T
+    n = rnd(O.rms_norm(u_dense, w["gamma"], cfg.rms_eps))
+    y = O.shared_experts(x, w["Wsg"], w["Wsv"], w["Wso"], cfg.situ_c, rnd) + n @ w["Wup"].T
     assert torch.allclose(out["y"], y, rtol=1e-12, atol=1e-12)
 
 
-def test_latent_projection_orientation():
+def test_latent_projection_orientation(O):
     """W_down = [I | 0] selects the first L hidden coordinates of x."""
     cfg = gen.CONFIGS["tiny"]
     w = _tiny_weights(cfg)
     w["Wdown"] = torch.zeros(cfg.L, cfg.H, dtype=F64)
     w["Wdown"][torch.arange(cfg.L), torch.arange(cfg.L)] = 1.0
     x = oin.x_rows(cfg, range(8))
-    out = oracle.layer_forward(cfg, w, x)
+    out = O.layer_forward(cfg, w, x)
     assert torch.equal(out["z"], x[:, : cfg.L])
 
 
-def test_top1_routing_uses_the_selected_expert_only():
+def test_top1_routing_uses_the_selected_expert_only(O):
     """k = 1: p = 1 and u is the chosen expert's output."""
     cfg = gen.CONFIGS["tiny"].with_(k=1)
     w = _tiny_weights(cfg)
     x = oin.x_rows(cfg, range(16))
-    out = oracle.layer_forward(cfg, w, x)
+    out = O.layer_forward(cfg, w, x)
     assert torch.equal(out["p"], torch.ones(16, 1, dtype=F64))
-    rnd = oracle.storage_round(cfg.act)
+    rnd = O.storage_round(cfg.act)
     for t in range(16):
         e = out["idx"][t, 0].item()
-        ye = oracle.expert_forward(out["z"][t : t + 1], w["Wg"][e], w["Wv"][e], w["Wo"][e], cfg.situ_c, rnd)
+        ye = O.expert_forward(out["z"][t : t + 1], w["Wg"][e], w["Wv"][e], w["Wo"][e], cfg.situ_c, rnd)
         assert torch.allclose(out["u"][t : t + 1], ye, rtol=1e-14, atol=1e-15)
 
 
-def test_streamed_forward_equals_in_memory_forward():
+def test_streamed_forward_equals_in_memory_forward(O):
     cfg = gen.CONFIGS["tiny"]
     w = _tiny_weights(cfg)
     x = oin.x_rows(cfg, range(cfg.T))
-    a = oracle.layer_forward(cfg, w, x)
-    b = oracle.layer_forward_streamed(cfg, w, x, lambda e: (w["Wg"][e], w["Wv"][e], w["Wo"][e]))
+    a = O.layer_forward(cfg, w, x)
+    b = O.layer_forward_streamed(cfg, w, x, lambda e: (w["Wg"][e], w["Wv"][e], w["Wo"][e]))
     assert torch.equal(a["idx"], b["idx"]) and torch.allclose(a["y"], b["y"], rtol=1e-14, atol=1e-14)
 
 
-def test_storage_rounding_points():
+def test_storage_rounding_points(O):
     """bf16 workloads: z, n (and h, shared h) are bf16 values; u, y are not."""
     cfg = gen.CONFIGS["mid"].with_(T=16)
     w = oin.dense_weights(cfg)
     x = oin.x_rows(cfg, range(16))
-    out = oracle.layer_forward_streamed(cfg, w, x, lambda e: oin.expert_weights(cfg, e))
-    assert torch.equal(oracle.bf16_round(out["z"]), out["z"])
-    assert torch.equal(oracle.bf16_round(out["n"]), out["n"])
-    assert not torch.equal(oracle.bf16_round(out["u"]), out["u"])
-    assert not torch.equal(oracle.bf16_round(out["y"]), out["y"])
+    out = O.layer_forward_streamed(cfg, w, x, lambda e: oin.expert_weights(cfg, e))
+    assert torch.equal(O.bf16_round(out["z"]), out["z"])
+    assert torch.equal(O.bf16_round(out["n"]), out["n"])
+    assert not torch.equal(O.bf16_round(out["u"]), out["u"])
+    assert not torch.equal(O.bf16_round(out["y"]), out["y"])
 
 
 def test_k3_parameter_count_matches_the_published_total():
@@ -333,3 +340,41 @@ def test_k3_parameter_count_matches_the_published_total():
     assert abs(total / t["total_params"] - 1.0) < 0.005
     active = (cfg.k * 3 * cfg.L * cfg.I + cfg.S * 3 * cfg.H * cfg.Is + 2 * cfg.H * cfg.L + cfg.E * cfg.H) * t["layers"]
     assert active < t["active_params"]  # the rest is attention and embeddings
+
+
+# ---------------------------------------------------------------- the two restatements
+def test_cpp_oracle_reads_raw_weight_bits_exactly():
+    """The C++ oracle decodes bf16 bit patterns and MXFP4 (codes, scales)
+    itself; the results equal those from exactly decoded fp64 weights."""
+    for name in ("mid", "mxfp4-small"):
+        cfg = gen.CONFIGS[name]
+        dense = oin.dense_weights(cfg)
+        x = oin.x_rows(cfg, range(8))
+        a = oracle.layer_forward_streamed(cfg, dense, x, lambda e: oin.expert_weights_raw(cfg, e))
+        b = oracle.layer_forward_streamed(cfg, dense, x, lambda e: oin.expert_weights(cfg, e))
+        for key in ("s", "idx", "p", "z", "u", "n", "y"):
+            assert torch.equal(a[key], b[key]), key
+
+
+def test_cpp_and_torch_oracles_agree_on_a_bf16_layer():
+    """Independent restatements (C++ loops, PyTorch ops) of the same layer:
+    identical selections, outputs equal up to fp64 summation order (and the
+    bf16 storage roundings that order can flip, one step at most)."""
+    cfg = gen.CONFIGS["mid"]
+    dense = oin.dense_weights(cfg)
+    x = oin.x_rows(cfg, range(24))
+    a = oracle.layer_forward_streamed(cfg, dense, x, lambda e: oin.expert_weights_raw(cfg, e))
+    b = oracle.torch_ref.layer_forward_streamed(cfg, dense, x, lambda e: oin.expert_weights(cfg, e))
+    assert torch.equal(a["idx"], b["idx"])
+    assert torch.allclose(a["s"], b["s"], rtol=1e-13, atol=0)
+    assert torch.allclose(a["p"], b["p"], rtol=1e-13, atol=0)
+    for key in ("u", "y"):
+        rms = b[key].pow(2).mean().sqrt()
+        assert ((a[key] - b[key]).abs().max() / rms).item() < 1e-4, key
+
+
+def test_cpp_oracle_thread_count_is_the_host_core_count():
+    import os
+
+    assert oracle.num_threads() == (int(os.environ["MOE_ORACLE_THREADS"]) if os.environ.get("MOE_ORACLE_THREADS")
+                                    else os.cpu_count())
