@@ -3,11 +3,17 @@
 
 One step = one moe_layer_forward over one batch of T synthetic tokens (all
 stages: router, top-k, latent projection, shared experts, permute, routed
-experts, combine + RMSNorm, output projection).  Default workload: the
-K3-shape prefill layer (T=16384, H=7168, L=3584, 896 experts top-16,
-I=3072, 2 shared experts, Zipf(0.8) expert load), bf16 with fp32 accumulation.
+experts, combine + RMSNorm, output projection).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config prefill|decode|mid|tiny]
+The default run measures three K3-shape workloads, one after the other:
+  prefill  T=16384, bf16, Zipf(0.8) expert load  -> the headline line
+  decode   T=256, bf16, bias N(0, 0.05)           -> "decode" sub-object
+  mxfp4    T=8192, MXFP4 routed weights           -> "mxfp4" sub-object
+(H=7168, L=3584, 896 experts top-16, I=3072, 2 shared experts, Is=3072).
+Each line carries its own device time, stage times, roofline, end-to-end
+number, near-tie count and an oracle sample (parity and CPU baseline).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--no-extra-lines]
   python bench.py --impl reference ...     # the CPU oracle on a bounded sample
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent
@@ -36,6 +42,7 @@ import sparse_moe_layer_renormalised_b200 as moe  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at K3 shape (bf16, MXFP4); % of tensor/HBM roofline"
 STAGE = {n: i for i, n in enumerate(moe.STAGE_NAMES)}
+NEAR_TIE = 1e-4  # key margin (k-th minus (k+1)-th largest key) counted as a near tie
 
 
 def load_peaks() -> dict:
@@ -123,9 +130,14 @@ def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: fl
     return tokens_per_rank_step * steps * world / (max_ms / 1e3)
 
 
+def barrier(world: int) -> None:
+    if world > 1:
+        torch.distributed.barrier()
+
+
 # ----------------------------------------------------------------------------------- roofline
-def dominant_stage(cfg) -> str:
-    return "expert_gate_up"
+def routed_weight_bytes_per_element(cfg) -> float:
+    return 0.53125 if cfg.routed == "mxfp4" else (2.0 if cfg.routed == "bf16" else 4.0)  # MXFP4: 4 bits + E8M0/32
 
 
 def stage_work(cfg, offsets: np.ndarray, T: int) -> dict:
@@ -135,10 +147,52 @@ def stage_work(cfg, offsets: np.ndarray, T: int) -> dict:
     R = T * cfg.k
     counts = np.diff(offsets)
     touched = int((counts > 0).sum())
-    wbytes = 2 * cfg.I * cfg.L * (0.53125 if cfg.routed == "mxfp4" else 2.0)  # MXFP4: 4 bits + E8M0/32
+    wbytes = 2 * cfg.I * cfg.L * routed_weight_bytes_per_element(cfg)
     flops = 2.0 * R * cfg.L * 2 * cfg.I
     bytes_ = touched * wbytes + R * cfg.L * 2 + R * cfg.I * 2
     return {"flops": flops, "bytes": bytes_, "touched_experts": touched}
+
+
+def layer_bytes(cfg, offsets: np.ndarray, T: int, y_bytes: int) -> float:
+    """Algorithmic HBM bytes of one whole layer step: every weight the step
+    touches (the three matrices of each expert with at least one row, the
+    router, W_down, W_up, the shared experts) plus x read and y written.  This
+    is the bound of the weight-streaming decode step."""
+    es = 2 if cfg.act == "bf16" else 4
+    touched = int((np.diff(offsets) > 0).sum())
+    routed = touched * 3 * cfg.I * cfg.L * routed_weight_bytes_per_element(cfg)
+    dense = (cfg.E * cfg.H + 2 * cfg.L * cfg.H + 3 * cfg.S * cfg.Is * cfg.H) * es + cfg.E * 4 + cfg.L * 4
+    return routed + dense + T * cfg.H * es + T * cfg.H * y_bytes
+
+
+def gate_up_roofline(cfg, offsets, stage_ms: dict, peaks: dict) -> dict:
+    """Roofline of the dominant kernel, the routed gate/up GEMM with the
+    SiTU-GLU epilogue, from its CUDA-event time inside the timed region."""
+    work = stage_work(cfg, offsets, cfg.T)
+    dom_ms = stage_ms["expert_gate_up"]
+    bound = "tensor" if (work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)) >= (
+        work["bytes"] / (peaks["hbm_gbs"] * 1e9)) else "hbm"
+    if bound == "tensor":
+        achieved = work["flops"] / (dom_ms / 1e3) / 1e12
+        peak, unit = peaks["bf16_tflops_sustained"], "TFLOP/s"
+        src = f"{peaks['source']} sustained bf16 (the MMA kind is kind::f16 with bf16 operands)"
+    else:
+        achieved = work["bytes"] / (dom_ms / 1e3) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        src = f"{peaks['source']} HBM copy (read+write bytes); a read-dominated stream can exceed it"
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}_expert_gate_up.json")
+    if os.path.exists(prof):
+        # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu
+        # capture of this workload (the file gives the command and kernel build)
+        with open(prof) as f:
+            traffic = json.load(f).get("dram_bytes_per_launch")
+    kern = "tc_expert_kernel (2-CTA grouped gate/up + SiTU epilogue" + (
+        ", MXFP4 weights decoded to bf16 in shared memory)" if cfg.routed == "mxfp4" else ")")
+    return {"kernel": f"{kern} = stage expert_gate_up", "bound": bound, "achieved": round(achieved, 1),
+            "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
+            "kernel_ms": round(dom_ms, 4), "algorithmic": {"flops": work["flops"], "bytes": work["bytes"]},
+            "touched_experts": work["touched_experts"]}
 
 
 def measure_qb(cfg, dev, stream, peaks: dict, reps: int = 10) -> dict:
@@ -180,15 +234,13 @@ def measure_qb(cfg, dev, stream, peaks: dict, reps: int = 10) -> dict:
 
 
 # ----------------------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
-    cfg = gen.CONFIGS[args.config]
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    inputs = gen.device_layer(cfg, dev)
-    x = inputs.pop("x")
-    layer = moe.MoeLayer(dims_for(cfg, args.y_out), inputs)
-    y = layer.output(cfg.T)
+def measure_layer(layer, x, cfg, args, world: int, local_rank: int, sample_clocks: bool) -> dict:
+    """Device time of `args.steps` layer steps (after `args.warmup`), the
+    per-stage times inside that region, and the end-to-end time through the
+    public API with pinned host copies in and out."""
+    dev = x.device
     stream = torch.cuda.current_stream(dev)
+    y = layer.output(cfg.T)
     offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
 
     def events():
@@ -197,7 +249,6 @@ def run_ours(args, rank, world, local_rank):
             e.record(stream)  # creates the event handle
         return evs
 
-    # warm-up (not timed)
     for _ in range(args.warmup):
         layer.forward(x, y)
     torch.cuda.synchronize()
@@ -206,10 +257,9 @@ def run_ours(args, rank, world, local_rank):
     step_events = [events() for _ in range(args.steps)]
     auxes = [moe.make_aux(stage_events=ev, expert_offsets=offsets) for ev in step_events]
     torch.cuda.synchronize()
-    sampler = ClockSampler(local_rank) if rank == 0 else None
+    sampler = ClockSampler(local_rank) if sample_clocks else None
     time.sleep(0.3 if sampler else 0.0)
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -218,131 +268,254 @@ def run_ours(args, rank, world, local_rank):
         moe.check(moe.moe_layer_forward(layer.dims, layer._w, x, y, auxes[i], layer.workspace, None, stream))
     t1.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(world)
     clocks = sampler.stop() if sampler else None
     ms = max_over_ranks(t0.elapsed_time(t1), dev)
-    ms_per_step = ms / args.steps
 
-    # per-stage device time inside the timed region
     stage_ms = {n: 0.0 for n in moe.STAGE_NAMES}
     for ev in step_events:
         for i, n in enumerate(moe.STAGE_NAMES):
             stage_ms[n] += ev[2 * i].elapsed_time(ev[2 * i + 1]) / args.steps
 
-    # end to end through the public API: pinned host x -> device, forward, y -> pinned host
-    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-    x_host.copy_(x)
-    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    x_in = torch.empty_like(x)
-    for _ in range(max(1, min(args.warmup, 2))):
-        x_in.copy_(x_host, non_blocking=True)
-        layer.forward(x_in, y)
-        y_host.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        x_in.copy_(x_host, non_blocking=True)
-        layer.forward(x_in, y)
-        y_host.copy_(y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-    if world > 1:
-        torch.distributed.barrier()
-
+    e2e_ms = measure_e2e(layer, x, y, cfg, args, world)
     st, code = moe.moe_device_error()
     if st != moe.MOE_OK:
         raise RuntimeError(f"device fault {code} during the bench")
-    if rank != 0:
-        return None
+    return {"ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clocks, "launches": launches_per_step,
+            "offsets": offsets.cpu().numpy().astype(np.int64), "y_bytes": y.element_size()}
 
-    peaks = load_peaks()
-    value = job_throughput(cfg.T, args.steps, world, ms)
-    off = offsets.cpu().numpy()
-    work = stage_work(cfg, off, cfg.T)
-    dom = dominant_stage(cfg)
-    dom_ms = stage_ms[dom]
-    flops_step = float(cfg.flops_per_token()) * cfg.T
-    R = cfg.T * cfg.k
+
+def measure_e2e(layer, x, y, cfg, args, world: int) -> float:
+    """End to end through the public API (MoeLayer.forward): every step copies
+    its input from pinned host memory to the device and reads its output back
+    to pinned host memory.  Two device buffers each way let the copies of one
+    step overlap the compute of the neighbouring steps (a copy-in stream and a
+    copy-out stream, ordered by events); the timed region runs from before the
+    first copy-in to after the last copy-out."""
+    dev = x.device
+    compute = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x)
+    y_host = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):  # every event has been recorded once before it is waited on
+        ev_done[b].record(compute)
+        ev_out[b].record(compute)
+
+    def run(steps: int):
+        for i in range(steps):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_done[b])  # buffer b's previous step has read its x
+                x_dev[b].copy_(x_host, non_blocking=True)
+                ev_in[b].record(s_in)
+            compute.wait_event(ev_in[b])
+            compute.wait_event(ev_out[b])  # buffer b's previous y has been read back
+            layer.forward(x_dev[b], y_dev[b], stream=compute)
+            ev_done[b].record(compute)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+                ev_out[b].record(s_out)
+
+    run(max(2, min(args.warmup, 3)))
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(compute)
+    s_in.wait_event(e0)
+    run(args.steps)
+    compute.wait_event(ev_out[0])
+    compute.wait_event(ev_out[1])
+    e1.record(compute)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    barrier(world)
+    return ms
+
+
+def near_ties_from_scores(layer, x, cfg) -> int:
+    """Tokens of the whole batch whose device-side selection margin (k-th minus
+    (k+1)-th largest fp32 key s + b) is below NEAR_TIE: where a device and the
+    fp64 oracle may legitimately choose different experts.  Outside any timed
+    region; the scores come from the layer itself (aux output)."""
+    if cfg.k >= cfg.E:
+        return 0
+    s = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=x.device)
+    layer.forward(x, aux={"scores": s})
+    key = s + layer.weights["bias"][None, :]
+    top = torch.topk(key, cfg.k + 1, dim=1).values
+    return int(((top[:, cfg.k - 1] - top[:, cfg.k]) < NEAR_TIE).sum())
+
+
+def oracle_sample(cfg, layer, x, n_tokens: int, seed_offset: int = 0) -> tuple[dict, dict]:
+    """The oracle on a seeded sample of the workload's tokens: the parity of
+    the device output there (index sets, near ties, max|dy|/rms(y_ref)) and
+    the oracle's own throughput on the host cores (the CPU baseline).  Weight
+    generation is excluded from the oracle's time."""
+    import oracle
+    from oracle import inputs as oin
+
+    tokens = gen.sample_tokens(cfg, n_tokens) if seed_offset == 0 else np.sort(
+        np.random.default_rng(cfg.seed + 1000 + seed_offset).choice(cfg.T, size=min(n_tokens, cfg.T),
+                                                                    replace=False))
+    from dataclasses import replace
+
+    # the same step with an fp32 y (the bf16 y is its rounding), same workspace
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=x.device)
+    y = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device=x.device)
+    d = replace(layer.dims, T=cfg.T, y_out="f32")
+    moe.check(moe.moe_layer_forward(d, layer._w, x, y, moe.make_aux(topk_idx=idx), layer.workspace))
+    torch.cuda.synchronize()
+    sel = torch.as_tensor(tokens)
+    y_dev = y.cpu().to(torch.float64)[sel]
+    idx_dev = idx.cpu().to(torch.int64)[sel]
+
+    dense = oin.dense_weights(cfg)
+    xr = oin.x_rows(cfg, tokens)
+    gen_s = [0.0]
+
+    def provider(e):
+        t = time.perf_counter()
+        w = oin.expert_weights_raw(cfg, e)
+        gen_s[0] += time.perf_counter() - t
+        return w
+
+    t0 = time.perf_counter()
+    ref = oracle.layer_forward_streamed(cfg, dense, xr, provider)
+    oracle_s = time.perf_counter() - t0 - gen_s[0]
+    differ = (torch.sort(idx_dev, 1).values != torch.sort(ref["idx"], 1).values).any(1)
+    near = ref["margin"] < NEAR_TIE
+    if bool(differ.any()):
+        forced = ref["idx"].clone()
+        forced[differ] = idx_dev[differ]
+        ref = oracle.layer_forward_streamed(cfg, dense, xr, provider, forced_idx=forced)
+    rms = float(ref["y"].pow(2).mean().sqrt())
+    parity = {"tokens": len(tokens), "index_set_differences": int(differ.sum()),
+              "differences_without_near_tie": int((differ & ~near).sum()), "near_tie_tokens": int(near.sum()),
+              "max_abs_dy_over_rms": round(float((y_dev - ref["y"]).abs().max()) / rms, 6),
+              "tolerance": 3e-2 if cfg.routed == "mxfp4" else 1e-2,
+              "oracle": "fp64 C++ oracle (oracle/moe_oracle.cpp), storage-faithful bf16 rounding"}
+    cpu = {"value": round(len(tokens) / oracle_s, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
+           "kind": "oracle",
+           "sample": f"{len(tokens)} seeded tokens of the {cfg.name} workload (fp64 C++ oracle, "
+                     f"{oracle.num_threads()} std::thread workers; weight generation excluded)"}
+    return parity, cpu
+
+
+def workload_line(cfg, layer, x, args, world, rank, local_rank, peaks, headline: bool) -> dict:
+    m = measure_layer(layer, x, cfg, args, world, local_rank, sample_clocks=(rank == 0))
+    off = m["offsets"]
+    ms_step = m["ms"] / args.steps
     counts = np.diff(off)
-    bound = "tensor" if (work["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)) >= (
-        work["bytes"] / (peaks["hbm_gbs"] * 1e9)) else "hbm"
-    if bound == "tensor":
-        achieved = work["flops"] / (dom_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        unit = "TFLOP/s"
-    else:
-        achieved = work["bytes"] / (dom_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}_{dom}.json")
-    if os.path.exists(prof):
-        # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu
-        # capture of this workload (see the file for the command and kernel build)
-        with open(prof) as f:
-            traffic = json.load(f).get("dram_bytes_per_launch")
+    flops_step = float(cfg.flops_per_token()) * cfg.T
+    lb = layer_bytes(cfg, off, cfg.T, m["y_bytes"])
+    out = {
+        "value": round(job_throughput(cfg.T, args.steps, world, m["ms"]), 1),
+        "unit": "tokens/s",
+        "ms_per_step": round(ms_step, 4),
+        "tflops": round(flops_step / (ms_step / 1e3) / 1e12, 2),
+        "stage_ms": {k: round(v, 4) for k, v in m["stage_ms"].items()},
+        "roofline": gate_up_roofline(cfg, off, m["stage_ms"], peaks),
+        # the whole step against HBM: the bound of the weight-streaming decode step
+        "layer_hbm": {"bytes": lb, "achieved": round(lb / (ms_step / 1e3) / 1e9, 1), "peak": peaks["hbm_gbs"],
+                      "unit": "GB/s", "frac": round(lb / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                      "peak_source": f"{peaks['source']} HBM copy (read+write); this stream is read-dominated"},
+        "layer_tensor": {"flops": flops_step, "frac_of_sustained_bf16": round(
+            flops_step / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4)},
+        "e2e": {
+            "value": round(job_throughput(cfg.T, args.steps, world, m["e2e_ms"]), 1),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": x.numel() * x.element_size(),
+            "d2h_bytes_per_step": cfg.T * cfg.H * m["y_bytes"],
+            "how": "MoeLayer.forward with pinned-host copies in and out every step, double-buffered on copy streams",
+        },
+        "gpu_launches": m["launches"] * args.steps,
+        "clocks": m["clocks"],
+        "config": {
+            "workload": workload_name(cfg),
+            "tokens_per_step_per_gpu": cfg.T,
+            "y_dtype": layer.dims.y_out,
+            "parallelism": f"replicas x{world} (no data-path collective)",
+            "l2": "inputs larger than L2 (routed weights %.1f GB, x %.0f MB per step)" % (
+                3 * cfg.E * cfg.I * cfg.L * routed_weight_bytes_per_element(cfg) / 1e9, cfg.T * cfg.H * 2 / 1e6),
+            "expert_rows_max": int(counts.max()),
+            "expert_rows_min": int(counts.min()),
+            "touched_experts": int((counts > 0).sum()),
+        },
+    }
+    if world == 1:
+        out["near_tie_tokens"] = near_ties_from_scores(layer, x, cfg)
+        if not args.no_oracle:
+            parity, cpu = oracle_sample(cfg, layer, x, args.cpu_tokens)
+            out["parity"] = parity
+            out["cpu_baseline"] = cpu
+    return out
+
+
+def build_layer(cfg, dev, y_out: str, weights=None):
+    inputs = gen.device_layer(cfg, dev) if weights is None else weights
+    x = inputs.pop("x") if "x" in inputs else None
+    return moe.MoeLayer(dims_for(cfg, y_out), inputs), x, inputs
+
+
+def run_ours(args, rank, world, local_rank):
+    cfg = gen.CONFIGS[args.config]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    layer, x, weights = build_layer(cfg, dev, args.y_out)
+    line = workload_line(cfg, layer, x, args, world, rank, local_rank, peaks, headline=True)
+    stream = torch.cuda.current_stream(dev)
     out = {
         "metric": METRIC,
-        "value": round(value, 1),
+        "value": line["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 4),
+        "ms_per_step": line["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": cfg.act,
         "data": "synthetic (seeded Philox inputs, random-init weights of the K3 layer shape)",
-        "config": {
-            "workload": workload_name(cfg),
-            "tokens_per_step_per_gpu": cfg.T,
-            "y_dtype": args.y_out,
-            "parallelism": f"replicas x{world} (no data-path collective)",
-            "l2": "inputs larger than L2 (routed weights %.1f GB, x %.0f MB per step)" % (
-                3 * cfg.E * cfg.I * cfg.L * 2 / 1e9, cfg.T * cfg.H * 2 / 1e6),
-            "expert_rows_max": int(counts.max()),
-            "expert_rows_min": int(counts.min()),
-            "touched_experts": work["touched_experts"],
-        },
-        "tflops": round(flops_step / (ms_per_step / 1e3) / 1e12, 2),
-        "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-        "roofline": {
-            "kernel": f"tc_expert_kernel (2-CTA grouped gate/up + SiTU epilogue) = stage {dom}",
-            "bound": bound,
-            "achieved": round(achieved, 1),
-            "peak": peak,
-            "unit": unit,
-            "frac": round(achieved / peak, 4),
-            "traffic": traffic,
-            "peak_source": peaks["source"] + (" sustained bf16" if bound == "tensor" else " HBM copy"),
-            "algorithmic": {"flops": work["flops"], "bytes": work["bytes"]},
-        },
-        "e2e": {
-            "value": round(job_throughput(cfg.T, args.steps, world, e2e_ms), 1),
-            "unit": "tokens/s",
-            "h2d_bytes_per_step": x.numel() * x.element_size(),
-            "d2h_bytes_per_step": y.numel() * y.element_size(),
-        },
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks,
     }
+    out.update({k: v for k, v in line.items() if k not in ("value", "unit", "ms_per_step")})
     out["qb_update"] = measure_qb(cfg, dev, stream, peaks)
-    if world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, seed_offset=0)
-    return out
+
+    extra = [] if args.no_extra_lines or args.config != "prefill" else ["decode", "mxfp4"]
+    for name in extra:
+        sub = gen.CONFIGS[name]
+        if name == "decode":
+            # same weights as the prefill layer (same seed and shapes), the
+            # decode workload's own bias, and the first 256 token rows of x
+            w = dict(weights)
+            w["bias"] = torch.from_numpy(gen.bias(sub)).to(dev)
+            lay = moe.MoeLayer(dims_for(sub, args.y_out), w)
+            xs = x[: sub.T].contiguous()
+            out["decode"] = workload_line(sub, lay, xs, args, world, rank, local_rank, peaks, headline=False)
+            del lay, xs, w
+        else:
+            # the bf16 routed weights are no longer needed
+            del layer, weights, x
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            layer, x, weights = build_layer(sub, dev, args.y_out)
+            out[name] = workload_line(sub, layer, x, args, world, rank, local_rank, peaks, headline=False)
+    return out if rank == 0 else None
 
 
 # ----------------------------------------------------------------------------------- the oracle
 def cpu_baseline(cfg, n_tokens: int, seed_offset: int = 0, dense=None) -> dict:
-    """The fp64 CPU oracle on a bounded sample of the workload's tokens.  The
-    time counts the oracle's own work (reading bf16 / MXFP4 weights into fp64
+    """The fp64 C++ oracle on a bounded sample of the workload's tokens.  The
+    time counts the oracle's own work (decoding the bf16 / MXFP4 weight bits
     and the layer arithmetic); generating the synthetic weights is excluded."""
     import oracle
     from oracle import inputs as oin
@@ -355,31 +528,30 @@ def cpu_baseline(cfg, n_tokens: int, seed_offset: int = 0, dense=None) -> dict:
 
     def provider(e):
         t = time.perf_counter()
-        raw = [gen.host_expert(cfg, n, e) for n in ("Wg", "Wv", "Wo")]
+        w = oin.expert_weights_raw(cfg, e)
         gen_s[0] += time.perf_counter() - t
-        out = []
-        for r in raw:
-            out.append(oracle.mxfp4_dequant(*r) if isinstance(r, tuple) else oin.to_f64(r))
-        return tuple(out)
+        return w
 
     t0 = time.perf_counter()
     oracle.layer_forward_streamed(cfg, dense, x, provider)
     total = time.perf_counter() - t0 - gen_s[0]
-    return {"value": round(len(sample) / total, 3), "unit": "tokens/s", "cores": torch.get_num_threads(),
+    return {"value": round(len(sample) / total, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"{len(sample)} seeded tokens of the {cfg.name} workload (fp64, torch CPU, "
-                      f"{torch.get_num_threads()} threads; weight generation excluded)"}
+            "sample": f"{len(sample)} seeded tokens of the {cfg.name} workload (fp64 C++ oracle, "
+                      f"{oracle.num_threads()} std::thread workers; weight generation excluded)"}
 
 
 def run_reference(args, rank, world):
     from oracle import inputs as oin
 
     cfg = gen.CONFIGS[args.config]
-    per_step = max(1, args.cpu_tokens // 4)
+    per_step = max(1, args.cpu_tokens // 8)
     dense = oin.dense_weights(cfg)
     times = []
+    cores = None
     for i in range(args.warmup + args.steps):
         cb = cpu_baseline(cfg, per_step, seed_offset=i, dense=dense)
+        cores = cb["cores"]
         if i >= args.warmup:
             times.append(per_step / cb["value"])
     total = sum(times)
@@ -387,7 +559,7 @@ def run_reference(args, rank, world):
     return {
         "impl": "reference",
         "metric": METRIC,
-        "value": round(value, 3),
+        "value": round(value, 4),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -399,10 +571,10 @@ def run_reference(args, rank, world):
         "dtype": "f64",
         "data": "synthetic (seeded Philox inputs)",
         "config": {"workload": workload_name(cfg), "tokens_per_step": per_step},
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": torch.get_num_threads(),
-                         "kind": "oracle",
-                         "sample": f"{per_step} seeded tokens per step of the {cfg.name} workload"},
-        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} seeded tokens per step of the {cfg.name} workload "
+                                   f"(fp64 C++ oracle, {cores} std::thread workers)"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
@@ -414,8 +586,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(gen.CONFIGS), default="prefill")
     ap.add_argument("--y-out", choices=["bf16", "f32"], default="bf16")
-    ap.add_argument("--cpu-tokens", type=int, default=8)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=16)
+    ap.add_argument("--no-oracle", "--no-cpu-baseline", dest="no_oracle", action="store_true",
+                    help="skip the oracle sample (parity + CPU baseline)")
+    ap.add_argument("--no-extra-lines", action="store_true", help="measure only --config (no decode / mxfp4 lines)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -201,21 +201,62 @@ MOE_API moe_status moe_combine(const moe_dims* d, const float* y_perm, const int
 MOE_API moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void* x, void* y, const moe_aux* aux,
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The x-side dense steps of the layer ("K3のエキスパートは896個の小型LLMではない":
+ * z = W_down x; the shared experts' E_shared,i(x) up to their down projection):
+ *   z[T, L]        = x[T, H] . Wdown[L, H]^T, stored in the activation type;
+ *   h_s[T, S*Is]   = SiTU-GLU(x . Wsg[i]^T, x . Wsv[i]^T) for i < S, expert i in
+ *                    columns [i*Is, (i+1)*Is), stored in the activation type.
+ * Reads w->Wdown, w->Wsg, w->Wsv only.  h_s may be NULL when S = 0.  For
+ * callers that run the layer stage by stage (e.g. with the routed experts on
+ * other GPUs); moe_layer_forward does the same work internally. */
+MOE_API moe_status moe_latent_shared(const moe_dims* d, const moe_weights* w, const void* x, void* z, void* h_s,
+                                     moe_stream_t stream);
+
+/* The output projection (same section: y = E1_shared(x) + E2_shared(x) +
+ * W_up RMSNorm(u)), as one GEMM over the concatenation [h_s | n]:
+ *   y[T, H] = sum_i h_s[:, i*Is:(i+1)*Is] . Wso[i]^T + n[T, L] . Wup[H, L]^T
+ * in type y_out, accumulated in fp32.  Reads w->Wso, w->Wup only. */
+MOE_API moe_status moe_output(const moe_dims* d, const moe_weights* w, const void* h_s, const void* n, void* y,
+                              moe_stream_t stream);
+
+/* Routed experts over rows that arrive as n_blocks expert-major blocks of the
+ * same E experts -- the rows an expert-parallel rank receives from each
+ * sending rank (the pages' MoonEP, "Kimi K3の二軸スケーリング戦略とは何か",
+ * section "MoonEP：疎なMoEを実際に動かす通信層"; the expert computation is that
+ * of moe_expert_ffn).
+ *  - x_rows [n_rows, L] (act type); block b's rows of expert e are
+ *    block_offsets[b*(E+1) + e] .. block_offsets[b*(E+1) + e + 1] - 1 (int32,
+ *    absolute row numbers in x_rows, non-decreasing within a block); rows no
+ *    block names are not computed.
+ *  - y_rows [n_rows, L] fp32: y_rows[r] = W_o[e] SiTU-GLU(W_g[e] x_r, W_v[e] x_r)
+ *    for the expert e of row r (same positions as x_rows).
+ *  - w->Wg / Wv / Wo (and Sg / Sv / So for MXFP4) hold the E experts of this
+ *    call (e.g. one rank's partition); other weight fields are not read.
+ *  - Workspace: moe_expert_ffn_blocks_workspace_size(d, n_rows, n_blocks)
+ *    bytes, 256-byte aligned.  Offsets outside [0, n_rows] are recorded as a
+ *    device fault (moe_device_error) and their segment is skipped.
+ * d->T and d->k are not used. */
+MOE_API size_t moe_expert_ffn_blocks_workspace_size(const moe_dims* d, int64_t n_rows, int32_t n_blocks);
+MOE_API moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const void* x_rows, int64_t n_rows,
+                                         const int32_t* block_offsets, int32_t n_blocks, float* y_rows, void* ws,
+                                         size_t ws_bytes, moe_stream_t stream);
+
 /* Allocation-free variant of moe_permute (the pages have no counterpart; this
  * is a library facility).  For callers that cannot allocate device memory when
  * they route tokens -- code running inside an allocator or memory-pool
  * callback, runtimes that forbid cudaMalloc after start-up to keep a fixed
  * footprint, hosts that own no allocator -- it takes no workspace: its scratch
- * (per-tile expert counts, in-tile ranks, tile table) lives in a fixed device
- * array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES inside the library, which every
- * GPU that loads the library keeps until the process exits.  The call itself
- * allocates nothing.  Arguments and outputs are those of moe_permute.
- *  - Scratch needed: 256-byte-rounded sum of 4*ceil(T/128)*E, 4*T*k,
- *    16*(ceil(T*k/128) + E) and 16 bytes; larger dims return
- *    MOE_ERR_INVALID_ARG (K3 shape: up to about 40k tokens).
+ * (per-tile expert counts and in-tile ranks) lives in a fixed device array of
+ * MOE_PERMUTE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library keeps until the process exits.  The call itself allocates
+ * nothing.  Arguments and outputs are those of moe_permute.
+ *  - Scratch needed: 4*ceil(T/128)*E and 4*T*k bytes, each rounded up to 256;
+ *    larger dims return MOE_ERR_INVALID_ARG (K3 shape: up to about 45k tokens).
  *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any stream
- *    capture.
+ *    device and context, with that device current); make that first call
+ *    before any stream capture.  After cudaDeviceReset (or with another
+ *    context current) the next call looks it up again, so that call too must
+ *    come before any capture.
  *  - All calls share the one array: calls whose work overlaps on the GPU
  *    (different streams, or different host threads without ordering) race and
  *    give wrong results.  Successive calls on one stream are safe; nothing in

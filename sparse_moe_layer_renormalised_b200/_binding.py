@@ -32,6 +32,10 @@ EXPORTED = (
     "moe_last_launch_count",
     "moe_permute_noalloc",
     "moe_qb_bias_update",
+    "moe_latent_shared",
+    "moe_output",
+    "moe_expert_ffn_blocks_workspace_size",
+    "moe_expert_ffn_blocks",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -103,8 +107,14 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_noalloc.argtypes = [pd, vp, vp, vp, vp, vp, vp, vp]
         f32 = ctypes.c_float
         L.moe_qb_bias_update.argtypes = [pd, vp, vp, vp, vp, vp, i32, f32, f32, vp]
+        L.moe_latent_shared.argtypes = [pd, pw, vp, vp, vp, vp]
+        L.moe_output.argtypes = [pd, pw, vp, vp, vp, vp]
+        L.moe_expert_ffn_blocks_workspace_size.argtypes = [pd, ctypes.c_int64, ctypes.c_int32]
+        L.moe_expert_ffn_blocks_workspace_size.restype = ctypes.c_size_t
+        L.moe_expert_ffn_blocks.argtypes = [pd, pw, vp, ctypes.c_int64, vp, ctypes.c_int32, vp, vp, ctypes.c_size_t,
+                                            vp]
         for f in EXPORTED:
-            if f not in ("moe_workspace_size", "moe_status_str"):
+            if f not in ("moe_workspace_size", "moe_status_str", "moe_expert_ffn_blocks_workspace_size"):
                 getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -228,6 +238,28 @@ def moe_qb_bias_update(d, scores, bias_in, bias_out, quantile_out, hist, nbins: 
     include/moe.h); hist is an [E, nbins] uint32 workspace, overwritten."""
     return lib().moe_qb_bias_update(ctypes.byref(_dims(d)), _ptr(scores), _ptr(bias_in), _ptr(bias_out),
                                     _ptr(quantile_out), _ptr(hist), int(nbins), float(lo), float(hi), _stream(stream))
+
+
+def moe_latent_shared(d, weights: moe_weights, x, z, h_s, stream=None) -> int:
+    return lib().moe_latent_shared(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(x), _ptr(z), _ptr(h_s),
+                                   _stream(stream))
+
+
+def moe_output(d, weights: moe_weights, h_s, n, y, stream=None) -> int:
+    return lib().moe_output(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(h_s), _ptr(n), _ptr(y),
+                            _stream(stream))
+
+
+def moe_expert_ffn_blocks_workspace_size(d, n_rows: int, n_blocks: int) -> int:
+    return int(lib().moe_expert_ffn_blocks_workspace_size(ctypes.byref(_dims(d)), int(n_rows), int(n_blocks)))
+
+
+def moe_expert_ffn_blocks(d, weights: moe_weights, x_rows, n_rows: int, block_offsets, n_blocks: int, y_rows, ws,
+                          ws_bytes=None, stream=None) -> int:
+    ws_bytes = _nbytes(ws) if ws_bytes is None else ws_bytes
+    return lib().moe_expert_ffn_blocks(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(x_rows), int(n_rows),
+                                       _ptr(block_offsets), int(n_blocks), _ptr(y_rows), _ptr(ws), ws_bytes,
+                                       _stream(stream))
 
 
 def moe_status_str(status: int) -> str:

@@ -6,11 +6,13 @@
 #include <stdint.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "combine.cuh"
 #include "gemm_expert.cuh"
+#include "gemm_expert2.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -447,8 +449,79 @@ cudaError_t launch_expert(int cg, bool mx, const ExMaps& maps, const ExParams& p
                  : launch_expert_inst<EPI, PAIRED, 1, false>(maps, p, s);
 }
 
+template <int EPI, bool PAIRED, int CG>
+cudaError_t launch_expert2_inst(const X2Maps& maps, const X2Params& p, cudaStream_t s) {
+  auto kern = tc_expert2_kernel<EPI, PAIRED, CG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(X2_SMEM));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(X2_THREADS);
+  cfg.dynamicSmemBytes = X2_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static int pairs_cache[128] = {};  // per instantiation and device
+    cfg.gridDim = dim3(2 * cluster_pairs(kern, cfg, pairs_cache));
+  } else {
+    cfg.gridDim = dim3(num_sms());
+    cfg.numAttrs = 0;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, maps, p);
+}
+
+// The two-weight-tile expert kernel (gemm_expert2.cuh) runs bf16 weights when
+// the weight tiles divide evenly; MOE_EXPERT_ONE_TILE=1 in the environment
+// selects the one-tile kernel instead (both compute the same result; used to
+// compare them).
+bool use_two_tile(const moe_dims& d, bool paired) {
+  if (d.act != MOE_BF16 || d.routed != MOE_BF16) return false;
+  const char* env = std::getenv("MOE_EXPERT_ONE_TILE");
+  if (env != nullptr && env[0] == '1') return false;
+  const int rows = 128 * expert_cg(d);
+  return paired ? d.I % rows == 0 : d.L % rows == 0;
+}
+
+moe_status stage_expert2(const moe_dims& d, bool paired, const void* w0, const void* w1, const void* act, int K,
+                         const int4* tile_table, const int32_t* num_tiles, void* out, cudaStream_t s) {
+  const long long R = d.T * d.k;
+  const int cg = expert_cg(d);
+  const int rows_per_expert = paired ? d.I : d.L;
+  X2Maps maps;
+  std::memset(&maps, 0, sizeof maps);
+  const uint64_t wrows = static_cast<uint64_t>(d.E) * rows_per_expert;
+  bool ok = make_token_maps(maps.b, act, static_cast<uint64_t>(R), K) && make_map(&maps.a0, w0, wrows, K, K, 128);
+  if (paired) ok = ok && make_map(&maps.a1, w1, wrows, K, K, 128);
+  if (!ok) return MOE_ERR_CUDA;
+  X2Params p{};
+  p.tile_table = tile_table;
+  p.num_tiles_dev = num_tiles;
+  p.n_wtiles = rows_per_expert / (128 * cg);
+  p.n_items = paired ? p.n_wtiles : (p.n_wtiles + 1) / 2;
+  p.w_rows_per_expert = rows_per_expert;
+  p.num_k_blocks = K / EX_BK;
+  p.out = out;
+  p.ldo = rows_per_expert;
+  p.out_cols = rows_per_expert;
+  p.situ_c = d.situ_c;
+  p.fault_site = paired ? 170 : 180;
+  cudaError_t e;
+  if (paired)
+    e = cg == 2 ? launch_expert2_inst<kEpiSituBF16, true, 2>(maps, p, s)
+                : launch_expert2_inst<kEpiSituBF16, true, 1>(maps, p, s);
+  else
+    e = cg == 2 ? launch_expert2_inst<kEpiF32, false, 2>(maps, p, s) : launch_expert2_inst<kEpiF32, false, 1>(maps, p, s);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const void* z_perm,
-                                const int4* tile_table, const int32_t* num_tiles, void* h_perm, cudaStream_t s) {
+                                const int4* tile_table, const int32_t* num_tiles, void* h_perm, cudaStream_t s,
+                                int max_tiles = -1) {
   const long long R = d.T * d.k;
   ++g_last_launches;
   if (d.act != MOE_BF16) {
@@ -458,7 +531,7 @@ moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const v
     g.M = R;
     g.tile_table = tile_table;
     g.num_m_tiles_dev = num_tiles;
-    g.max_m_tiles = static_cast<int>(cdiv(R, 128) + d.E);
+    g.max_m_tiles = max_tiles > 0 ? max_tiles : static_cast<int>(cdiv(R, 128) + d.E);
     g.N = d.I;
     g.b_rows_per_expert = d.I;
     g.nseg = 1;
@@ -469,6 +542,7 @@ moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const v
     g.situ_c = d.situ_c;
     return run_gemm_simt(g, s);
   }
+  if (use_two_tile(d, true)) return stage_expert2(d, true, w.Wg, w.Wv, z_perm, d.L, tile_table, num_tiles, h_perm, s);
   const int cg = expert_cg(d);
   const bool mx = d.routed == MOE_MXFP4;
   ExMaps maps;
@@ -496,7 +570,7 @@ moe_status stage_expert_gate_up(const moe_dims& d, const moe_weights& w, const v
 }
 
 moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void* h_perm, const int4* tile_table,
-                             const int32_t* num_tiles, float* y_perm, cudaStream_t s) {
+                             const int32_t* num_tiles, float* y_perm, cudaStream_t s, int max_tiles = -1) {
   const long long R = d.T * d.k;
   ++g_last_launches;
   if (d.act != MOE_BF16) {
@@ -505,7 +579,7 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
     g.M = R;
     g.tile_table = tile_table;
     g.num_m_tiles_dev = num_tiles;
-    g.max_m_tiles = static_cast<int>(cdiv(R, 128) + d.E);
+    g.max_m_tiles = max_tiles > 0 ? max_tiles : static_cast<int>(cdiv(R, 128) + d.E);
     g.N = d.L;
     g.b_rows_per_expert = d.L;
     g.nseg = 1;
@@ -515,6 +589,7 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
     g.situ_c = d.situ_c;
     return run_gemm_simt(g, s);
   }
+  if (use_two_tile(d, false)) return stage_expert2(d, false, w.Wo, nullptr, h_perm, d.I, tile_table, num_tiles, y_perm, s);
   const int cg = expert_cg(d);
   const bool mx = d.routed == MOE_MXFP4;
   ExMaps maps;
@@ -600,6 +675,29 @@ moe_status check_scales(const moe_dims& d, const moe_weights& w) {
     if (!mx && p != nullptr) return MOE_ERR_INVALID_ARG;
   }
   return MOE_OK;
+}
+
+// Workspace of moe_expert_ffn_blocks: h for every row, and a tile table for
+// up to ceil(n_rows / 128) + E * n_blocks tiles.
+struct BlocksWsLayout {
+  size_t h, tile_table, num_tiles, total;
+  int max_tiles;
+};
+
+BlocksWsLayout blocks_ws_layout(const moe_dims& d, long long n_rows, int n_blocks) {
+  BlocksWsLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, kAlign);
+    return o;
+  };
+  l.max_tiles = static_cast<int>(cdiv(n_rows, 128) + static_cast<long long>(d.E) * n_blocks);
+  l.h = take(static_cast<size_t>(n_rows) * d.I * act_bytes(d));
+  l.tile_table = take(static_cast<size_t>(l.max_tiles) * 16);
+  l.num_tiles = take(16);
+  l.total = off;
+  return l;
 }
 
 bool ws_ok(const moe_dims& d, const void* ws, size_t ws_bytes) {
@@ -795,6 +893,79 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
   return st;
 }
 
+moe_status moe_latent_shared(const moe_dims* d, const moe_weights* w, const void* x, void* z, void* h_s,
+                             moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (w == nullptr || x == nullptr || z == nullptr || !aligned16(x) || !aligned16(z) || w->Wdown == nullptr ||
+      !aligned16(w->Wdown))
+    return MOE_ERR_INVALID_ARG;
+  if (d->S > 0 && (h_s == nullptr || !aligned16(h_s) || w->Wsg == nullptr || w->Wsv == nullptr ||
+                   !aligned16(w->Wsg) || !aligned16(w->Wsv)))
+    return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = stage_dense(*d, d->act == MOE_BF16 ? kEpiBF16 : kEpiF32, x, d->H, w->Wdown, d->L, d->H, z, d->L, 120,
+                        s)) != MOE_OK)
+    return st;
+  if (d->S > 0) st = stage_shared_gate_up(*d, *w, x, h_s, s);
+  return st;
+}
+
+moe_status moe_output(const moe_dims* d, const moe_weights* w, const void* h_s, const void* n, void* y,
+                      moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (w == nullptr || n == nullptr || y == nullptr || !aligned16(n) || !aligned16(y) || w->Wup == nullptr ||
+      !aligned16(w->Wup))
+    return MOE_ERR_INVALID_ARG;
+  if (d->S > 0 && (h_s == nullptr || !aligned16(h_s) || w->Wso == nullptr || !aligned16(w->Wso)))
+    return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  return stage_output(*d, *w, h_s, n, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_expert_ffn_blocks_workspace_size(const moe_dims* d, int64_t n_rows, int32_t n_blocks) {
+  if (!dims_ok(d) || n_rows < 0 || n_blocks < 1) return 0;
+  return blocks_ws_layout(*d, n_rows, n_blocks).total;
+}
+
+moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const void* x_rows, int64_t n_rows,
+                                 const int32_t* block_offsets, int32_t n_blocks, float* y_rows, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (w == nullptr || x_rows == nullptr || block_offsets == nullptr || y_rows == nullptr || n_rows < 0 ||
+      n_blocks < 1 || n_rows > 0x7fffffffLL)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->Wg) || !aligned16(w->Wv) || !aligned16(w->Wo) || w->Wg == nullptr || w->Wv == nullptr ||
+      w->Wo == nullptr || !aligned16(x_rows) || !aligned16(y_rows))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_scales(*d, *w)) != MOE_OK) return st;
+  const BlocksWsLayout L = blocks_ws_layout(*d, n_rows, n_blocks);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < L.total)
+    return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (n_rows == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The stages size their row tensor maps from d->T * d->k: describe the rows as
+  // n_rows single-slot tokens.
+  moe_dims dr = *d;
+  dr.T = n_rows;
+  dr.k = 1;
+  tile_table_blocks_kernel<<<1, 1024, 0, s>>>(block_offsets, n_blocks, d->E, n_rows, expert_tile_rows(dr),
+                                              at<int4>(ws, L.tile_table), at<int32_t>(ws, L.num_tiles));
+  ++g_last_launches;
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  const int4* table = at<int4>(ws, L.tile_table);
+  const int32_t* n_tiles = at<int32_t>(ws, L.num_tiles);
+  st = stage_expert_gate_up(dr, *w, x_rows, table, n_tiles, at<void>(ws, L.h), s, L.max_tiles);
+  if (st != MOE_OK) return st;
+  return stage_expert_down(dr, *w, at<void>(ws, L.h), table, n_tiles, y_rows, s, L.max_tiles);
+}
+
 moe_status moe_device_error(int* code, moe_stream_t stream) {
   if (code == nullptr) return MOE_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -819,8 +990,8 @@ moe_status moe_device_error(int* code, moe_stream_t stream) {
 // runtime that forbids cudaMalloc after start-up so its memory footprint stays
 // fixed, or a host that hands this library its inputs and outputs but owns no
 // allocator of its own.  This variant keeps its scratch (per-tile expert
-// counts, in-tile ranks, tile table) in a file-scope device array instead of a
-// caller workspace.  The array is part of the library image: every GPU that
+// counts and in-tile ranks) in a file-scope device array instead of a caller
+// workspace.  The array is part of the library image: every GPU that
 // loads the library holds it until the process exits.
 namespace moe {
 namespace {
@@ -829,7 +1000,7 @@ constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(MOE_PERMUTE_NOALLOC_
 static __device__ __align__(256) uint8_t g_permute_scratch[kNoAllocScratchBytes];
 
 struct NoAllocLayout {
-  size_t tile_base, rank, tile_table, num_m_tiles, total;
+  size_t tile_base, rank, total;
 };
 
 NoAllocLayout noalloc_layout(const moe_dims& d) {
@@ -843,28 +1014,55 @@ NoAllocLayout noalloc_layout(const moe_dims& d) {
   const size_t T = static_cast<size_t>(d.T), R = T * d.k;
   l.tile_base = take(static_cast<size_t>(cdiv(d.T, PERM_TILE)) * d.E * 4);
   l.rank = take(R * 4);
-  l.tile_table = take((static_cast<size_t>(cdiv(static_cast<long long>(R), TC_BM)) + d.E) * 16);
-  l.num_m_tiles = take(16);
   l.total = off;
   return l;
 }
 
-// Device address of g_permute_scratch on the current device.  The host-side
+// Device address of g_permute_scratch in the current context.  The host-side
 // name of a __device__ array is only a stand-in, so the address is asked for
-// once per device (with that device current) and cached.
+// with the device current and cached per device together with the context it
+// belongs to; a different current context (after cudaDeviceReset, or a
+// context the caller created) makes it ask again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  return fn;
+}
+
+struct NoAllocCache {
+  CUcontext ctx;
+  void* ptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[128] = {};
+NoAllocCache g_noalloc[128] = {};
 
 moe_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return MOE_ERR_CUDA;
+  CtxGetCurrentFn ctx_fn = ctx_get_current_fn();
+  if (ctx_fn == nullptr) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  if (ctx_fn(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  NoAllocCache& c = g_noalloc[dev];
+  if (c.ptr == nullptr || ctx == nullptr || c.ctx != ctx) {
+    // The first runtime call with the device current creates its primary
+    // context if needed; the context is read again after it.
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    if (ctx_fn(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MOE_ERR_CUDA;
+    c.ctx = ctx;
+    c.ptr = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = c.ptr;
   return MOE_OK;
 }
 
@@ -894,8 +1092,9 @@ extern "C" moe_status moe_permute_noalloc(const moe_dims* d, const int32_t* topk
   int32_t* rank = at<int32_t>(scratch, L.rank);
   perm_rank_kernel<<<static_cast<unsigned>(ntiles), PERM_TILE, static_cast<size_t>(d->E) * 16, s>>>(
       topk_idx, d->T, d->E, d->k, tile_base, rank);
-  perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d->E, nullptr, expert_offsets, 128,
-                                      at<int4>(scratch, L.tile_table), at<int32_t>(scratch, L.num_m_tiles));
+  // no grouped GEMM follows, so no tile table is built
+  perm_scan_kernel<<<1, 1024, 0, s>>>(tile_base, static_cast<int>(ntiles), d->E, nullptr, expert_offsets,
+                                      expert_tile_rows(*d), nullptr, nullptr);
   const long long pairs = d->T * d->k;
   perm_scatter_kernel<<<static_cast<unsigned>(cdiv(pairs, 256)), 256, 0, s>>>(
       topk_idx, d->T, d->E, d->k, tile_base, rank, expert_offsets, perm_token, inv_perm);

@@ -168,7 +168,8 @@ __device__ __forceinline__ void emit_tiles(int e, int off, int cnt, int first, i
 
 // One block of 1024 threads, thread = expert.  Turns the per-tile counts into
 // per-tile exclusive bases (in place), the expert counts, the CSR offsets, the
-// tile table and its length.
+// tile table and its length (tile_table / num_m_tiles may be NULL when the
+// caller runs no grouped GEMM on the result).
 __global__ void __launch_bounds__(1024)
     perm_scan_kernel(int32_t* __restrict__ tile_counts, int ntiles, int E, int32_t* __restrict__ counts_out,
                      int32_t* __restrict__ offsets, int max_tile_rows, int4* __restrict__ tile_table,
@@ -192,11 +193,11 @@ __global__ void __launch_bounds__(1024)
   if (e < E) {
     offsets[e] = incl_off - cnt;
     if (counts_out != nullptr) counts_out[e] = cnt;
-    emit_tiles(e, incl_off - cnt, cnt, incl_mt - mt, max_tile_rows, tile_table);
+    if (tile_table != nullptr) emit_tiles(e, incl_off - cnt, cnt, incl_mt - mt, max_tile_rows, tile_table);
   }
   if (e == E - 1) {
     offsets[E] = incl_off;
-    *num_m_tiles = incl_mt;
+    if (num_m_tiles != nullptr) *num_m_tiles = incl_mt;
   }
 }
 
@@ -222,6 +223,42 @@ __global__ void __launch_bounds__(1024)
   const int mt = tiles_of(cnt, max_tile_rows);
   const int incl_mt = block_incl_scan_1024(mt, buf);
   if (e < E) emit_tiles(e, off, cnt, incl_mt - mt, max_tile_rows, tile_table);
+  if (e == E - 1) *num_m_tiles = incl_mt;
+}
+
+// Tile table over n_blocks CSR blocks of the same E experts (rows received
+// from several ranks, each block expert-major): block b's rows of expert e are
+// offsets[b*(E+1)+e] .. offsets[b*(E+1)+e+1]-1.  Tiles are emitted expert by
+// expert (all blocks of expert 0, then expert 1, ...), so the tiles of one
+// expert stay adjacent in the grouped GEMM's work order.  Bad offsets are
+// recorded as a fault and that segment gets no rows.
+__global__ void __launch_bounds__(1024)
+    tile_table_blocks_kernel(const int32_t* __restrict__ offsets, int n_blocks, int E, long long max_rows,
+                             int max_tile_rows, int4* __restrict__ tile_table, int32_t* __restrict__ num_m_tiles) {
+  __shared__ int buf[1024];
+  const int e = threadIdx.x;
+  int mt = 0;
+  if (e < E) {
+    for (int b = 0; b < n_blocks; ++b) {
+      const int32_t* o = offsets + static_cast<long long>(b) * (E + 1);
+      const int off = o[e], end = o[e + 1];
+      if (off < 0 || end < off || end > max_rows)
+        record_fault(kFaultOffsets);
+      else
+        mt += tiles_of(end - off, max_tile_rows);
+    }
+  }
+  const int incl_mt = block_incl_scan_1024(mt, buf);
+  if (e < E) {
+    int first = incl_mt - mt;
+    for (int b = 0; b < n_blocks; ++b) {
+      const int32_t* o = offsets + static_cast<long long>(b) * (E + 1);
+      const int off = o[e], end = o[e + 1];
+      if (off < 0 || end < off || end > max_rows) continue;
+      emit_tiles(e, off, end - off, first, max_tile_rows, tile_table);
+      first += tiles_of(end - off, max_tile_rows);
+    }
+  }
   if (e == E - 1) *num_m_tiles = incl_mt;
 }
 

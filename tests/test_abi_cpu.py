@@ -25,7 +25,7 @@ def _dims(**kw):
 
 def test_library_exports_every_declared_symbol():
     names = _declared()
-    assert len(names) == 11
+    assert len(names) == 15
     lib = ctypes.CDLL(moe.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -137,3 +137,20 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(b, "_lib", None)
     with pytest.raises(moe.MoeLibraryMissing):
         b.lib()
+
+
+def test_stage_entry_points_validate_before_launching():
+    """moe_latent_shared / moe_output / moe_expert_ffn_blocks reject bad
+    arguments on the host (no GPU needed: nothing is launched)."""
+    d = _dims(T=64)
+    w = moe.make_weights(Wdown=FAKE, Wup=FAKE, Wsg=FAKE, Wsv=FAKE, Wso=FAKE, Wg=FAKE, Wv=FAKE, Wo=FAKE)
+    assert moe.moe_latent_shared(d, w, None, FAKE, FAKE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_latent_shared(d, w, FAKE + 4, FAKE, FAKE) == moe.MOE_ERR_INVALID_ARG  # misaligned x
+    assert moe.moe_output(d, w, FAKE, None, FAKE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_output(_dims(k=200), w, FAKE, FAKE, FAKE) == moe.MOE_ERR_INVALID_ARG
+    n = moe.moe_expert_ffn_blocks_workspace_size(d, 1000, 4)
+    assert n > 0 and n > moe.moe_expert_ffn_blocks_workspace_size(d, 1000, 1)
+    assert moe.moe_expert_ffn_blocks_workspace_size(d, 1000, 0) == 0
+    assert moe.moe_expert_ffn_blocks(d, w, FAKE, 1000, FAKE, 0, FAKE, FAKE, n) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_expert_ffn_blocks(d, w, FAKE, 1000, FAKE, 4, FAKE, FAKE, n - 1) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_expert_ffn_blocks(d, w, FAKE, -1, FAKE, 4, FAKE, FAKE, n) == moe.MOE_ERR_INVALID_ARG

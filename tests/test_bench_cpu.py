@@ -56,7 +56,7 @@ def test_reference_arm_prints_one_contract_line():
     """`bench.py --impl reference` runs the oracle on the host and prints one
     JSON line with the contract's keys (tiny layer, one timed step)."""
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny", "--steps", "1",
-                        "--warmup", "3", "--cpu-tokens", "4"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+                        "--warmup", "3", "--cpu-tokens", "8"], cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
     assert len(lines) == 1

@@ -120,10 +120,17 @@ def test_combine_rmsnorm(T, L, k, act):
 
 
 # ------------------------------------------------------------------------------ experts
+@pytest.mark.parametrize("kernel", ["two_tile", "one_tile"])
 @pytest.mark.parametrize("T,L", [(512, 1024), (37, 1024), (300, 1152)])
-def test_expert_ffn_mid_dims(T, L):
+def test_expert_ffn_mid_dims(T, L, kernel, monkeypatch):
     # L = 1024 runs the expert GEMMs on CTA pairs; L = 1152 (not a multiple of
-    # 256) on single CTAs.
+    # 256) on single CTAs, where the down projection's 9 weight tiles leave the
+    # last two-tile item with one tile.  bf16 weights run the two-weight-tile
+    # kernel unless MOE_EXPERT_ONE_TILE=1 selects the one-tile kernel.
+    if kernel == "one_tile":
+        monkeypatch.setenv("MOE_EXPERT_ONE_TILE", "1")
+    else:
+        monkeypatch.delenv("MOE_EXPERT_ONE_TILE", raising=False)
     cfg = gen.CONFIGS["mid"].with_(L=L)
     E, k, L, I = cfg.E, cfg.k, cfg.L, cfg.I
     d = dims_for(cfg, T=T)
