@@ -165,6 +165,20 @@ def layer_bytes(cfg, offsets: np.ndarray, T: int, y_bytes: int) -> float:
     return routed + dense + T * cfg.H * es + T * cfg.H * y_bytes
 
 
+def gate_up_kernel(cfg) -> str:
+    """The routed gate/up kernel the library runs for this workload (the rule
+    of moe_api.cu's use_two_tile: bf16 weights whose tiles divide evenly take
+    the two-weight-tile kernel when the average expert has fewer than 64 rows,
+    or as MOE_EXPERT_KERNEL forces; MXFP4 takes the one-tile kernel)."""
+    cg = 2 if (cfg.I % 128 == 0 and cfg.L % 256 == 0) else 1
+    env = os.environ.get("MOE_EXPERT_KERNEL", "")
+    two = cfg.routed == "bf16" and cfg.I % (128 * cg) == 0 and (
+        env == "two" or (env != "one" and cfg.T * cfg.k < 64 * cfg.E))
+    if two:
+        return f"tc_expert2_kernel<3, 1, {cg}>"
+    return f"tc_expert_kernel<3, 1, {cg}, {1 if cfg.routed == 'mxfp4' else 0}>"
+
+
 def gate_up_roofline(cfg, offsets, stage_ms: dict, peaks: dict) -> dict:
     """Roofline of the dominant kernel, the routed gate/up GEMM with the
     SiTU-GLU epilogue, from its CUDA-event time inside the timed region."""
@@ -180,15 +194,18 @@ def gate_up_roofline(cfg, offsets, stage_ms: dict, peaks: dict) -> dict:
         achieved = work["bytes"] / (dom_ms / 1e3) / 1e9
         peak, unit = peaks["hbm_gbs"], "GB/s"
         src = f"{peaks['source']} HBM copy (read+write bytes); a read-dominated stream can exceed it"
+    kname = gate_up_kernel(cfg)
     traffic = None
     prof = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}_expert_gate_up.json")
     if os.path.exists(prof):
         # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu
-        # capture of this workload (the file gives the command and kernel build)
+        # capture of this workload; only if it measured the kernel that ran here
         with open(prof) as f:
-            traffic = json.load(f).get("dram_bytes_per_launch")
-    kern = "tc_expert_kernel (2-CTA grouped gate/up + SiTU epilogue" + (
-        ", MXFP4 weights decoded to bf16 in shared memory)" if cfg.routed == "mxfp4" else ")")
+            rec = json.load(f)
+        if rec.get("kernel") == kname:
+            traffic = rec.get("dram_bytes_per_launch")
+    kern = kname + (" (2-CTA grouped gate/up, SiTU epilogue, MXFP4 weights decoded to bf16 in shared memory)"
+                    if cfg.routed == "mxfp4" else " (2-CTA grouped gate/up, SiTU epilogue)")
     return {"kernel": f"{kern} = stage expert_gate_up", "bound": bound, "achieved": round(achieved, 1),
             "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
             "kernel_ms": round(dom_ms, 4), "algorithmic": {"flops": work["flops"], "bytes": work["bytes"]},
@@ -459,6 +476,63 @@ def workload_line(cfg, layer, x, args, world, rank, local_rank, peaks, headline:
     return out
 
 
+# fp32 CUDA-core peak of B200 for the backward pass's contractions: 148 SMs x
+# 128 fp32 FMA lanes x 2 flops x the SM clock (1965 MHz maximum).
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_flops(cfg) -> float:
+    """Algorithmic flops of moe_layer_backward: the forward contractions it
+    recomputes (router, W_down, the selected experts' gate/up and down, the
+    shared experts' gate/up; not the output projection) plus two contractions
+    per forward one for the gradients of its two operands (all of them)."""
+    T, H, L, E, k, I, S, Is = cfg.T, cfg.H, cfg.L, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is
+    fwd_all = cfg.flops_per_token() * T
+    recompute = fwd_all - T * (2 * L * H + S * 2 * Is * H)  # no output projection
+    return recompute + 2 * fwd_all
+
+
+def measure_backward(cfg, layer, x, reps: int = 3) -> dict:
+    """moe_layer_backward (the layer's backward pass with the forward's
+    selection held fixed) on this workload, timed with CUDA events after one
+    warm-up call; reported against the fp32 CUDA-core peak."""
+    dev = x.device
+    stream = torch.cuda.current_stream(dev)
+    d = dims_for(cfg, "f32")
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    layer.forward(x, aux={"topk_idx": idx})
+    dy = torch.randn(cfg.T, cfg.H, generator=torch.Generator().manual_seed(1)).to(dev)
+    shapes = {"dx": (cfg.T, cfg.H), "dWr": (cfg.E, cfg.H), "dWdown": (cfg.L, cfg.H), "dWup": (cfg.H, cfg.L),
+              "dgamma": (cfg.L,), "dWg": (cfg.E, cfg.I, cfg.L), "dWv": (cfg.E, cfg.I, cfg.L),
+              "dWo": (cfg.E, cfg.L, cfg.I), "dWsg": (cfg.S, cfg.Is, cfg.H), "dWsv": (cfg.S, cfg.Is, cfg.H),
+              "dWso": (cfg.S, cfg.H, cfg.Is)}
+    grads = {n: torch.empty(s, dtype=torch.float32, device=dev) for n, s in shapes.items()}
+    g = moe.make_grads(**grads)
+    ws = torch.empty(moe.moe_backward_workspace_size(d), dtype=torch.uint8, device=dev)
+
+    def call():
+        moe.check(moe.moe_layer_backward(d, layer._w, x, dy, idx, g, ws, None, stream))
+
+    call()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    flops = backward_flops(cfg)
+    achieved = flops / (ms / 1e3) / 1e12
+    del grads, ws
+    return {"ms": round(ms, 3), "tokens_per_s": round(cfg.T / (ms / 1e3), 1), "flops": flops, "bound": "alu",
+            "achieved": round(achieved, 2), "peak": round(FP32_ALU_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / FP32_ALU_PEAK_TFLOPS, 4),
+            "peak_source": "derived: 148 SMs x 128 fp32 FMA/clock x 2 x 1965 MHz (contractions on CUDA cores)",
+            "workload": workload_name(cfg)}
+
+
 def build_layer(cfg, dev, y_out: str, weights=None):
     inputs = gen.device_layer(cfg, dev) if weights is None else weights
     x = inputs.pop("x") if "x" in inputs else None
@@ -509,6 +583,15 @@ def run_ours(args, rank, world, local_rank):
             torch.cuda.empty_cache()
             layer, x, weights = build_layer(sub, dev, args.y_out)
             out[name] = workload_line(sub, layer, x, args, world, rank, local_rank, peaks, headline=False)
+    if extra and not args.no_backward:
+        # the backward pass on the mid layer (at the K3 shape the fp32 gradients
+        # of all 896 experts' weights alone would take 118 GB)
+        del layer, weights, x
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        mid = gen.CONFIGS["mid"]
+        layer, x, weights = build_layer(mid, dev, "f32")
+        out["backward"] = measure_backward(mid, layer, x)
     return out if rank == 0 else None
 
 
@@ -590,6 +673,7 @@ def main():
     ap.add_argument("--no-oracle", "--no-cpu-baseline", dest="no_oracle", action="store_true",
                     help="skip the oracle sample (parity + CPU baseline)")
     ap.add_argument("--no-extra-lines", action="store_true", help="measure only --config (no decode / mxfp4 lines)")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -292,6 +292,46 @@ MOE_API moe_status moe_qb_bias_update(const moe_dims* d, const float* scores, co
                                       float* quantile_out, uint32_t* hist, int32_t nbins, float lo, float hi,
                                       moe_stream_t stream);
 
+/* Gradients of moe_layer_backward, fp32, in the shapes of the weights
+ * (moe_weights) and of x.  Every pointer must be non-NULL (dWsg / dWsv / dWso
+ * may be NULL when S = 0); all are overwritten. */
+typedef struct {
+  float* dx;      /* [T, H] */
+  float* dWr;     /* [E, H] */
+  float* dWdown;  /* [L, H] */
+  float* dWup;    /* [H, L] */
+  float* dgamma;  /* [L] */
+  float* dWg;     /* [E, I, L] */
+  float* dWv;     /* [E, I, L] */
+  float* dWo;     /* [E, L, I] */
+  float* dWsg;    /* [S, Is, H] */
+  float* dWsv;    /* [S, Is, H] */
+  float* dWso;    /* [S, H, Is] */
+} moe_grads;
+
+/* Backward pass of the layer with the expert selection held fixed: the
+ * vector-Jacobian product of y(x, weights) with dy = dLoss/dy.  The top-k
+ * choice is discrete and has no gradient; the mixture weights
+ * p_j = s_{e_j} / sum_j' s_{e_j'} are differentiable in the router scores
+ * s = Sigmoid(W_r x), so gradients reach the router through p only and the
+ * selection bias gets none (page "Kimi K3の896エキスパートを「896人の専門家」と
+ * 呼ぶと何がズレるか", sections "ルーターは計算の割当器" and "ルーター専用の
+ * 独立訓練はない": the router trains with the model, the bias is set by
+ * Quantile Balancing).  Experts no token selected get zero gradients.
+ *  - x [T, H] (act), dy [T, H] fp32, topk_idx [T, k] int32: the selection the
+ *    forward pass made (moe_aux.topk_idx of moe_layer_forward); rows must hold
+ *    k distinct experts in [0, E).
+ *  - The forward quantities are recomputed in fp32 from x and the weights,
+ *    without the forward pass's bf16 storage rounding, so the result is the
+ *    gradient of the layer function itself; accumulation is fp32 and the
+ *    order of every sum is fixed (deterministic).
+ *  - Supported: act = routed = MOE_F32 or MOE_BF16 (no MXFP4).
+ *  - Workspace: moe_backward_workspace_size(d) bytes, 256-byte aligned. */
+MOE_API size_t moe_backward_workspace_size(const moe_dims* d);
+MOE_API moe_status moe_layer_backward(const moe_dims* d, const moe_weights* w, const void* x, const float* dy,
+                                      const int32_t* topk_idx, const moe_grads* g, void* ws, size_t ws_bytes,
+                                      moe_stream_t stream);
+
 /* Human-readable name of a status. */
 MOE_API const char* moe_status_str(moe_status s);
 

@@ -36,6 +36,8 @@ EXPORTED = (
     "moe_output",
     "moe_expert_ffn_blocks_workspace_size",
     "moe_expert_ffn_blocks",
+    "moe_backward_workspace_size",
+    "moe_layer_backward",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -70,6 +72,13 @@ class moe_weights(ctypes.Structure):
 MOE_NUM_STAGES = 10
 STAGE_NAMES = ("router", "topk", "latent_down", "shared_gate_up", "permute", "gather", "expert_gate_up",
                "expert_down", "combine", "output")
+
+
+_GRAD_FIELDS = ("dx", "dWr", "dWdown", "dWup", "dgamma", "dWg", "dWv", "dWo", "dWsg", "dWsv", "dWso")
+
+
+class moe_grads(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in _GRAD_FIELDS]
 
 
 class moe_aux(ctypes.Structure):
@@ -113,8 +122,12 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_ffn_blocks_workspace_size.restype = ctypes.c_size_t
         L.moe_expert_ffn_blocks.argtypes = [pd, pw, vp, ctypes.c_int64, vp, ctypes.c_int32, vp, vp, ctypes.c_size_t,
                                             vp]
+        L.moe_backward_workspace_size.argtypes = [pd]
+        L.moe_backward_workspace_size.restype = ctypes.c_size_t
+        L.moe_layer_backward.argtypes = [pd, pw, vp, vp, vp, ctypes.POINTER(moe_grads), vp, ctypes.c_size_t, vp]
         for f in EXPORTED:
-            if f not in ("moe_workspace_size", "moe_status_str", "moe_expert_ffn_blocks_workspace_size"):
+            if f not in ("moe_workspace_size", "moe_status_str", "moe_expert_ffn_blocks_workspace_size",
+                         "moe_backward_workspace_size"):
                 getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -260,6 +273,26 @@ def moe_expert_ffn_blocks(d, weights: moe_weights, x_rows, n_rows: int, block_of
     return lib().moe_expert_ffn_blocks(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(x_rows), int(n_rows),
                                        _ptr(block_offsets), int(n_blocks), _ptr(y_rows), _ptr(ws), ws_bytes,
                                        _stream(stream))
+
+
+def make_grads(**tensors) -> moe_grads:
+    """moe_grads from keyword tensors named as the C struct fields."""
+    unknown = set(tensors) - set(_GRAD_FIELDS)
+    if unknown:
+        raise KeyError(f"unknown gradient fields {sorted(unknown)}")
+    return moe_grads(*[_ptr(tensors.get(f)) for f in _GRAD_FIELDS])
+
+
+def moe_backward_workspace_size(d) -> int:
+    return int(lib().moe_backward_workspace_size(ctypes.byref(_dims(d))))
+
+
+def moe_layer_backward(d, weights: moe_weights, x, dy, topk_idx, grads: moe_grads, ws, ws_bytes=None,
+                       stream=None) -> int:
+    """Backward pass with the forward's selection held fixed (see include/moe.h)."""
+    ws_bytes = _nbytes(ws) if ws_bytes is None else ws_bytes
+    return lib().moe_layer_backward(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(x), _ptr(dy), _ptr(topk_idx),
+                                    ctypes.byref(grads), _ptr(ws), ws_bytes, _stream(stream))
 
 
 def moe_status_str(status: int) -> str:

@@ -151,6 +151,31 @@ __device__ __forceinline__ void ex_tma_load(void* dst, const CUtensorMap* map, u
   }
 }
 
+// The same load with an L2 cache-eviction hint.
+template <int CG>
+__device__ __forceinline__ void ex_tma_load_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
+                                                 int32_t c1, uint64_t policy) {
+  if (CG == 2) {
+    const uint32_t mb = smem_u32(bar) & 0xFEFFFFFFu;
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(mb), "l"(policy)
+        : "memory");
+  } else {
+    tma_load_2d_hint(dst, map, bar, c0, c1, policy);
+  }
+}
+
+// L2 eviction hints on the expert kernels' loads: the weight rows of experts
+// with a single token tile are read once and are marked evict-first, so that
+// streaming them does not push out of L2 the token rows, which every weight
+// tile of their group re-reads and which are marked evict-last; the weight
+// rows of experts with several token tiles are re-read through L2 by each and
+// keep the default policy.  (Evict-first on every weight row raised the
+// gate/up kernel's DRAM reads from 60 to 65 GB at the K3 prefill shape.)
+constexpr bool kExL2Hints = true;
+
 template <int CG>
 __device__ __forceinline__ void ex_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -204,6 +229,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 struct ExTile {
   int expert, row0, ntok, n_mma, wt;
+  bool multi;  // the tile's expert has several token tiles (its weight tiles are re-read through L2)
 };
 
 // Work order: token tiles are taken in groups of EX_GROUP consecutive tiles;
@@ -211,23 +237,47 @@ struct ExTile {
 // then share a weight tile (its rows stream from HBM once per group, not once
 // per token tile, when a large expert has many token tiles) while the
 // group's token rows stay in L2 across the weight tiles.
-constexpr int EX_GROUP = 8;
+#ifndef MOE_EX_GROUP
+#define MOE_EX_GROUP 8
+#endif
+constexpr int EX_GROUP = MOE_EX_GROUP;
 
-__device__ __forceinline__ ExTile ex_decode(int w, int num_tiles, const ExParams& p) {
+// Item i of a list of token tiles [t0, t0 + n) in the grouped order above.
+__device__ __forceinline__ ExTile ex_decode_list(int i, int t0, int n, int num_multi, const ExParams& p) {
   const int gsize = EX_GROUP * p.n_wtiles;
-  const int grp = w / gsize;
-  const int r = w - grp * gsize;
-  const int in_grp = min(EX_GROUP, num_tiles - grp * EX_GROUP);
+  const int grp = i / gsize;
+  const int r = i - grp * gsize;
+  const int in_grp = min(EX_GROUP, n - grp * EX_GROUP);
   const int wt = r / in_grp;
-  const int tt = grp * EX_GROUP + (r - wt * in_grp);
+  const int tt = t0 + grp * EX_GROUP + (r - wt * in_grp);
   ExTile t;
   t.wt = wt;
+  t.multi = tt < num_multi;
   const int4 e = p.tile_table[tt];
   t.expert = e.x;
   t.row0 = e.y;
   t.ntok = e.z;
   t.n_mma = max(16, (t.ntok + 15) & ~15);
   return t;
+}
+
+// The tile table lists the tiles of experts with several tiles first
+// (num_multi of them: their weight tiles are shared through L2 by the
+// expert's token tiles) and then those of single-tile experts (weights
+// streamed from DRAM once).  kExInterleave = true would interleave the two
+// lists in proportion to their sizes so that items of both kinds run at the
+// same time; measured at the K3 prefill shape it raised the gate/up kernel's
+// DRAM reads from 58 to 68 GB and its time by 5%, so items run in list order.
+constexpr bool kExInterleave = false;
+
+__device__ __forceinline__ ExTile ex_decode(int w, int num_tiles, int num_multi, const ExParams& p) {
+  if (!kExInterleave || num_multi <= 0 || num_multi >= num_tiles) return ex_decode_list(w, 0, num_tiles, num_multi, p);
+  const long long total = static_cast<long long>(num_tiles) * p.n_wtiles;
+  const long long n_multi = static_cast<long long>(num_multi) * p.n_wtiles;
+  const int before = static_cast<int>(static_cast<long long>(w) * n_multi / total);  // multi items before w
+  const bool multi = static_cast<int>((static_cast<long long>(w) + 1) * n_multi / total) > before;
+  return multi ? ex_decode_list(before, 0, num_multi, num_multi, p)
+               : ex_decode_list(w - before, num_multi, num_tiles - num_multi, num_multi, p);
 }
 
 template <int EPI, bool PAIRED, int CG, bool MX>
@@ -292,7 +342,8 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int num_tiles = *p.num_tiles_dev;
+  const int num_tiles = p.num_tiles_dev[0];
+  const int num_multi = p.num_tiles_dev[1];
   const int total = num_tiles * p.n_wtiles;
 
   if (warp == 0) {
@@ -302,6 +353,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0u, issued_parity = 0u;
       bool ok = true;
+      const uint64_t pol_w = l2_policy_evict_first(), pol_t = l2_policy_evict_last();
       // No separate L2 prefetch of the weight rows: on B200 the extra bulk
       // requests cost more than the latency they hide (measured, prefill
       // gate/up about 15% slower with a 12-k-block-ahead prefetch).
@@ -310,7 +362,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
         return t.expert * p.w_rows_per_expert + wrow_pair + static_cast<int>(rank) * (PAIRED ? 64 : 128);
       };
       for (int w = pair; w < total && ok; w += npairs) {
-        const ExTile t = ex_decode(w, num_tiles, p);
+        const ExTile t = ex_decode(w, num_tiles, num_multi, p);
         const int rows_cta = CG == 2 ? t.n_mma / 2 : t.n_mma;   // token rows this CTA stages
         // Staged as ONE box of 128, 64, 32 or 16 rows, the smallest that covers
         // the tile: measured on B200, a single TMA request per operand and
@@ -345,13 +397,19 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
               tma_load_2d(q_dst, &maps.a0, &raw[stage], kb * 32, wrow);
               tma_load_2d(s_dst, &maps.s0, &raw[stage], sc0, wrow);
             }
+          } else if (kExL2Hints && !t.multi) {
+            ex_tma_load_hint<CG>(a_dst, &maps.a0, &full[stage], kc, wrow, pol_w);
+            if (PAIRED) ex_tma_load_hint<CG>(a_dst + EX_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
           } else if (PAIRED) {
             ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
             ex_tma_load<CG>(a_dst + EX_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
           } else {
             ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
           }
-          ex_tma_load<CG>(b_dst, &maps.b[bsel], &full[stage], kc, tok0);
+          if (kExL2Hints)
+            ex_tma_load_hint<CG>(b_dst, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
+          else
+            ex_tma_load<CG>(b_dst, &maps.b[bsel], &full[stage], kc, tok0);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == EX_STAGES) {
@@ -380,7 +438,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int w = pair; w < total && ok; w += npairs) {
-        const ExTile t = ex_decode(w, num_tiles, p);
+        const ExTile t = ex_decode(w, num_tiles, num_multi, p);
         const uint32_t idesc = idesc_bf16_f32(128 * CG, t.n_mma);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort, p.fault_site + 3)) break;
         tc_fence_after();
@@ -484,7 +542,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
     uint32_t acc_phase = 0;
     int xbuf = 0;
     for (int w = pair; w < total; w += npairs) {
-      const ExTile t = ex_decode(w, num_tiles, p);
+      const ExTile t = ex_decode(w, num_tiles, num_multi, p);
       bool got;
       if constexpr (PAIRED) {
         // One thread waits; the verdict reaches all four warps through the

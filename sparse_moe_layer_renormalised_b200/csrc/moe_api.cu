@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "backward.cuh"
 #include "combine.cuh"
 #include "gemm_expert.cuh"
 #include "gemm_expert2.cuh"
@@ -475,16 +476,25 @@ cudaError_t launch_expert2_inst(const X2Maps& maps, const X2Params& p, cudaStrea
   return cudaLaunchKernelEx(&cfg, kern, maps, p);
 }
 
-// The two-weight-tile expert kernel (gemm_expert2.cuh) runs bf16 weights when
-// the weight tiles divide evenly; MOE_EXPERT_ONE_TILE=1 in the environment
-// selects the one-tile kernel instead (both compute the same result; used to
-// compare them).
+// Which grouped expert kernel runs bf16 weights.  The two-weight-tile kernel
+// (gemm_expert2.cuh) halves the token rows moved per flop and issues MMAs from
+// two threads, but its accumulators are single-buffered; measured on B200 it
+// streams decode-shaped weights (a few rows per expert) 3.5% faster and is 6%
+// slower at the prefill shape (~290 rows per expert), where the one-tile
+// kernel's double-buffered accumulators hide the epilogue.  So it runs when
+// the average expert has fewer than kTwoTileMaxRows rows and its tiles divide
+// evenly.  MOE_EXPERT_KERNEL=one / =two in the environment forces either (both
+// compute the same result; used to compare them).
+constexpr long long kTwoTileMaxRows = 64;
+
 bool use_two_tile(const moe_dims& d, bool paired) {
   if (d.act != MOE_BF16 || d.routed != MOE_BF16) return false;
-  const char* env = std::getenv("MOE_EXPERT_ONE_TILE");
-  if (env != nullptr && env[0] == '1') return false;
   const int rows = 128 * expert_cg(d);
-  return paired ? d.I % rows == 0 : d.L % rows == 0;
+  if (paired ? d.I % rows != 0 : d.L % rows != 0) return false;
+  const char* env = std::getenv("MOE_EXPERT_KERNEL");
+  if (env != nullptr && std::strcmp(env, "one") == 0) return false;
+  if (env != nullptr && std::strcmp(env, "two") == 0) return true;
+  return d.T * d.k < kTwoTileMaxRows * d.E;
 }
 
 moe_status stage_expert2(const moe_dims& d, bool paired, const void* w0, const void* w1, const void* act, int K,
@@ -702,6 +712,254 @@ BlocksWsLayout blocks_ws_layout(const moe_dims& d, long long n_rows, int n_block
 
 bool ws_ok(const moe_dims& d, const void* ws, size_t ws_bytes) {
   return ws != nullptr && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0 && ws_bytes >= ws_layout(d).total;
+}
+
+// ------------------------------------------------------------------------------ backward pass
+struct BwLayout {
+  size_t s, p, tile_base, rank, offsets, perm_token, inv_perm, tile_table, num_tiles, z, z_perm, g, v, h, y_perm, u,
+      n, r, gs, vs, hs, dn, du, dp, dy_perm, dh, dz_perm, dz, dhs, dl, total;
+  int max_tiles;
+};
+
+BwLayout bw_layout(const moe_dims& d) {
+  BwLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, kAlign);
+    return o;
+  };
+  const size_t T = static_cast<size_t>(d.T), R = T * d.k, E = d.E, L = d.L, I = d.I, SI = static_cast<size_t>(d.S) * d.Is;
+  l.max_tiles = static_cast<int>(cdiv(static_cast<long long>(R), BW_TILE) + d.E);
+  l.s = take(T * E * 4);
+  l.p = take(R * 4);
+  l.tile_base = take(static_cast<size_t>(cdiv(d.T, PERM_TILE)) * E * 4);
+  l.rank = take(R * 4);
+  l.offsets = take((E + 1) * 4);
+  l.perm_token = take(R * 4);
+  l.inv_perm = take(R * 4);
+  l.tile_table = take(static_cast<size_t>(l.max_tiles) * 16);
+  l.num_tiles = take(16);
+  l.z = take(T * L * 4);
+  l.z_perm = take(R * L * 4);
+  l.g = take(R * I * 4);
+  l.v = take(R * I * 4);
+  l.h = take(R * I * 4);
+  l.y_perm = take(R * L * 4);
+  l.u = take(T * L * 4);
+  l.n = take(T * L * 4);
+  l.r = take(T * 4);
+  l.gs = take(T * SI * 4);
+  l.vs = take(T * SI * 4);
+  l.hs = take(T * SI * 4);
+  l.dn = take(T * L * 4);
+  l.du = take(T * L * 4);
+  l.dp = take(R * 4);
+  l.dy_perm = take(R * L * 4);
+  l.dh = take(R * I * 4);
+  l.dz_perm = take(R * L * 4);
+  l.dz = take(T * L * 4);
+  l.dhs = take(T * SI * 4);
+  l.dl = take(T * E * 4);
+  l.total = off;
+  return l;
+}
+
+// One strided GEMM launch (backward.cuh).  ta / tb: element types of A and B
+// (true = bf16, false = fp32).
+template <typename TA, typename TB>
+void bw_launch_t(int mode, const BwGemm& g, int e_count, int max_tiles, cudaStream_t s) {
+  const unsigned gx = static_cast<unsigned>(cdiv(g.N, BW_TILE));
+  if (mode == kBwDense)
+    bw_gemm_kernel<TA, TB, kBwDense><<<dim3(gx, static_cast<unsigned>(cdiv(g.M, BW_TILE))), BW_THREADS, 0, s>>>(g);
+  else if (mode == kBwRows)
+    bw_gemm_kernel<TA, TB, kBwRows><<<dim3(gx, static_cast<unsigned>(max_tiles)), BW_THREADS, 0, s>>>(g);
+  else
+    bw_gemm_kernel<TA, TB, kBwKRows>
+        <<<dim3(gx, static_cast<unsigned>(cdiv(g.M, BW_TILE)), static_cast<unsigned>(e_count)), BW_THREADS, 0, s>>>(g);
+}
+
+void bw_launch(bool a_bf16, bool b_bf16, int mode, const BwGemm& g, int e_count, int max_tiles, cudaStream_t s) {
+  ++g_last_launches;
+  if (a_bf16 && b_bf16)
+    bw_launch_t<__nv_bfloat16, __nv_bfloat16>(mode, g, e_count, max_tiles, s);
+  else if (a_bf16)
+    bw_launch_t<__nv_bfloat16, float>(mode, g, e_count, max_tiles, s);
+  else if (b_bf16)
+    bw_launch_t<float, __nv_bfloat16>(mode, g, e_count, max_tiles, s);
+  else
+    bw_launch_t<float, float>(mode, g, e_count, max_tiles, s);
+}
+
+// C[M, N] (+)= A(m, k) B(k, n) with explicit strides (a dense problem).
+BwGemm bw_dense(const void* a, long long a_m, long long a_k, const void* b, long long b_k, long long b_n, float* c,
+                long long ldc, int M, int N, int K, float beta) {
+  BwGemm g{};
+  g.a = a;
+  g.a_m = a_m;
+  g.a_k = a_k;
+  g.b = b;
+  g.b_k = b_k;
+  g.b_n = b_n;
+  g.c = c;
+  g.ldc = ldc;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.beta = beta;
+  return g;
+}
+
+moe_status run_backward(const moe_dims& d, const moe_weights& w, const void* x, const float* dy, const int32_t* idx,
+                        const moe_grads& gr, void* ws, cudaStream_t st) {
+  const BwLayout Lw = bw_layout(d);
+  const bool bf = d.act == MOE_BF16;
+  const int T = static_cast<int>(d.T), H = d.H, L = d.L, E = d.E, k = d.k, I = d.I, S = d.S, Is = d.Is;
+  const long long R = static_cast<long long>(T) * k;
+  const int SI = S * Is;
+  const size_t es = act_bytes(d);
+  float* s = at<float>(ws, Lw.s);
+  float* p = at<float>(ws, Lw.p);
+  int32_t* offsets = at<int32_t>(ws, Lw.offsets);
+  int32_t* perm_token = at<int32_t>(ws, Lw.perm_token);
+  int32_t* inv_perm = at<int32_t>(ws, Lw.inv_perm);
+  const int4* table = at<int4>(ws, Lw.tile_table);
+  const int32_t* ntiles = at<int32_t>(ws, Lw.num_tiles);
+  float *z = at<float>(ws, Lw.z), *z_perm = at<float>(ws, Lw.z_perm), *g = at<float>(ws, Lw.g),
+        *v = at<float>(ws, Lw.v), *h = at<float>(ws, Lw.h), *y_perm = at<float>(ws, Lw.y_perm),
+        *u = at<float>(ws, Lw.u), *n = at<float>(ws, Lw.n), *r = at<float>(ws, Lw.r), *gs = at<float>(ws, Lw.gs),
+        *vs = at<float>(ws, Lw.vs), *hs = at<float>(ws, Lw.hs), *dn = at<float>(ws, Lw.dn),
+        *du = at<float>(ws, Lw.du), *dp = at<float>(ws, Lw.dp), *dy_perm = at<float>(ws, Lw.dy_perm),
+        *dh = at<float>(ws, Lw.dh), *dz_perm = at<float>(ws, Lw.dz_perm), *dz = at<float>(ws, Lw.dz),
+        *dhs = at<float>(ws, Lw.dhs), *dl = at<float>(ws, Lw.dl);
+  const int mt = Lw.max_tiles;
+  auto ew = [](long long count) { return static_cast<unsigned>(cdiv(count, BW_EW_THREADS)); };
+
+  // ---- forward quantities, fp32
+  bw_launch(bf, bf, kBwDense, bw_dense(x, H, 1, w.Wr, 1, H, s, E, T, E, H, 0.f), 0, 0, st);  // logits
+  bw_sigmoid_kernel<<<ew(static_cast<long long>(T) * E), BW_EW_THREADS, 0, st>>>(s, static_cast<long long>(T) * E);
+  bw_mix_kernel<<<ew(T), BW_EW_THREADS, 0, st>>>(s, idx, T, E, k, p);
+  bw_launch(bf, bf, kBwDense, bw_dense(x, H, 1, w.Wdown, 1, H, z, L, T, L, H, 0.f), 0, 0, st);  // z
+  const long long ntok = cdiv(d.T, PERM_TILE);
+  perm_rank_kernel<<<static_cast<unsigned>(ntok), PERM_TILE, static_cast<size_t>(E) * 16, st>>>(
+      idx, d.T, E, k, at<int32_t>(ws, Lw.tile_base), at<int32_t>(ws, Lw.rank));
+  perm_scan_kernel<<<1, 1024, 0, st>>>(at<int32_t>(ws, Lw.tile_base), static_cast<int>(ntok), E, nullptr, offsets,
+                                       BW_TILE, at<int4>(ws, Lw.tile_table), at<int32_t>(ws, Lw.num_tiles));
+  perm_scatter_kernel<<<static_cast<unsigned>(cdiv(R, 256)), 256, 0, st>>>(
+      idx, d.T, E, k, at<int32_t>(ws, Lw.tile_base), at<int32_t>(ws, Lw.rank), offsets, perm_token, inv_perm);
+  g_last_launches += 5;
+  bw_gather_rows_f32_kernel<float><<<ew(R * L), BW_EW_THREADS, 0, st>>>(z, perm_token, R, L, z_perm);
+  // g / v / h / y_perm of the routed experts over the expert-major rows
+  BwGemm gg = bw_dense(z_perm, L, 1, w.Wg, 1, L, g, I, 0, I, L, 0.f);
+  gg.tile_table = table;
+  gg.num_tiles = ntiles;
+  gg.b_e = static_cast<long long>(I) * L;
+  bw_launch(false, bf, kBwRows, gg, 0, mt, st);
+  gg.b = w.Wv;
+  gg.c = v;
+  bw_launch(false, bf, kBwRows, gg, 0, mt, st);
+  bw_situ_kernel<<<ew(R * I), BW_EW_THREADS, 0, st>>>(g, v, R * I, d.situ_c, h);
+  BwGemm gy = bw_dense(h, I, 1, w.Wo, 1, I, y_perm, L, 0, L, I, 0.f);
+  gy.tile_table = table;
+  gy.num_tiles = ntiles;
+  gy.b_e = static_cast<long long>(L) * I;
+  bw_launch(false, bf, kBwRows, gy, 0, mt, st);
+  bw_combine_kernel<<<static_cast<unsigned>(T), BW_EW_THREADS, 0, st>>>(y_perm, inv_perm, p, w.gamma, k, L, d.rms_eps,
+                                                                       u, n, r);
+  for (int i = 0; i < S; ++i) {  // shared experts' pre-activations
+    const uint8_t* wsg = static_cast<const uint8_t*>(w.Wsg) + static_cast<size_t>(i) * Is * H * es;
+    const uint8_t* wsv = static_cast<const uint8_t*>(w.Wsv) + static_cast<size_t>(i) * Is * H * es;
+    bw_launch(bf, bf, kBwDense, bw_dense(x, H, 1, wsg, 1, H, gs + i * Is, SI, T, Is, H, 0.f), 0, 0, st);
+    bw_launch(bf, bf, kBwDense, bw_dense(x, H, 1, wsv, 1, H, vs + i * Is, SI, T, Is, H, 0.f), 0, 0, st);
+  }
+  if (S > 0) bw_situ_kernel<<<ew(static_cast<long long>(T) * SI), BW_EW_THREADS, 0, st>>>(gs, vs, static_cast<long long>(T) * SI, d.situ_c, hs);
+
+  // ---- gradients
+  bw_launch(false, bf, kBwDense, bw_dense(dy, H, 1, w.Wup, L, 1, dn, L, T, L, H, 0.f), 0, 0, st);       // dn
+  bw_launch(false, false, kBwDense, bw_dense(dy, 1, H, n, L, 1, gr.dWup, L, H, L, T, 0.f), 0, 0, st);   // dW_up
+  for (int i = 0; i < S; ++i) {
+    const uint8_t* wso = static_cast<const uint8_t*>(w.Wso) + static_cast<size_t>(i) * H * Is * es;
+    bw_launch(false, bf, kBwDense, bw_dense(dy, H, 1, wso, Is, 1, dhs + i * Is, SI, T, Is, H, 0.f), 0, 0, st);
+    bw_launch(false, false, kBwDense,
+              bw_dense(dy, 1, H, hs + i * Is, SI, 1, gr.dWso + static_cast<size_t>(i) * H * Is, Is, H, Is, T, 0.f), 0,
+              0, st);
+  }
+  if (S > 0) {
+    bw_situ_grad_kernel<<<ew(static_cast<long long>(T) * SI), BW_EW_THREADS, 0, st>>>(gs, vs, dhs,
+                                                                                      static_cast<long long>(T) * SI,
+                                                                                      d.situ_c);
+    for (int i = 0; i < S; ++i) {
+      bw_launch(false, bf, kBwDense,
+                bw_dense(gs + i * Is, 1, SI, x, H, 1, gr.dWsg + static_cast<size_t>(i) * Is * H, H, Is, H, T, 0.f), 0,
+                0, st);
+      bw_launch(false, bf, kBwDense,
+                bw_dense(vs + i * Is, 1, SI, x, H, 1, gr.dWsv + static_cast<size_t>(i) * Is * H, H, Is, H, T, 0.f), 0,
+                0, st);
+    }
+  }
+  bw_combine_grad_kernel<<<static_cast<unsigned>(T), BW_EW_THREADS, 0, st>>>(dn, u, r, w.gamma, y_perm, inv_perm, p,
+                                                                            k, L, du, dp, dy_perm);
+  bw_dgamma_kernel<<<static_cast<unsigned>(cdiv(L, 128)), 128, 0, st>>>(dn, u, r, d.T, L, gr.dgamma);
+  // routed experts
+  BwGemm gdh = bw_dense(dy_perm, L, 1, w.Wo, I, 1, dh, I, 0, I, L, 0.f);
+  gdh.tile_table = table;
+  gdh.num_tiles = ntiles;
+  gdh.b_e = static_cast<long long>(L) * I;
+  bw_launch(false, bf, kBwRows, gdh, 0, mt, st);  // dh = dy_perm W_o[e]
+  BwGemm gwo{};
+  gwo.a = dy_perm;
+  gwo.a_m = 1;
+  gwo.a_row = L;
+  gwo.b = h;
+  gwo.b_row = I;
+  gwo.b_n = 1;
+  gwo.c = gr.dWo;
+  gwo.ldc = I;
+  gwo.c_e = static_cast<long long>(L) * I;
+  gwo.M = L;
+  gwo.N = I;
+  gwo.offsets = offsets;
+  bw_launch(false, false, kBwKRows, gwo, E, 0, st);  // dW_o[e] = dy_e^T h_e
+  bw_situ_grad_kernel<<<ew(R * I), BW_EW_THREADS, 0, st>>>(g, v, dh, R * I, d.situ_c);  // g, v <- dg, dv
+  BwGemm gwg = gwo;
+  gwg.a = g;
+  gwg.a_row = I;
+  gwg.b = z_perm;
+  gwg.b_row = L;
+  gwg.c = gr.dWg;
+  gwg.ldc = L;
+  gwg.c_e = static_cast<long long>(I) * L;
+  gwg.M = I;
+  gwg.N = L;
+  bw_launch(false, false, kBwKRows, gwg, E, 0, st);  // dW_g[e] = dg_e^T z_e
+  gwg.a = v;
+  gwg.c = gr.dWv;
+  bw_launch(false, false, kBwKRows, gwg, E, 0, st);  // dW_v[e] = dv_e^T z_e
+  BwGemm gdz = bw_dense(g, I, 1, w.Wg, L, 1, dz_perm, L, 0, L, I, 0.f);
+  gdz.tile_table = table;
+  gdz.num_tiles = ntiles;
+  gdz.b_e = static_cast<long long>(I) * L;
+  bw_launch(false, bf, kBwRows, gdz, 0, mt, st);  // dz_perm = dg W_g[e]
+  gdz.a = v;
+  gdz.b = w.Wv;
+  gdz.beta = 1.f;
+  bw_launch(false, bf, kBwRows, gdz, 0, mt, st);  //        + dv W_v[e]
+  bw_gather_sum_kernel<<<ew(static_cast<long long>(T) * L), BW_EW_THREADS, 0, st>>>(dz_perm, inv_perm, d.T, k, L, dz);
+  bw_router_grad_kernel<<<static_cast<unsigned>(T), 128, 0, st>>>(s, idx, p, dp, d.T, E, k, dl);
+  g_last_launches += 11;
+  // latent projection and router weight gradients, then dx
+  bw_launch(false, bf, kBwDense, bw_dense(dz, 1, L, x, H, 1, gr.dWdown, H, L, H, T, 0.f), 0, 0, st);
+  bw_launch(false, bf, kBwDense, bw_dense(dl, 1, E, x, H, 1, gr.dWr, H, E, H, T, 0.f), 0, 0, st);
+  bw_launch(false, bf, kBwDense, bw_dense(dz, L, 1, w.Wdown, H, 1, gr.dx, H, T, H, L, 0.f), 0, 0, st);
+  bw_launch(false, bf, kBwDense, bw_dense(dl, E, 1, w.Wr, H, 1, gr.dx, H, T, H, E, 1.f), 0, 0, st);
+  for (int i = 0; i < S; ++i) {
+    const uint8_t* wsg = static_cast<const uint8_t*>(w.Wsg) + static_cast<size_t>(i) * Is * H * es;
+    const uint8_t* wsv = static_cast<const uint8_t*>(w.Wsv) + static_cast<size_t>(i) * Is * H * es;
+    bw_launch(false, bf, kBwDense, bw_dense(gs + i * Is, SI, 1, wsg, H, 1, gr.dx, H, T, H, Is, 1.f), 0, 0, st);
+    bw_launch(false, bf, kBwDense, bw_dense(vs + i * Is, SI, 1, wsv, H, 1, gr.dx, H, T, H, Is, 1.f), 0, 0, st);
+  }
+  (void)du;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -964,6 +1222,36 @@ moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const 
   st = stage_expert_gate_up(dr, *w, x_rows, table, n_tiles, at<void>(ws, L.h), s, L.max_tiles);
   if (st != MOE_OK) return st;
   return stage_expert_down(dr, *w, at<void>(ws, L.h), table, n_tiles, y_rows, s, L.max_tiles);
+}
+
+size_t moe_backward_workspace_size(const moe_dims* d) {
+  if (!dims_ok(d)) return 0;
+  return bw_layout(*d).total;
+}
+
+moe_status moe_layer_backward(const moe_dims* d, const moe_weights* w, const void* x, const float* dy,
+                              const int32_t* topk_idx, const moe_grads* g, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  moe_status st = check_dims(d);
+  if (st != MOE_OK) return st;
+  if (d->routed != d->act) return MOE_ERR_UNSUPPORTED;
+  if (w == nullptr || g == nullptr || x == nullptr || dy == nullptr || topk_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  const void* need[] = {w->Wr, w->Wdown, w->Wup, w->gamma, w->Wg, w->Wv, w->Wo, x, dy, topk_idx,
+                        g->dx, g->dWr, g->dWdown, g->dWup, g->dgamma, g->dWg, g->dWv, g->dWo};
+  for (const void* q : need)
+    if (q == nullptr || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (d->S > 0) {
+    const void* sh[] = {w->Wsg, w->Wsv, w->Wso, g->dWsg, g->dWsv, g->dWso};
+    for (const void* q : sh)
+      if (q == nullptr || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  }
+  const BwLayout L = bw_layout(*d);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || ws_bytes < L.total)
+    return MOE_ERR_INVALID_ARG;
+  if (d->T > 0x7fffffffLL / (d->H > d->E ? d->H : d->E)) return MOE_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (d->T == 0) return MOE_OK;
+  return run_backward(*d, *w, x, dy, topk_idx, *g, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_device_error(int* code, moe_stream_t stream) {

@@ -168,8 +168,10 @@ __device__ __forceinline__ void emit_tiles(int e, int off, int cnt, int first, i
 
 // One block of 1024 threads, thread = expert.  Turns the per-tile counts into
 // per-tile exclusive bases (in place), the expert counts, the CSR offsets, the
-// tile table and its length (tile_table / num_m_tiles may be NULL when the
-// caller runs no grouped GEMM on the result).
+// tile table, its length (num_m_tiles[0]) and the number of its leading tiles
+// that belong to experts with more than one tile (num_m_tiles[1]);
+// tile_table / num_m_tiles may be NULL when the caller runs no grouped GEMM
+// on the result.
 __global__ void __launch_bounds__(1024)
     perm_scan_kernel(int32_t* __restrict__ tile_counts, int ntiles, int E, int32_t* __restrict__ counts_out,
                      int32_t* __restrict__ offsets, int max_tile_rows, int4* __restrict__ tile_table,
@@ -187,17 +189,28 @@ __global__ void __launch_bounds__(1024)
   }
   const int cnt = e < E ? run : 0;
   const int mt = tiles_of(cnt, max_tile_rows);
+  // Tiles of experts with several tiles (their weight tiles are re-read from
+  // L2 by each) come first, then the tiles of single-tile experts (weights
+  // streamed once); each part in expert order.
+  const int mt_multi = mt >= 2 ? mt : 0, mt_single = mt == 1 ? 1 : 0;
   const int incl_off = block_incl_scan_1024(cnt, buf);
   __syncthreads();
-  const int incl_mt = block_incl_scan_1024(mt, buf);
+  const int incl_multi = block_incl_scan_1024(mt_multi, buf);
+  const int n_multi = buf[1023];
+  __syncthreads();
+  const int incl_single = block_incl_scan_1024(mt_single, buf);
   if (e < E) {
     offsets[e] = incl_off - cnt;
     if (counts_out != nullptr) counts_out[e] = cnt;
-    if (tile_table != nullptr) emit_tiles(e, incl_off - cnt, cnt, incl_mt - mt, max_tile_rows, tile_table);
+    const int first = mt >= 2 ? incl_multi - mt_multi : n_multi + incl_single - mt_single;
+    if (tile_table != nullptr) emit_tiles(e, incl_off - cnt, cnt, first, max_tile_rows, tile_table);
   }
   if (e == E - 1) {
     offsets[E] = incl_off;
-    if (num_m_tiles != nullptr) *num_m_tiles = incl_mt;
+    if (num_m_tiles != nullptr) {
+      num_m_tiles[0] = n_multi + incl_single;
+      num_m_tiles[1] = n_multi;
+    }
   }
 }
 
@@ -223,7 +236,10 @@ __global__ void __launch_bounds__(1024)
   const int mt = tiles_of(cnt, max_tile_rows);
   const int incl_mt = block_incl_scan_1024(mt, buf);
   if (e < E) emit_tiles(e, off, cnt, incl_mt - mt, max_tile_rows, tile_table);
-  if (e == E - 1) *num_m_tiles = incl_mt;
+  if (e == E - 1) {
+    num_m_tiles[0] = incl_mt;
+    num_m_tiles[1] = 0;  // one list, in expert order
+  }
 }
 
 // Tile table over n_blocks CSR blocks of the same E experts (rows received
@@ -259,7 +275,10 @@ __global__ void __launch_bounds__(1024)
       first += tiles_of(end - off, max_tile_rows);
     }
   }
-  if (e == E - 1) *num_m_tiles = incl_mt;
+  if (e == E - 1) {
+    num_m_tiles[0] = incl_mt;
+    num_m_tiles[1] = 0;  // one list, in expert order
+  }
 }
 
 // Thread = pair (t, j): position = offset of its expert + base of its tile +

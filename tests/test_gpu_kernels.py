@@ -125,12 +125,9 @@ def test_combine_rmsnorm(T, L, k, act):
 def test_expert_ffn_mid_dims(T, L, kernel, monkeypatch):
     # L = 1024 runs the expert GEMMs on CTA pairs; L = 1152 (not a multiple of
     # 256) on single CTAs, where the down projection's 9 weight tiles leave the
-    # last two-tile item with one tile.  bf16 weights run the two-weight-tile
-    # kernel unless MOE_EXPERT_ONE_TILE=1 selects the one-tile kernel.
-    if kernel == "one_tile":
-        monkeypatch.setenv("MOE_EXPERT_ONE_TILE", "1")
-    else:
-        monkeypatch.delenv("MOE_EXPERT_ONE_TILE", raising=False)
+    # last two-tile item with one tile.  MOE_EXPERT_KERNEL picks the bf16
+    # expert kernel (one weight tile or two per work item).
+    monkeypatch.setenv("MOE_EXPERT_KERNEL", "one" if kernel == "one_tile" else "two")
     cfg = gen.CONFIGS["mid"].with_(L=L)
     E, k, L, I = cfg.E, cfg.k, cfg.L, cfg.I
     d = dims_for(cfg, T=T)
