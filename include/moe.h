@@ -345,6 +345,15 @@ MOE_API moe_status moe_device_error(int* code, moe_stream_t stream);
  * enqueued (for launch accounting). */
 MOE_API int moe_last_launch_count(void);
 
+/* Diagnostics, no counterpart in the pages: checks that the kernels' bounded
+ * pipeline waits end.  Launches one thread that waits on an mbarrier nothing
+ * completes (no copy or MMA in flight); after limit_ms (1..2000) it gives up,
+ * records MOE_FAULT_SELFTEST_WAIT in the device fault flag (read and cleared
+ * by moe_device_error) and writes the time it waited, in ns, to *waited_ns
+ * (a device pointer).  The context stays usable. */
+#define MOE_FAULT_SELFTEST_WAIT 9
+MOE_API moe_status moe_selftest_wait_timeout(int32_t limit_ms, unsigned long long* waited_ns, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,6 +38,7 @@ EXPORTED = (
     "moe_expert_ffn_blocks",
     "moe_backward_workspace_size",
     "moe_layer_backward",
+    "moe_selftest_wait_timeout",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -122,6 +123,7 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_ffn_blocks_workspace_size.restype = ctypes.c_size_t
         L.moe_expert_ffn_blocks.argtypes = [pd, pw, vp, ctypes.c_int64, vp, ctypes.c_int32, vp, vp, ctypes.c_size_t,
                                             vp]
+        L.moe_selftest_wait_timeout.argtypes = [ctypes.c_int32, vp, vp]
         L.moe_backward_workspace_size.argtypes = [pd]
         L.moe_backward_workspace_size.restype = ctypes.c_size_t
         L.moe_layer_backward.argtypes = [pd, pw, vp, vp, vp, ctypes.POINTER(moe_grads), vp, ctypes.c_size_t, vp]
@@ -293,6 +295,14 @@ def moe_layer_backward(d, weights: moe_weights, x, dy, topk_idx, grads: moe_grad
     ws_bytes = _nbytes(ws) if ws_bytes is None else ws_bytes
     return lib().moe_layer_backward(ctypes.byref(_dims(d)), ctypes.byref(weights), _ptr(x), _ptr(dy), _ptr(topk_idx),
                                     ctypes.byref(grads), _ptr(ws), ws_bytes, _stream(stream))
+
+
+MOE_FAULT_SELFTEST_WAIT = 9
+
+
+def moe_selftest_wait_timeout(limit_ms: int, waited_ns, stream=None) -> int:
+    """Runs the bounded-wait self-test (see include/moe.h)."""
+    return lib().moe_selftest_wait_timeout(int(limit_ms), _ptr(waited_ns), _stream(stream))
 
 
 def moe_status_str(status: int) -> str:

@@ -1254,6 +1254,14 @@ moe_status moe_layer_backward(const moe_dims* d, const moe_weights* w, const voi
   return run_backward(*d, *w, x, dy, topk_idx, *g, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_selftest_wait_timeout(int32_t limit_ms, unsigned long long* waited_ns, moe_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000 || waited_ns == nullptr) return MOE_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ms) * 1000000ull, MOE_FAULT_SELFTEST_WAIT, waited_ns);
+  g_last_launches = 1;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_device_error(int* code, moe_stream_t stream) {
   if (code == nullptr) return MOE_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;

@@ -58,9 +58,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up (returns
-// false) after kWaitLimitNs, or as soon as another role of this CTA has
-// raised *abort; a timeout records `site` in the device fault flag.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+// false) after limit_ns, or as soon as another role of this CTA has raised
+// *abort; a timeout records `site` in the device fault flag.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int site,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -68,13 +69,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_fault(site);
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+// Self-test of the bounded wait: one thread waits on an mbarrier nothing
+// arrives on (no copy or MMA is in flight), gives up after limit_ns and
+// records `site`.  *waited_ns receives the time it waited.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, int site, unsigned long long* waited_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const uint64_t t0 = globaltimer_ns();
+  const bool ok = mbar_wait(&bar, 0u, &abort_flag, site, limit_ns);
+  *waited_ns = ok ? 0ull : static_cast<unsigned long long>(globaltimer_ns() - t0);
 }
 
 // ---------------------------------------------------------------------------- TMA

@@ -213,3 +213,20 @@ def test_expert_ffn_mxfp4(T):
         Wg, Wv, Wo = oin.expert_weights(cfg, e)
         ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wv, Wo, cfg.situ_c, oracle.bf16_round)
     assert parity(y_perm.cpu().to(F64), ref) <= 1e-2
+
+
+# ------------------------------------------------------------------------------ bounded waits
+def test_bounded_wait_gives_up_and_reports():
+    """A pipeline wait that nothing completes (no copy or MMA in flight) gives
+    up after its limit, records its site in the device fault flag, and leaves
+    the context usable."""
+    waited = torch.zeros(1, dtype=torch.int64, device="cuda")
+    assert moe.moe_selftest_wait_timeout(50, waited) == moe.MOE_OK
+    st, code = moe.moe_device_error()
+    assert st == moe.MOE_ERR_DEVICE and code == moe.MOE_FAULT_SELFTEST_WAIT
+    ns = int(waited.item())
+    assert 50_000_000 <= ns < 2_000_000_000, ns
+    _no_fault()  # the flag was cleared
+    assert moe.moe_selftest_wait_timeout(0, waited) == moe.MOE_ERR_INVALID_ARG
+    # the context still runs kernels
+    test_permute_exact(300, 32, 4, False)
