@@ -90,6 +90,25 @@ __device__ __forceinline__ TcTile tc_decode(int w, const TcParams& p) {
   return t;
 }
 
+// 32 consecutive bf16 (four 16-byte vectors) at dst, of which the first
+// `valid` are inside the row.
+__device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* dst, uint4 q0, uint4 q1, uint4 q2, uint4 q3,
+                                                 int valid) {
+  if (valid >= 32) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    d4[0] = q0;
+    d4[1] = q1;
+    d4[2] = q2;
+    d4[3] = q3;
+  } else {
+    const uint32_t w[16] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w,
+                            q2.x, q2.y, q2.z, q2.w, q3.x, q3.y, q3.z, q3.w};
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid) dst[i] = bf16_half(w[i >> 1], i & 1);
+  }
+}
+
 template <int EPI, bool PAIRED>
 __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
   extern __shared__ uint8_t tc_smem_raw[];
@@ -287,20 +306,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_gemm_kernel(const __grid_con
                 for (int i = 0; i < 32; ++i) a[i] = sigmoid_f32(a[i]);
               }
               if (EPI == kEpiBF16) {
-                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.ldo + col;
-                uint32_t pk[16];
+                uint4 q[4];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(a[2 * i], a[2 * i + 1]);
-                if (col + 32 <= p.N) {
-                  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-                  for (int i = 0; i < 4; ++i)
-                    d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                } else {
-#pragma unroll
-                  for (int i = 0; i < 32; ++i)
-                    if (col + i < p.N) dst[i] = bf16_half(pk[i >> 1], i & 1);
-                }
+                for (int i = 0; i < 4; ++i)
+                  q[i] = make_uint4(pack_bf16x2(a[8 * i], a[8 * i + 1]), pack_bf16x2(a[8 * i + 2], a[8 * i + 3]),
+                                    pack_bf16x2(a[8 * i + 4], a[8 * i + 5]), pack_bf16x2(a[8 * i + 6], a[8 * i + 7]));
+                store_bf16_chunk(reinterpret_cast<__nv_bfloat16*>(p.out) + grow * p.ldo + col, q[0], q[1], q[2], q[3],
+                                 min(32, p.N - col));
               } else {
                 float* dst = reinterpret_cast<float*>(p.out) + grow * p.ldo + col;
                 if (col + 32 <= p.N) {

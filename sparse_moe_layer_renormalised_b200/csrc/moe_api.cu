@@ -88,7 +88,7 @@ int expert_tile_rows(const moe_dims& d) { return d.act == MOE_BF16 ? 128 * exper
 // ------------------------------------------------------------------------------ workspace
 struct WsLayout {
   size_t scores, topk_idx, topk_w, rank, tile_base, counts, offsets, tile_table, num_m_tiles, perm_token,
-      inv_perm, z, z_perm, h_perm, y_perm, n, h_s, total;
+      inv_perm, z, z_perm, h_perm, y_perm, n, h_s, dense_tiles, dense_num, total;
 };
 
 WsLayout ws_layout(const moe_dims& d) {
@@ -119,6 +119,8 @@ WsLayout ws_layout(const moe_dims& d) {
   w.y_perm = take(R * d.L * 4);
   w.n = take(T * d.L * es);
   w.h_s = take(T * static_cast<size_t>(d.S) * d.Is * es);
+  w.dense_tiles = take(static_cast<size_t>(cdiv(static_cast<long long>(T), 128) + 1) * 16);
+  w.dense_num = take(16);
   w.total = off;
   return w;
 }
@@ -347,7 +349,11 @@ moe_status stage_dense(const moe_dims& d, int epi, const void* A, long long lda,
   return run_gemm(d, g, s);
 }
 
-moe_status stage_shared_gate_up(const moe_dims& d, const moe_weights& w, const void* x, void* h_s, cudaStream_t s) {
+moe_status stage_shared_gate_up(const moe_dims& d, const moe_weights& w, const void* x, void* h_s, cudaStream_t s,
+                                int4* dense_tiles = nullptr, int32_t* dense_num = nullptr);
+
+moe_status stage_shared_gate_up_simple(const moe_dims& d, const moe_weights& w, const void* x, void* h_s,
+                                       cudaStream_t s) {
   GemmDesc g{};
   g.epi = kEpiSituBF16;
   g.paired = true;
@@ -623,6 +629,42 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
   p.situ_c = d.situ_c;
   p.fault_site = 150;
   return launch_expert<kEpiF32, false>(cg, mx, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// The shared experts' gate/up projection with the SiTU-GLU epilogue.  With
+// bf16 weights it runs on the 2-CTA grouped expert kernel as one "expert"
+// whose S*Is weight rows are W_sg / W_sv (paired row by row) over token tiles
+// of 256 rows covering all T rows (its 2-CTA M = 256 tiles move less data per
+// MMA than the dense kernel's M = 128 tiles); MOE_SHARED_KERNEL=dense in the
+// environment, no workspace for the tile table, or dims that do not tile
+// evenly select the one-CTA dense kernel.
+moe_status stage_shared_gate_up(const moe_dims& d, const moe_weights& w, const void* x, void* h_s, cudaStream_t s,
+                                int4* dense_tiles, int32_t* dense_num) {
+  const int rows = d.S * d.Is;
+  const char* env = std::getenv("MOE_SHARED_KERNEL");
+  const bool pairs = d.act == MOE_BF16 && dense_tiles != nullptr && dense_num != nullptr && rows % 128 == 0 &&
+                     d.H % 64 == 0 && !(env != nullptr && std::strcmp(env, "dense") == 0);
+  if (!pairs) return stage_shared_gate_up_simple(d, w, x, h_s, s);
+  dense_tile_table_kernel<<<1, 256, 0, s>>>(d.T, 256, dense_tiles, dense_num);
+  ++g_last_launches;
+  ExMaps maps;
+  std::memset(&maps, 0, sizeof maps);
+  bool ok = make_token_maps(maps.b, x, static_cast<uint64_t>(d.T), d.H) &&
+            make_map(&maps.a0, w.Wsg, rows, d.H, d.H, 64) && make_map(&maps.a1, w.Wsv, rows, d.H, d.H, 64);
+  if (!ok) return MOE_ERR_CUDA;
+  ExParams p{};
+  p.tile_table = dense_tiles;
+  p.num_tiles_dev = dense_num;
+  p.n_wtiles = rows / 128;
+  p.w_rows_per_expert = rows;
+  p.num_k_blocks = d.H / EX_BK;
+  p.out = h_s;
+  p.ldo = rows;
+  p.out_cols = rows;
+  p.situ_c = d.situ_c;
+  p.fault_site = 130;
+  ++g_last_launches;
+  return launch_expert<kEpiSituBF16, true>(2, false, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 template <typename OutT>
@@ -1121,7 +1163,9 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
     return st;
   mark(MOE_STAGE_LATENT_DOWN, 1);
   mark(MOE_STAGE_SHARED_GATE_UP, 0);
-  if (d->S > 0 && (st = stage_shared_gate_up(*d, *w, x, h_s, s)) != MOE_OK) return st;
+  if (d->S > 0 && (st = stage_shared_gate_up(*d, *w, x, h_s, s, at<int4>(ws, L.dense_tiles),
+                                             at<int32_t>(ws, L.dense_num))) != MOE_OK)
+    return st;
   mark(MOE_STAGE_SHARED_GATE_UP, 1);
   // dispatch
   mark(MOE_STAGE_PERMUTE, 0);

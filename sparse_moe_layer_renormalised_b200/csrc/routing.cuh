@@ -281,6 +281,24 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// Tile table of a dense problem run on the grouped expert kernels: rows
+// 0 .. T-1 as consecutive tiles of tile_rows rows of "expert" 0.
+// num_m_tiles[0] = number of tiles; num_m_tiles[1] = the same (one expert with
+// several tiles: its weight tiles are re-read through L2).
+__global__ void dense_tile_table_kernel(long long T, int tile_rows, int4* __restrict__ tile_table,
+                                        int32_t* __restrict__ num_m_tiles) {
+  const long long ntiles = (T + tile_rows - 1) / tile_rows;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < ntiles;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r0 = i * tile_rows;
+    tile_table[i] = make_int4(0, static_cast<int>(r0), static_cast<int>(min(static_cast<long long>(tile_rows), T - r0)), 0);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    num_m_tiles[0] = static_cast<int32_t>(ntiles);
+    num_m_tiles[1] = static_cast<int32_t>(ntiles);
+  }
+}
+
 // Thread = pair (t, j): position = offset of its expert + base of its tile +
 // rank in the tile.  Token-ascending within each expert by construction.
 __global__ void __launch_bounds__(256)
@@ -319,7 +337,16 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32)
     return;
   }
   const uint4* s = src + static_cast<long long>(t) * row_vecs;
-  for (int i = lane; i < row_vecs; i += 32) d[i] = s[i];
+  // four 16-byte loads in flight per lane before their stores
+  int i = lane;
+  for (; i + 96 < row_vecs; i += 128) {
+    const uint4 a = s[i], b = s[i + 32], c = s[i + 64], e = s[i + 96];
+    d[i] = a;
+    d[i + 32] = b;
+    d[i + 64] = c;
+    d[i + 96] = e;
+  }
+  for (; i < row_vecs; i += 32) d[i] = s[i];
 }
 
 }  // namespace moe
