@@ -35,7 +35,8 @@ class oc_mat(ctypes.Structure):
 class oc_dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("L", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("S", ctypes.c_int32), ("Is", ctypes.c_int32),
-                ("situ_c", ctypes.c_double), ("rms_eps", ctypes.c_double), ("mode", ctypes.c_int32)]
+                ("situ_c", ctypes.c_double), ("rms_eps", ctypes.c_double), ("mode", ctypes.c_int32),
+                ("routed_act_mx8", ctypes.c_int32)]
 
 
 class oc_weights(ctypes.Structure):
@@ -76,7 +77,10 @@ def lib() -> ctypes.CDLL:
         L.oc_select_f32.argtypes = [vp, vp, i64, i64, i64, vp, vp]
         L.oc_permute.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
         L.oc_permute.restype = ctypes.c_int
-        L.oc_expert_forward.argtypes = [vp, i64, i64, pm, pm, pm, f64, i32, vp]
+        L.oc_expert_forward.argtypes = [vp, i64, i64, pm, pm, pm, f64, i32, i32, vp]
+        L.oc_e4m3_decode.argtypes = [vp, i64, vp]
+        L.oc_e4m3_encode.argtypes = [vp, i64, vp]
+        L.oc_mx8_quantize.argtypes = [vp, i64, i64, vp, vp]
         L.oc_combine.argtypes = [vp, vp, i64, i64, i64, vp]
         L.oc_rms_norm.argtypes = [vp, vp, i64, i64, f64, vp]
         L.oc_shared_experts.argtypes = [vp, i64, i64, i64, i64, pm, pm, pm, f64, i32, vp]
@@ -253,18 +257,63 @@ def _linear(a: torch.Tensor, W) -> torch.Tensor:
     return out
 
 
-def expert_forward(z_rows: torch.Tensor, Wg, Wv, Wo, c: float, rnd):
-    """g = W_g z, v = W_v z, h = rnd(SiTU-GLU(g, v)), y = W_o h (fp64)."""
+def expert_forward(z_rows: torch.Tensor, Wg, Wv, Wo, c: float, rnd, act_mx8: bool = False):
+    """g = W_g z, v = W_v z, h = rnd(SiTU-GLU(g, v)), y = W_o h (fp64); with
+    act_mx8 the rows of z and of h (after rnd) are first replaced by their
+    MXFP8 values."""
     mode = _mode_of(rnd)
     if mode is None:  # a caller-supplied rounding function: the same steps, one call each
-        return _linear(rnd(situ_glu(_linear(z_rows, Wg), _linear(z_rows, Wv), c)), Wo)
+        zq = mx8_round(z_rows) if act_mx8 else z_rows
+        h = rnd(situ_glu(_linear(zq, Wg), _linear(zq, Wv), c))
+        return _linear(mx8_round(h) if act_mx8 else h, Wo)
     z = _f64(z_rows)
     keep: list = []
     mg, mv, mo = _mat(Wg, keep), _mat(Wv, keep), _mat(Wo, keep)
     y = torch.empty(z.shape[0], mo.rows, dtype=F64)
     lib().oc_expert_forward(_ptr(z), z.shape[0], z.shape[1], ctypes.byref(mg), ctypes.byref(mv), ctypes.byref(mo),
-                            float(c), mode, _ptr(y))
+                            float(c), mode, 1 if act_mx8 else 0, _ptr(y))
     return y
+
+
+def e4m3_decode(codes) -> torch.Tensor:
+    """E4M3 codes (uint8) -> fp64 values (NaN for 0x7F / 0xFF)."""
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = torch.empty(c.shape, dtype=F64)
+    lib().oc_e4m3_decode(c.ctypes.data, c.size, _ptr(out))
+    return out
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """fp64 values -> nearest E4M3 codes (ties to even, saturating to +-448)."""
+    v = _f64(v)
+    out = np.empty(tuple(v.shape), dtype=np.uint8)
+    lib().oc_e4m3_encode(_ptr(v), v.numel(), out.ctypes.data)
+    return out
+
+
+def mx8_quantize(v) -> tuple[np.ndarray, np.ndarray]:
+    """Rows of fp64 values [R, K] -> MXFP8 (codes [R, K] uint8, E8M0 scale
+    bytes [R, K/32] uint8)."""
+    v = _f64(v)
+    R, K = v.shape
+    codes = np.empty((R, K), dtype=np.uint8)
+    scales = np.empty((R, K // 32), dtype=np.uint8)
+    lib().oc_mx8_quantize(_ptr(v), R, K, codes.ctypes.data, scales.ctypes.data)
+    return codes, scales
+
+
+def mx8_round(v) -> torch.Tensor:
+    """The values of the MXFP8 encoding of rows v [R, K] (fp64)."""
+    codes, scales = mx8_quantize(v)
+    return mx8_dequant(codes, scales)
+
+
+def mx8_dequant(codes, scales) -> torch.Tensor:
+    """MXFP8 codes [R, K] and E8M0 scale bytes [R, K/32] -> fp64 values."""
+    v = e4m3_decode(codes)
+    s = torch.from_numpy(np.ascontiguousarray(np.asarray(scales, dtype=np.int64))).repeat_interleave(32, dim=1)
+    f = torch.pow(torch.tensor(2.0, dtype=F64), (s - 127).to(F64))
+    return v * torch.where(s == 255, torch.tensor(float("nan"), dtype=F64), f)
 
 
 def combine(y_slots: torch.Tensor, p: torch.Tensor) -> torch.Tensor:
@@ -306,7 +355,8 @@ def _run_layer(cfg, dense: dict, x: torch.Tensor, routed, forced_idx) -> dict:
     T = x.shape[0]
     keep: list = []
     mode = {"bf16": ROUND_BF16, "f32": ROUND_F32}[cfg.act]
-    d = oc_dims(T, cfg.H, cfg.L, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is, float(cfg.situ_c), float(cfg.rms_eps), mode)
+    d = oc_dims(T, cfg.H, cfg.L, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is, float(cfg.situ_c), float(cfg.rms_eps), mode,
+                1 if getattr(cfg, "routed", None) == "mxfp4_a8" else 0)
     bias, gamma = _f64(dense["bias"]), _f64(dense["gamma"])
     keep += [bias, gamma]
     shared = [_mat(dense[n], keep) if cfg.S > 0 else _empty_mat() for n in ("Wsg", "Wsv", "Wso")]

@@ -21,6 +21,9 @@
 //  [K3-QAT] ai-tech-express.jp article on K3, section "量子化を前提とした学習
 //     「MXFP4 Quantization-Aware Training」": routed weights served in MXFP4
 //     (format fixed by the OCP Microscaling Formats specification v1.0).
+//     The pages give no activation format; where the routed experts take
+//     MXFP8 inputs (the block-scaled variant) the library's reading is the
+//     same specification's MXFP8 E4M3 with its shared-scale rule (below).
 //
 // Readings where the pages are silent (the same in the GPU library):
 //  * SiTU-GLU(g, v) = sigmoid(g) * c*tanh(g/c) * c*tanh(v/c), c = 10;
@@ -119,6 +122,71 @@ double e2m1_value(unsigned code) {
 double e8m0_value(uint8_t s) {
   if (s == 0xFF) return std::numeric_limits<double>::quiet_NaN();
   return std::ldexp(1.0, static_cast<int>(s) - 127);
+}
+
+// OCP FP8 E4M3 (OCP MX v1.0, FP8 E4M3): sign bit 7, exponent bits 6-3 (bias
+// 7), mantissa bits 2-0; exponent field 0 is subnormal (m/8 * 2^-6); no
+// infinities; S.1111.111 is NaN; largest finite 1.75 * 2^8 = 448.
+double e4m3_value(uint8_t code) {
+  const unsigned e = (code >> 3) & 15u, m = code & 7u;
+  if (e == 15u && m == 7u) return std::numeric_limits<double>::quiet_NaN();
+  const double mag = e == 0 ? std::ldexp(static_cast<double>(m), -9) : std::ldexp(8.0 + m, static_cast<int>(e) - 10);
+  return (code & 0x80u) ? -mag : mag;
+}
+
+// Nearest E4M3 code to v, ties to the even code, magnitudes past 448
+// saturated to 448 (the spec leaves overflow to the implementation; the
+// library saturates).  The sign of v (of -0 too) is kept.
+uint8_t e4m3_encode(double v) {
+  const uint8_t sign = std::signbit(v) ? 0x80u : 0u;
+  double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  if (a >= 448.0) return sign | 0x7Eu;
+  // spacing of E4M3 numbers around a: 2^(floor(log2 a) - 3), at least 2^-9
+  int e2 = 0;
+  std::frexp(a, &e2);  // a in [2^(e2-1), 2^e2)
+  const int q = std::max(e2 - 1, -6);
+  const double units = std::rint(std::ldexp(a, 3 - q));  // a / spacing, to nearest even integer
+  // units in [8, 16] for q >= -6 normal numbers (16 carries into the next
+  // exponent), in [0, 8] in the subnormal range
+  if (q == -6 && units < 8.0) return sign | static_cast<uint8_t>(units);
+  int exp_field = q + 7, mant = static_cast<int>(units) - 8;
+  if (mant == 8) {
+    ++exp_field;
+    mant = 0;
+  }
+  if (exp_field > 15 || (exp_field == 15 && mant > 6)) return sign | 0x7Eu;
+  return sign | static_cast<uint8_t>((exp_field << 3) | mant);
+}
+
+// OCP MX v1.0 shared scale of a block: s = floor(log2(max |v|)) - 8 (8 = the
+// largest E4M3 exponent), clamped to the E8M0 range [-127, 127]; an all-zero
+// block takes the lowest, -127.
+int mx8_block_exponent(const double* v, int64_t n) {
+  double amax = 0.0;
+  for (int64_t i = 0; i < n; ++i) amax = std::max(amax, std::fabs(v[i]));
+  if (amax == 0.0) return -127;
+  int e2 = 0;
+  std::frexp(amax, &e2);  // floor(log2 amax) = e2 - 1
+  return std::max(-127, std::min(127, e2 - 1 - 8));
+}
+
+// One row of K values (K a multiple of 32) -> E4M3 codes [K] and E8M0 scale
+// bytes [K/32]: block b's codes are e4m3_encode(v / 2^s_b), its scale byte
+// s_b + 127.
+void mx8_quantize_row(const double* v, int64_t K, uint8_t* codes, uint8_t* scales) {
+  for (int64_t b = 0; b < K / 32; ++b) {
+    const int s = mx8_block_exponent(v + 32 * b, 32);
+    scales[b] = static_cast<uint8_t>(s + 127);
+    for (int64_t i = 0; i < 32; ++i) codes[32 * b + i] = e4m3_encode(std::ldexp(v[32 * b + i], -s));
+  }
+}
+
+// The values the MXFP8 encoding of a row stands for (quantise, then decode).
+void mx8_round_row(const double* v, int64_t K, double* out) {
+  std::vector<uint8_t> c(static_cast<size_t>(K)), sc(static_cast<size_t>(K / 32));
+  mx8_quantize_row(v, K, c.data(), sc.data());
+  for (int64_t k = 0; k < K; ++k) out[k] = e4m3_value(c[k]) * e8m0_value(sc[k / 32]);
 }
 
 double sigmoid(double t) { return 1.0 / (1.0 + std::exp(-t)); }
@@ -233,13 +301,26 @@ void linear(const double* a, int64_t R, int64_t K, const oc_mat& W, double* out)
 
 // y[n, L] = W_o SiTU-GLU(W_g z, W_v z), h stored with `mode` ([K3-896]
 // "K3のエキスパートは896個の小型LLMではない"; SiTU-GLU from [K3-report]).
+// act_mx8: the expert's two GEMM inputs (the rows of z, and h after its
+// storage rounding) are first replaced row by row by their MXFP8 values.
 void expert(const double* z, int64_t n, int64_t L, const oc_mat& Wg, const oc_mat& Wv, const oc_mat& Wo, double c,
-            int mode, double* y) {
+            int mode, int act_mx8, double* y) {
   const int64_t I = Wg.rows;
+  std::vector<double> zq;
+  if (act_mx8) {
+    zq.resize(static_cast<size_t>(n * L));
+    for (int64_t r = 0; r < n; ++r) mx8_round_row(z + r * L, L, &zq[r * L]);
+    z = zq.data();
+  }
   std::vector<double> g(static_cast<size_t>(n * I)), v(static_cast<size_t>(n * I));
   linear(z, n, L, Wg, g.data());
   linear(z, n, L, Wv, v.data());
   for (int64_t i = 0; i < n * I; ++i) g[i] = store(situ_glu(g[i], v[i], c), mode);
+  if (act_mx8)
+    for (int64_t r = 0; r < n; ++r) {
+      std::vector<double> row(g.begin() + r * I, g.begin() + (r + 1) * I);
+      mx8_round_row(row.data(), I, &g[r * I]);
+    }
   linear(g.data(), n, I, Wo, y);
 }
 
@@ -351,8 +432,23 @@ int oc_permute(const int64_t* idx, int64_t T, int64_t k, int64_t E, int64_t* cou
 }
 
 void oc_expert_forward(const double* z, int64_t n, int64_t L, const oc_mat* Wg, const oc_mat* Wv, const oc_mat* Wo,
-                       double c, int mode, double* y) {
-  expert(z, n, L, *Wg, *Wv, *Wo, c, mode, y);
+                       double c, int mode, int act_mx8, double* y) {
+  expert(z, n, L, *Wg, *Wv, *Wo, c, mode, act_mx8, y);
+}
+
+// E4M3 codes -> values; values -> nearest E4M3 codes (ties to even,
+// saturating); rows of values -> MXFP8 codes [rows, K] and E8M0 scale bytes
+// [rows, K/32] (OCP MX v1.0; K a multiple of 32).
+void oc_e4m3_decode(const uint8_t* codes, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
+}
+
+void oc_e4m3_encode(const double* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_encode(v[i]);
+}
+
+void oc_mx8_quantize(const double* v, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales) {
+  for (int64_t r = 0; r < rows; ++r) mx8_quantize_row(v + r * K, K, codes + r * K, scales + r * (K / 32));
 }
 
 // u[t] = sum_j p[t, j] y_slots[t, j]   (j ascending)
@@ -382,7 +478,7 @@ void oc_shared_experts(const double* x, int64_t T, int64_t H, int64_t S, int64_t
   std::vector<double> yi(static_cast<size_t>(T * H));
   for (int64_t i = 0; i < T * H; ++i) y[i] = 0.0;
   for (int64_t s = 0; s < S; ++s) {
-    expert(x, T, H, row_view(*Wsg, s * Is, Is), row_view(*Wsv, s * Is, Is), row_view(*Wso, s * H, H), c, mode,
+    expert(x, T, H, row_view(*Wsg, s * Is, Is), row_view(*Wsv, s * Is, Is), row_view(*Wso, s * H, H), c, mode, 0,
            yi.data());
     for (int64_t i = 0; i < T * H; ++i) y[i] += yi[i];
   }
@@ -396,6 +492,7 @@ typedef struct {
   int32_t H, L, E, k, I, S, Is;
   double situ_c, rms_eps;
   int32_t mode;  // storage rounding of z, h, shared h, n
+  int32_t routed_act_mx8;  // 1: the routed experts take MXFP8 inputs (block-scaled variant)
 } oc_dims;
 
 typedef struct {
@@ -474,7 +571,7 @@ int oc_layer_forward(const oc_dims* d, const oc_weights* w, const double* x, con
     zr.assign(static_cast<size_t>(n * L), 0.0);
     yr.assign(static_cast<size_t>(n * L), 0.0);
     for (int64_t r = 0; r < n; ++r) std::memcpy(&zr[r * L], o->z + (pe[r] / k) * L, sizeof(double) * L);
-    expert(zr.data(), n, L, Wg, Wv, Wo, d->situ_c, d->mode, yr.data());
+    expert(zr.data(), n, L, Wg, Wv, Wo, d->situ_c, d->mode, d->routed_act_mx8, yr.data());
     for (int64_t r = 0; r < n; ++r) std::memcpy(&y_slots[pe[r] * L], &yr[r * L], sizeof(double) * L);
   }
   oc_combine(y_slots.data(), o->p, T, k, L, o->u);

@@ -18,7 +18,10 @@ Sources (web pages; cited by title and section):
    "幅のスケーリング：Stable LatentMoE": SiTU-GLU keeps SwiGLU's local
    non-linearity and puts smooth caps on both the linear and the up branch.
 [K3-QAT] ai-tech-express.jp article, section "量子化を前提とした学習「MXFP4
-   Quantization-Aware Training」": routed weights are served in MXFP4.
+   Quantization-Aware Training」": routed weights are served in MXFP4.  The
+   pages name no activation format; for the block-scaled variant, whose routed
+   experts take MXFP8 inputs, the reading is OCP MX v1.0's MXFP8 (E4M3) with
+   that specification's shared-scale rule.
 
 Readings where the pages are silent (each is also listed in the design notes):
   * SiTU-GLU is taken as  h = sigmoid(g) * c*tanh(g/c) * c*tanh(v/c),  c = 10:
@@ -49,6 +52,11 @@ __all__ = [
     "f32_to_f64",
     "E2M1_VALUES",
     "mxfp4_dequant",
+    "e4m3_decode",
+    "e4m3_encode",
+    "mx8_quantize",
+    "mx8_dequant",
+    "mx8_round",
     "sigmoid",
     "router_scores",
     "select_experts",
@@ -129,6 +137,79 @@ def mxfp4_dequant(codes, scales) -> torch.Tensor:
     factor = torch.pow(torch.tensor(2.0, dtype=F64), (s - 127).to(F64))
     factor = torch.where(s == 255, torch.tensor(float("nan"), dtype=F64), factor)
     return val * factor
+
+
+def e4m3_decode(codes) -> torch.Tensor:
+    """OCP FP8 E4M3 codes -> fp64: sign bit 7, exponent bits 6-3 with bias 7,
+    mantissa bits 2-0; exponent field 0 is subnormal (m/8 * 2^-6); no
+    infinities; S.1111.111 is NaN."""
+    c = torch.from_numpy(np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))).to(torch.int64)
+    e = (c >> 3) & 15
+    m = (c & 7).to(F64)
+    two = torch.tensor(2.0, dtype=F64)
+    normal = (1.0 + m / 8.0) * torch.pow(two, (e - 7).to(F64))
+    sub = (m / 8.0) * torch.pow(two, torch.tensor(-6.0, dtype=F64))
+    mag = torch.where(e == 0, sub, normal)
+    mag = torch.where((e == 15) & ((c & 7) == 7), torch.tensor(float("nan"), dtype=F64), mag)
+    return torch.where((c & 0x80) != 0, -mag, mag)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """Nearest E4M3 code to each fp64 value, ties to the even code, magnitudes
+    beyond 448 (the largest finite E4M3) saturated to 448; -0 keeps its sign.
+
+    Between 2^q and 2^(q+1) the E4M3 numbers are spaced 2^(q-3) (2^-9 below
+    2^-6, the subnormal range), so rounding is  round_half_even(a / spacing)
+    spacing units."""
+    v = torch.as_tensor(v).to(F64)
+    neg = torch.signbit(v)
+    a = torch.clamp(v.abs(), max=448.0)
+    _, ex = torch.frexp(a)                  # a in [2^(ex-1), 2^ex)
+    q = torch.clamp(ex.to(torch.int64) - 1, min=-6)
+    q = torch.where(a == 0, torch.full_like(q, -6), q)   # zero: the subnormal range
+    units = torch.round(torch.ldexp(a, (3 - q).to(torch.int64)))   # half to even
+    # units: 0..8 in the subnormal range (8 = the smallest normal, 2^-6); 8..16 else
+    carry = units >= 16
+    q = torch.where(carry, q + 1, q)
+    units = torch.where(carry, units / 2, units)
+    sub = (q == -6) & (units < 8)
+    exp_field = torch.where(sub, torch.zeros_like(q), q + 7)
+    mant = torch.where(sub, units, units - 8).to(torch.int64)
+    code = (exp_field << 3) | mant
+    code = torch.where(neg, code | 0x80, code)
+    return code.to(torch.uint8).numpy()
+
+
+def mx8_quantize(v) -> tuple[np.ndarray, np.ndarray]:
+    """Rows of fp64 values [R, K] (K a multiple of 32) -> OCP MXFP8: per block
+    of 32 along K the shared scale 2^s, s = floor(log2(max |v|)) - 8 (8 = the
+    largest E4M3 exponent) clamped to the E8M0 range [-127, 127] (an all-zero
+    block takes -127), and the E4M3 codes of v / 2^s.  Returns (codes [R, K],
+    scale bytes s + 127 [R, K/32]), both uint8."""
+    v = torch.as_tensor(v).to(F64)
+    R, K = v.shape
+    blocks = v.reshape(R, K // 32, 32)
+    amax = blocks.abs().amax(dim=2)
+    _, ex = torch.frexp(amax)
+    s = torch.clamp(ex.to(torch.int64) - 1 - 8, min=-127, max=127)
+    s = torch.where(amax == 0, torch.full_like(s, -127), s)
+    scaled = torch.ldexp(blocks, (-s)[:, :, None].expand(R, K // 32, 32))
+    codes = e4m3_encode(scaled.reshape(R, K))
+    return codes, (s + 127).to(torch.uint8).numpy()
+
+
+def mx8_dequant(codes, scales) -> torch.Tensor:
+    """MXFP8 codes [R, K] and scale bytes [R, K/32] -> fp64 values."""
+    val = e4m3_decode(codes)
+    s = torch.from_numpy(np.ascontiguousarray(np.asarray(scales, dtype=np.int64))).repeat_interleave(32, dim=1)
+    factor = torch.pow(torch.tensor(2.0, dtype=F64), (s - 127).to(F64))
+    factor = torch.where(s == 255, torch.tensor(float("nan"), dtype=F64), factor)
+    return val * factor
+
+
+def mx8_round(v) -> torch.Tensor:
+    """The values the MXFP8 encoding of rows v stands for."""
+    return mx8_dequant(*mx8_quantize(v))
 
 
 # ----------------------------------------------------------------------------------------------
@@ -219,12 +300,19 @@ def situ_glu(g: torch.Tensor, v: torch.Tensor, c: float) -> torch.Tensor:
     return sigmoid(g) * (c * torch.tanh(g / c)) * (c * torch.tanh(v / c))
 
 
-def expert_forward(z_rows: torch.Tensor, Wg: torch.Tensor, Wv: torch.Tensor, Wo: torch.Tensor, c: float, rnd):
+def expert_forward(z_rows: torch.Tensor, Wg: torch.Tensor, Wv: torch.Tensor, Wo: torch.Tensor, c: float, rnd,
+                   act_mx8: bool = False):
     """One GLU expert on latent rows: g = W_g z, v = W_v z, h = SiTU-GLU(g, v)
-    (stored, so rounded by rnd), y = W_o h (fp64, not rounded)."""
+    (stored, so rounded by rnd), y = W_o h (fp64, not rounded).  act_mx8 (the
+    block-scaled variant): the rows of z, and of h after rnd, are replaced by
+    their MXFP8 values before they enter the products."""
+    if act_mx8:
+        z_rows = mx8_round(z_rows)
     g = z_rows @ Wg.T
     v = z_rows @ Wv.T
     h = rnd(situ_glu(g, v, c))
+    if act_mx8:
+        h = mx8_round(h)
     return h @ Wo.T
 
 
@@ -289,7 +377,8 @@ def layer_forward(cfg, w: dict, x: torch.Tensor, forced_idx=None) -> dict:
     y_slots = torch.zeros(T, k, cfg.L, dtype=F64)
     for e in torch.unique(idx).tolist():
         t, j = torch.nonzero(idx == e, as_tuple=True)
-        y_slots[t, j] = expert_forward(z[t], w["Wg"][e], w["Wv"][e], w["Wo"][e], cfg.situ_c, rnd)
+        y_slots[t, j] = expert_forward(z[t], w["Wg"][e], w["Wv"][e], w["Wo"][e], cfg.situ_c, rnd,
+                                       act_mx8=getattr(cfg, "routed", None) == "mxfp4_a8")
     out = _finish(x, z, idx, p, y_slots, w, cfg, rnd)
     out.update({"s": s, "idx": idx, "p": p, "margin": margin})
     return out
@@ -313,7 +402,7 @@ def layer_forward_streamed(cfg, dense: dict, x: torch.Tensor, expert_weights, fo
     for e in torch.unique(idx).tolist():
         t, j = torch.nonzero(idx == e, as_tuple=True)
         Wg, Wv, Wo = expert_weights(e)
-        y_slots[t, j] = expert_forward(z[t], Wg, Wv, Wo, cfg.situ_c, rnd)
+        y_slots[t, j] = expert_forward(z[t], Wg, Wv, Wo, cfg.situ_c, rnd, act_mx8=getattr(cfg, "routed", None) == "mxfp4_a8")
     out = _finish(x, z, idx, p, y_slots, dense, cfg, rnd)
     out.update({"s": s, "idx": idx, "p": p, "margin": margin})
     return out

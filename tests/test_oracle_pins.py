@@ -75,6 +75,103 @@ def test_mxfp4_dequant_of_generator_output_is_bf16_exact(O):
 
 
 # ---------------------------------------------------------------- router
+def test_e4m3_decode_matches_torch_float8(O):
+    """All 256 E4M3 codes decode as PyTorch's float8_e4m3fn (a library
+    implementation of the same OCP format), NaN codes included."""
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(F64)
+    got = O.e4m3_decode(codes)
+    assert torch.equal(torch.isnan(got), torch.isnan(want))
+    assert torch.equal(torch.nan_to_num(got, nan=0.0), torch.nan_to_num(want, nan=0.0))
+    assert got[0x7E].item() == 448.0 and got[0x01].item() == 2.0**-9 and got[0x08].item() == 2.0**-6
+
+
+def test_e4m3_encode_matches_torch_cast_and_tie_rules(O):
+    """Nearest-even encoding: PyTorch's fp32 -> float8_e4m3fn cast on values in
+    range (fp32-exact, so one rounding), exact midpoints, saturation and the
+    sign of zero."""
+    g = torch.Generator().manual_seed(11)
+    v = torch.randn(50_000, generator=g, dtype=torch.float64) * torch.exp2(
+        torch.randint(-14, 9, (50_000,), generator=g).to(F64))
+    v = v.to(torch.float32).clamp(-448, 448).to(F64)
+    # midpoints between neighbouring E4M3 values (normal and subnormal ranges)
+    vals = O.e4m3_decode(np.arange(0, 0x7E, dtype=np.uint8))
+    mids = (vals[:-1] + vals[1:]) / 2
+    v = torch.cat([v, mids, -mids])
+    want = v.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(v), want)
+    sat = O.e4m3_encode(torch.tensor([448.0, 463.9, 464.0, 1e6, -500.0, 0.0, -0.0], dtype=F64))
+    assert list(sat) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x00, 0x80]
+
+
+def test_mx8_scale_rule_closed_forms(O):
+    """OCP MX v1.0 shared scale s = floor(log2 max|v|) - 8, clamped to the
+    E8M0 range; codes of v / 2^s."""
+    def q(block):
+        c, s = O.mx8_quantize(torch.tensor([block], dtype=F64))
+        return c[0], int(s[0, 0])
+
+    c, s = q([1.0] * 32)                      # s = -8: 1 -> 256 = 2^8, code 0x78
+    assert s == 119 and set(c) == {0x78}
+    c, s = q([1.9375] + [0.0] * 31)           # 1.9375 * 2^8 = 496 saturates to 448
+    assert s == 119 and c[0] == 0x7E and set(c[1:]) == {0}
+    c, s = q([0.0] * 32)                      # all-zero block: the lowest scale
+    assert s == 0 and set(c) == {0}
+    c, s = q([2.0**-130] + [0.0] * 31)        # clamped at -127: 2^-130 * 2^127 = 2^-3
+    assert s == 0 and c[0] == (4 << 3)
+    c, s = q([2.0**127] * 32)                 # s = 119 (byte 246): 2^127 / 2^119 = 2^8
+    assert s == 246 and set(c) == {0x78}
+    c, s = q([-3.0, 0.75] + [0.0] * 30)       # max 3 -> s = -7: -3 * 128 = -384, 0.75 * 128 = 96
+    assert s == 120 and c[0] == 0x80 | (15 << 3) | 4 and c[1] == (13 << 3) | 4
+    v = torch.tensor([[2.0**-20] * 16 + [5.0] * 16], dtype=F64)  # tiny elements flush within the block
+    assert O.mx8_round(v)[0, 0].item() == 0.0
+
+
+def test_mx8_round_is_idempotent_and_within_half_a_step(O):
+    """Quantising MXFP8 values again changes nothing, and each element moves by
+    at most half an E4M3 step: 2^-4 of itself in the normal range, 2^-10 of
+    the block scale below it; only elements above 448 units clip."""
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn(64, 256, generator=g, dtype=F64) * torch.exp2(torch.randint(-20, 20, (64, 8), generator=g)
+                                                                   .to(F64)).repeat_interleave(32, dim=1)
+    x = x.to(torch.bfloat16).to(F64)
+    r = O.mx8_round(x)
+    assert torch.equal(O.mx8_round(r), r)
+    _, s = O.mx8_quantize(x)
+    scale = torch.exp2(torch.from_numpy(s.astype(np.int64) - 127).to(F64)).repeat_interleave(32, dim=1)
+    units = (x / scale).abs()
+    bound = torch.where(units >= 2.0**-6, x.abs() * 2.0**-4, scale * 2.0**-10)
+    clipped = units > 448
+    assert bool(((r - x).abs() <= bound + 1e-300)[~clipped].all())
+    assert bool((r.abs()[clipped] == 448 * scale[clipped]).all())
+
+
+def test_cpp_and_torch_mx8_agree_bit_for_bit():
+    x = torch.randn(200, 1024, generator=torch.Generator().manual_seed(13), dtype=F64).to(torch.bfloat16).to(F64)
+    x = x * torch.exp2(torch.randint(-40, 40, (200, 1), generator=torch.Generator().manual_seed(14)).to(F64))
+    a = oracle.mx8_quantize(x)
+    b = oracle.torch_ref.mx8_quantize(x)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_expert_forward_mx8_rounds_both_inputs(O):
+    """act_mx8: the expert sees the MXFP8 values of its z rows and of h.  With
+    z already MXFP8-exact the gate/up inputs are unchanged, so the result is
+    W_o applied to mx8_round(h); with an identity-like W_o that is h's MXFP8
+    rounding itself, which differs from the unquantised expert."""
+    g = torch.Generator().manual_seed(15)
+    L, I, n = 64, 64, 5
+    z = O.mx8_round(torch.randn(n, L, generator=g, dtype=F64))
+    Wg = torch.randn(I, L, generator=g, dtype=F64) / 8
+    Wv = torch.randn(I, L, generator=g, dtype=F64) / 8
+    Wo = torch.eye(L, I, dtype=F64)
+    y8 = O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round, act_mx8=True)
+    h = O.bf16_round(O.situ_glu(z @ Wg.T, z @ Wv.T, 10.0))
+    assert torch.equal(y8, O.mx8_round(h))
+    y = O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round)
+    assert torch.equal(y, h) and not torch.equal(y, y8)
+
+
 def test_sigmoid_matches_scipy(O):
     x = torch.linspace(-30, 30, 2001, dtype=F64)
     assert torch.allclose(O.sigmoid(x), torch.from_numpy(scipy.special.expit(x.numpy())), rtol=1e-15, atol=0)
