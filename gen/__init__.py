@@ -251,7 +251,7 @@ def device_layer(cfg: LayerConfig, device="cuda", with_x: bool = True) -> dict:
         out[name] = t
     for name in ("Wg", "Wv", "Wo"):
         E, R, K = tensor_shape(cfg, name)
-        if cfg.routed == "mxfp4":
+        if tensor_dtype(cfg, name) == "mxfp4":
             codes = torch.empty((E, R, K // 2), dtype=torch.uint8, device=dev)
             scales = torch.empty((E, R, K // 32), dtype=torch.uint8, device=dev)
             stream = torch.cuda.current_stream(dev).cuda_stream
@@ -262,7 +262,7 @@ def device_layer(cfg: LayerConfig, device="cuda", with_x: bool = True) -> dict:
             out[name] = codes
             out[{"Wg": "Sg", "Wv": "Sv", "Wo": "So"}[name]] = scales
         else:
-            t = torch.empty((E, R, K), dtype=tdt[cfg.routed], device=dev)
+            t = torch.empty((E, R, K), dtype=tdt[tensor_dtype(cfg, name)], device=dev)
             _dev_fill(t, cfg, name)
             out[name] = t
     out["bias"] = torch.from_numpy(bias(cfg)).to(dev)

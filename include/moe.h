@@ -48,6 +48,18 @@
  *    「MXFP4 Quantization-Aware Training」"), everything else bf16; the kernels
  *    decode each weight exactly to bf16 in shared memory and multiply in bf16
  *    with fp32 accumulation.  Additionally L and I must be multiples of 512.
+ *  - MOE_BF16 / MOE_MXFP4_A8  the same MXFP4 routed weights, and the routed
+ *    experts' input activations (the expert-major z rows and h) quantised to
+ *    OCP MXFP8: per row, blocks of 32 consecutive elements along K, each with
+ *    an E8M0 scale 2^s, s = floor(log2(max |v|)) - 8 clamped to [-127, 127]
+ *    (-127 for an all-zero block), and E4M3 codes round-to-nearest-even(v / 2^s)
+ *    saturated to +-448 (the pages name no activation format; this is the OCP
+ *    MX v1.0 rule, the library's reading).  Both expert GEMMs then run on the
+ *    block-scaled tensor-core MMA (tcgen05.mma kind::mxf8f6f4), which applies
+ *    the scales of both operands; accumulation is fp32.  The weight scales are
+ *    read in the tiled order of moe_mx_tile_scales (moe_weights.Sgv_tiled,
+ *    So_tiled); Wg, Wv and Wo must be 32-byte aligned.  Same dims rules as
+ *    MOE_MXFP4.
  * Stored activations (z, expert h, shared h, n) are held in the activation type;
  * y_perm, u and the router scores are fp32.
  */
@@ -78,7 +90,7 @@ typedef enum {
   MOE_ERR_DEVICE = 4       /* moe_device_error only: a kernel recorded a device-side fault */
 } moe_status;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP4 = 2 } moe_dtype;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP4 = 2, MOE_MXFP4_A8 = 3 } moe_dtype;
 
 /* Layer shape and numerics.  K3 values: H=7168, L=3584, E=896, k=16, I=3072,
  * S=2, Is=3072 (dimension table of the page cited above). */
@@ -117,6 +129,11 @@ typedef struct {
   const void* Wsg;     /* [S, Is, H] shared gate projections */
   const void* Wsv;     /* [S, Is, H] shared up projections */
   const void* Wso;     /* [S, H, Is] shared down projections */
+  /* MOE_MXFP4_A8 only (NULL otherwise): the E8M0 scales of W_g / W_v and of
+   * W_o in the tiled order written by moe_mx_tile_scales (Sg, Sv, So are not
+   * read on that path and may be NULL). */
+  const uint8_t* Sgv_tiled;
+  const uint8_t* So_tiled;
 } moe_weights;
 
 /* Stages of moe_layer_forward, in launch order (for moe_aux.stage_events). */
@@ -182,7 +199,9 @@ MOE_API moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, const
  * r in expert_offsets[e] .. expert_offsets[e+1]-1:
  *   h = SiTU-GLU(z_perm[r] . Wg[e]^T, z_perm[r] . Wv[e]^T)   (stored in act type)
  *   y_perm[r] = h . Wo[e]^T                                    (fp32 [T*k, L])
- * Only w->Wg, w->Wv, w->Wo (and for MXFP4 w->Sg, w->Sv, w->So) are read.
+ * Only w->Wg, w->Wv, w->Wo (and for MXFP4 w->Sg, w->Sv, w->So; for
+ * MOE_MXFP4_A8 w->Sgv_tiled, w->So_tiled, with z_perm and h quantised to
+ * MXFP8 first) are read.
  * Workspace: moe_workspace_size(d) bytes. */
 MOE_API moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z_perm,
                           const int32_t* expert_offsets, float* y_perm, void* ws, size_t ws_bytes,
@@ -331,6 +350,33 @@ MOE_API size_t moe_backward_workspace_size(const moe_dims* d);
 MOE_API moe_status moe_layer_backward(const moe_dims* d, const moe_weights* w, const void* x, const float* dy,
                                       const int32_t* topk_idx, const moe_grads* g, void* ws, size_t ws_bytes,
                                       moe_stream_t stream);
+
+/* The activation quantiser of the block-scaled path (routed = MOE_MXFP4_A8),
+ * on its own: rows of x [rows, K] bf16 -> OCP MXFP8 codes [rows, K] (E4M3,
+ * uint8) and E8M0 scale bytes [rows, K/32] (row-major), by the rule stated at
+ * MOE_MXFP4_A8 above.  K a multiple of 32; x and codes 16-byte aligned;
+ * device pointers owned by the caller.  rows = 0 is a no-op. */
+MOE_API moe_status moe_mx8_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
+                                    moe_stream_t stream);
+
+/* Weight scales for the block-scaled routed experts (routed = MOE_MXFP4_A8).
+ * The block-scaled MMA takes its scales from tensor memory, loaded from
+ * shared memory in 512-byte atoms of 128 rows x 4 blocks of 32 along K (byte
+ * 16*(m%32) + 4*(m/32) + j = row m, block j); moe_mx_tile_scales re-orders the
+ * row-major E8M0 scales once, at load time, into the atoms each 2-CTA weight
+ * tile reads:
+ *   Sgv_tiled [E][I/128][2][L/128][512]: CTA c of weight tile t holds rows
+ *             t*128 + c*64 .. +63 of Sg (atom rows 0-63) and of Sv (64-127);
+ *   So_tiled  [E][L/256][2][I/128][512]: CTA c of tile t holds rows
+ *             t*256 + c*128 .. +127 of So.
+ * moe_mx_tiled_scales_size gives both sizes (each equals the row-major
+ * scales' size: E*I*L/16 and E*L*I/32 bytes).  Requires L and I multiples of
+ * 512 (MOE_ERR_UNSUPPORTED otherwise); Sg, Sv, So [E, I, L/32], [E, I, L/32],
+ * [E, L, I/32] as in moe_weights; all pointers device, 16-byte aligned, owned
+ * by the caller.  Enqueued on `stream`; no allocation. */
+MOE_API moe_status moe_mx_tiled_scales_size(const moe_dims* d, size_t* gate_up_bytes, size_t* down_bytes);
+MOE_API moe_status moe_mx_tile_scales(const moe_dims* d, const uint8_t* Sg, const uint8_t* Sv, const uint8_t* So,
+                                      uint8_t* Sgv_tiled, uint8_t* So_tiled, moe_stream_t stream);
 
 /* Human-readable name of a status. */
 MOE_API const char* moe_status_str(moe_status s);

@@ -17,8 +17,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE = 0, 1, 2, 3, 4
-MOE_F32, MOE_BF16, MOE_MXFP4 = 0, 1, 2
-_DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "mxfp4": MOE_MXFP4}
+MOE_F32, MOE_BF16, MOE_MXFP4, MOE_MXFP4_A8 = 0, 1, 2, 3
+_DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "mxfp4": MOE_MXFP4, "mxfp4_a8": MOE_MXFP4_A8}
 
 EXPORTED = (
     "moe_workspace_size",
@@ -39,6 +39,9 @@ EXPORTED = (
     "moe_backward_workspace_size",
     "moe_layer_backward",
     "moe_selftest_wait_timeout",
+    "moe_mx_tiled_scales_size",
+    "moe_mx_tile_scales",
+    "moe_mx8_quantize",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -62,7 +65,8 @@ class moe_dims(ctypes.Structure):
     ]
 
 
-_WEIGHT_FIELDS = ("Wr", "bias", "Wdown", "Wup", "gamma", "Wg", "Wv", "Wo", "Sg", "Sv", "So", "Wsg", "Wsv", "Wso")
+_WEIGHT_FIELDS = ("Wr", "bias", "Wdown", "Wup", "gamma", "Wg", "Wv", "Wo", "Sg", "Sv", "So", "Wsg", "Wsv", "Wso",
+                  "Sgv_tiled", "So_tiled")
 _AUX_FIELDS = ("scores", "topk_idx", "topk_w", "expert_offsets", "u", "n", "z")
 
 
@@ -127,6 +131,9 @@ def lib() -> ctypes.CDLL:
         L.moe_backward_workspace_size.argtypes = [pd]
         L.moe_backward_workspace_size.restype = ctypes.c_size_t
         L.moe_layer_backward.argtypes = [pd, pw, vp, vp, vp, ctypes.POINTER(moe_grads), vp, ctypes.c_size_t, vp]
+        L.moe_mx_tiled_scales_size.argtypes = [pd, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_mx_tile_scales.argtypes = [pd, vp, vp, vp, vp, vp, vp]
+        L.moe_mx8_quantize.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
         for f in EXPORTED:
             if f not in ("moe_workspace_size", "moe_status_str", "moe_expert_ffn_blocks_workspace_size",
                          "moe_backward_workspace_size"):
@@ -180,12 +187,21 @@ def _dims(d) -> moe_dims:
     return d.c() if isinstance(d, Dims) else d
 
 
+def _keep_alive(struct, tensors: dict):
+    """The struct holds device addresses only; it also keeps a reference to
+    the tensors behind them, so that a tensor made for the call (e.g.
+    make_weights(**tile_weight_scales(...))) is not freed, and its memory
+    reused, while the struct is in use."""
+    struct._tensors = dict(tensors)
+    return struct
+
+
 def make_weights(**tensors) -> moe_weights:
     """moe_weights from keyword tensors named as the C struct fields."""
     unknown = set(tensors) - set(_WEIGHT_FIELDS)
     if unknown:
         raise KeyError(f"unknown weight fields {sorted(unknown)}")
-    return moe_weights(*[_ptr(tensors.get(f)) for f in _WEIGHT_FIELDS])
+    return _keep_alive(moe_weights(*[_ptr(tensors.get(f)) for f in _WEIGHT_FIELDS]), tensors)
 
 
 def make_aux(stage_events=None, **tensors) -> moe_aux:
@@ -195,7 +211,7 @@ def make_aux(stage_events=None, **tensors) -> moe_aux:
     unknown = set(tensors) - set(_AUX_FIELDS)
     if unknown:
         raise KeyError(f"unknown aux fields {sorted(unknown)}")
-    a = moe_aux(*[_ptr(tensors.get(f)) for f in _AUX_FIELDS])
+    a = _keep_alive(moe_aux(*[_ptr(tensors.get(f)) for f in _AUX_FIELDS]), tensors)
     if stage_events is not None:
         if len(stage_events) != 2 * MOE_NUM_STAGES:
             raise ValueError("need 2 * MOE_NUM_STAGES events")
@@ -282,7 +298,7 @@ def make_grads(**tensors) -> moe_grads:
     unknown = set(tensors) - set(_GRAD_FIELDS)
     if unknown:
         raise KeyError(f"unknown gradient fields {sorted(unknown)}")
-    return moe_grads(*[_ptr(tensors.get(f)) for f in _GRAD_FIELDS])
+    return _keep_alive(moe_grads(*[_ptr(tensors.get(f)) for f in _GRAD_FIELDS]), tensors)
 
 
 def moe_backward_workspace_size(d) -> int:
@@ -298,6 +314,22 @@ def moe_layer_backward(d, weights: moe_weights, x, dy, topk_idx, grads: moe_grad
 
 
 MOE_FAULT_SELFTEST_WAIT = 9
+
+
+def moe_mx_tiled_scales_size(d) -> tuple[int, int, int]:
+    """(status, gate/up bytes, down bytes) of the tiled weight scales."""
+    gu, dn = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = lib().moe_mx_tiled_scales_size(ctypes.byref(_dims(d)), ctypes.byref(gu), ctypes.byref(dn))
+    return st, gu.value, dn.value
+
+
+def moe_mx_tile_scales(d, Sg, Sv, So, Sgv_tiled, So_tiled, stream=None) -> int:
+    return lib().moe_mx_tile_scales(ctypes.byref(_dims(d)), _ptr(Sg), _ptr(Sv), _ptr(So), _ptr(Sgv_tiled),
+                                    _ptr(So_tiled), _stream(stream))
+
+
+def moe_mx8_quantize(x, rows: int, K: int, codes, scales, stream=None) -> int:
+    return lib().moe_mx8_quantize(_ptr(x), int(rows), int(K), _ptr(codes), _ptr(scales), _stream(stream))
 
 
 def moe_selftest_wait_timeout(limit_ms: int, waited_ns, stream=None) -> int:

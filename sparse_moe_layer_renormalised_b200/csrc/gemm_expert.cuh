@@ -229,6 +229,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 struct ExTile {
   int expert, row0, ntok, n_mma, wt;
+  int tt;      // index of the token tile in the tile table
   bool multi;  // the tile's expert has several token tiles (its weight tiles are re-read through L2)
 };
 
@@ -252,6 +253,7 @@ __device__ __forceinline__ ExTile ex_decode_list(int i, int t0, int n, int num_m
   const int tt = t0 + grp * EX_GROUP + (r - wt * in_grp);
   ExTile t;
   t.wt = wt;
+  t.tt = tt;
   t.multi = tt < num_multi;
   const int4 e = p.tile_table[tt];
   t.expert = e.x;

@@ -1,0 +1,385 @@
+// Block-scaled grouped routed-expert GEMM for sm_100a: MXFP4 weights times
+// MXFP8 activations on tcgen05.mma kind::mxf8f6f4 (the tensor cores apply
+// both operands' E8M0 block scales; no decode pass).
+//
+//   D[w, t] = sum_k (Wq[w, k] * 2^(sw[w, k/32] - 127)) * (Xq[t, k] * 2^(sx[t, k/32] - 127))
+//
+// Same work decomposition, operand swap and warp roles as gemm_expert.cuh
+// (weight rows are the MMA's M on a 2-CTA pair, M = 256; token rows its N;
+// warp 0 TMA producer, warp 1 TMEM owner and MMA issuer on the even CTA,
+// warps 2-5 epilogue), with these differences:
+//  * a stage covers K = 128: four MMAs of K = 32;
+//  * the weight tile is loaded from the packed E2M1 codes with the TMA type
+//    that spreads 16 codes over 16 bytes of shared memory (8 bytes of codes,
+//    8 bytes of gap), the operand layout this MMA kind reads for 4-bit types;
+//    its completion count is the packed size (64 bytes per row);
+//  * the activation tile is E4M3 codes, one byte each;
+//  * per stage both CTAs also load their weight rows' scale atom (512 bytes)
+//    and the whole token tile's scale atoms (two, 1 KB: each CTA's half of the
+//    accumulator needs the scales of every token column); the MMA thread
+//    copies them to tensor memory with tcgen05.cp (cta_group::2: each CTA
+//    from its own shared memory) ahead of the stage's MMAs.  tcgen05.cp and
+//    tcgen05.mma from one thread execute in issue order, so one scale region
+//    serves every stage;
+//  * token tiles hold at most 240 rows, so two accumulators (2 x 240 fp32
+//    columns) and the scale columns (12) fit the 512 columns of tensor memory.
+// Every wait is bounded.
+#pragma once
+
+#include "gemm_expert.cuh"
+#include "mx8.cuh"
+
+namespace moe {
+
+constexpr int BS_BK = 128;                         // K elements per stage: 4 MMAs of K = 32
+constexpr uint32_t BS_A_BYTES = 128 * BS_BK;       // 128 weight rows, one byte slot per E2M1 code
+constexpr uint32_t BS_A_TX = 128 * BS_BK / 2;      // bytes the A tile's TMA completes (packed codes)
+constexpr uint32_t BS_B_BYTES = 128 * BS_BK;       // up to 128 token rows of E4M3 codes per CTA
+constexpr uint32_t BS_SFA_BYTES = 512;             // scale atom: 128 weight rows x 4 k-blocks
+constexpr uint32_t BS_SFB_BYTES = 1024;            // token rows 0-127 and 128-255
+constexpr int BS_STAGES = 6;
+constexpr int BS_MAX_TILE_ROWS = 240;              // largest token tile (MMA N)
+constexpr uint32_t BS_ACC_COLS = BS_MAX_TILE_ROWS;
+constexpr uint32_t BS_SF_COL = 2 * BS_ACC_COLS;    // SFA in columns 480-483, SFB in 484-491
+constexpr int BS_THREADS = 192;
+constexpr uint32_t BS_STAGE_BYTES = BS_A_BYTES + BS_B_BYTES + BS_SFA_BYTES + BS_SFB_BYTES;
+constexpr size_t BS_SMEM = 1024 + static_cast<size_t>(BS_STAGES) * BS_STAGE_BYTES + EX_XCH_BYTES + 512;
+static_assert(BS_SF_COL + 12 <= 2 * EX_ACC_COLS, "tensor memory columns");
+static_assert(BS_SMEM <= 232448, "shared memory per CTA");
+
+struct BsMaps {
+  CUtensorMap a0;    // E2M1 codes, 16 per 16-byte slot: PAIRED W_g [E*I, L] (64-row boxes), else W_o [E*L, I] (128-row)
+  CUtensorMap a1;    // PAIRED: W_v, as a0
+  CUtensorMap sa;    // weight scale tiles as [n, 16] bytes, 32-row (512-byte) boxes
+  CUtensorMap b[4];  // E4M3 activation codes [R, K]: 128-byte wide boxes of 128, 64, 32, 16 rows, 128-byte swizzle
+  CUtensorMap sb[2]; // activation scale tiles as [n, 16] bytes: 64-row (both atoms) and 32-row boxes
+};
+
+// Shared-memory descriptor of a scale atom for tcgen05.cp: 32 rows of 16
+// bytes, no swizzle, i.e. core matrices of 8 rows x 16 bytes, 16 bytes apart
+// along K (leading offset) and 128 bytes apart along the rows (stride
+// offset); version 1 in bits [46, 48).
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(16u >> 4) << 16) |
+         (static_cast<uint64_t>(128u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46);
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4 with A = E2M1 (format
+// 5 in bits [7, 10)), B = E4M3 (0 in [10, 13)), both K-major, E8M0 scales
+// (bit 23), N >> 3 in [17, 23), M >> 4 in [24, 29), and the byte j of the
+// scale column that holds this K = 32 step's scales: A's in [29, 31), B's in
+// [4, 6).
+__host__ __device__ constexpr uint32_t idesc_mxf4_mxf8(int M, int N, int j) {
+  return (static_cast<uint32_t>(j) << 4) | (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(j) << 29);
+}
+
+// 32 rows x 128 bits of shared memory -> tensor memory lanes 0-31 of every
+// lane quarter (4 columns from taddr), in both CTAs of the pair.
+__device__ __forceinline__ void bs_copy_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= (A . 2^sfa) (B . 2^sfb)^T, one 256 x N x 32 step on the pair.
+__device__ __forceinline__ void bs_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane (32x32b shape, x16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* r) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]), "=r"(u[8]),
+        "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+      : "r"(taddr));
+}
+
+// Columns ch*32 .. ch*32+31 of the accumulator (only the first 16 when the
+// tile ends within them, so that no load reaches past the tile's columns).
+__device__ __forceinline__ void bs_load_chunk(uint32_t tbase, int ch, int ntok, float (&r)[32]) {
+  if (ch * 32 + 16 >= ntok) {
+    tmem_ld16(tbase + ch * 32, r);
+#pragma unroll
+    for (int i = 16; i < 32; ++i) r[i] = 0.f;
+  } else {
+    tmem_ld32(tbase + ch * 32, r);
+  }
+}
+
+// A work item with the token tile clamped to BS_MAX_TILE_ROWS rows (a table
+// built for larger tiles records `site` in the fault flag and is cut, so that
+// no accumulator column outside the tile's 240 is written or read).  Every
+// role decodes the same item, so all see the same clamp.
+__device__ __forceinline__ ExTile bs_decode(int w, int num_tiles, int num_multi, const ExParams& p, bool report) {
+  ExTile t = ex_decode(w, num_tiles, num_multi, p);
+  if (t.ntok > BS_MAX_TILE_ROWS) {
+    if (report) record_fault(p.fault_site + 9);
+    t.ntok = BS_MAX_TILE_ROWS;
+    t.n_mma = BS_MAX_TILE_ROWS;
+  }
+  return t;
+}
+
+template <int EPI, bool PAIRED>
+__global__ void __launch_bounds__(BS_THREADS, 1)
+    tc_expert_bs_kernel(const __grid_constant__ BsMaps maps, const ExParams p) {
+  constexpr int CG = 2;
+  extern __shared__ uint8_t bs_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bs_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + BS_STAGES * BS_A_BYTES;
+  uint8_t* sSA = sB + BS_STAGES * BS_B_BYTES;
+  uint8_t* sSB = sSA + BS_STAGES * BS_SFA_BYTES;
+  float* xch = reinterpret_cast<float*>(sSB + BS_STAGES * BS_SFB_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + EX_XCH_BYTES);
+  uint64_t* empty = full + BS_STAGES;
+  uint64_t* acc_full = empty + BS_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_ok = abort + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < BS_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4 * CG);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.a0);
+    if (PAIRED) tma_prefetch_desc(&maps.a1);
+    tma_prefetch_desc(&maps.sa);
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(&maps.b[i]);
+    tma_prefetch_desc(&maps.sb[0]);
+    tma_prefetch_desc(&maps.sb[1]);
+  }
+  if (warp == 1) ex_tmem_alloc<CG>(tmem_holder);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int num_tiles = p.num_tiles_dev[0];
+  const int num_multi = p.num_tiles_dev[1];
+  const int total = num_tiles * p.n_wtiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0u, issued_parity = 0u;
+      bool ok = true;
+      const uint64_t pol_w = l2_policy_evict_first(), pol_t = l2_policy_evict_last();
+      for (int w = pair; w < total && ok; w += npairs) {
+        const ExTile t = bs_decode(w, num_tiles, num_multi, p, true);
+        const int rows_cta = t.n_mma / 2;  // token rows this CTA stages
+        const int bsel = rows_cta > 64 ? 0 : rows_cta > 32 ? 1 : rows_cta > 16 ? 2 : 3;
+        const int brows = 128 >> bsel;
+        const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
+        const bool two_atoms = t.n_mma > 128;
+        const uint32_t bytes = static_cast<uint32_t>(CG) * (BS_A_TX + static_cast<uint32_t>(brows) * BS_BK +
+                                                            BS_SFA_BYTES + (two_atoms ? 1024u : 512u));
+        const int wrow = t.expert * p.w_rows_per_expert + (PAIRED ? t.wt * 128 : t.wt * 256) +
+                         static_cast<int>(rank) * (PAIRED ? 64 : 128);
+        // 16-byte rows of the scale tiles: 32 per atom
+        const int sa_row0 = ((t.expert * p.n_wtiles + t.wt) * 2 + static_cast<int>(rank)) * p.num_k_blocks * 32;
+        const int sb_row0 = t.tt * p.num_k_blocks * 64;
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.fault_site + 1)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
+          const int kc = kb * BS_BK;
+          uint8_t* a_dst = sA + stage * BS_A_BYTES;
+          if (kExL2Hints && !t.multi) {
+            ex_tma_load_hint<CG>(a_dst, &maps.a0, &full[stage], kc, wrow, pol_w);
+            if (PAIRED) ex_tma_load_hint<CG>(a_dst + BS_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
+          } else {
+            ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
+            if (PAIRED) ex_tma_load<CG>(a_dst + BS_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
+          }
+          ex_tma_load<CG>(sSA + stage * BS_SFA_BYTES, &maps.sa, &full[stage], 0, sa_row0 + kb * 32);
+          ex_tma_load_hint<CG>(sB + stage * BS_B_BYTES, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
+          ex_tma_load<CG>(sSB + stage * BS_SFB_BYTES, &maps.sb[two_atoms ? 0 : 1], &full[stage], 0, sb_row0 + kb * 64);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == BS_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // The even CTA's barriers count both CTAs' bytes: it waits for every
+      // load of the pair to land before the pair may exit.
+      if (leader) {
+        volatile int never = 0;
+        for (int s = 0; s < BS_STAGES; ++s)
+          if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_parity >> s) & 1u, &never, p.fault_site + 2);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      const uint32_t sf_a = tmem_base + BS_SF_COL, sf_b = sf_a + 4u;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const ExTile t = bs_decode(w, num_tiles, num_multi, p, false);
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort, p.fault_site + 3)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * BS_ACC_COLS;
+        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort, p.fault_site + 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          bs_copy_sf(sf_a, sf_atom_desc(smem_u32(sSA + stage * BS_SFA_BYTES)));
+          bs_copy_sf(sf_b, sf_atom_desc(smem_u32(sSB + stage * BS_SFB_BYTES)));
+          if (t.n_mma > 128) bs_copy_sf(sf_b + 4u, sf_atom_desc(smem_u32(sSB + stage * BS_SFB_BYTES + 512)));
+          const uint32_t a_addr = smem_u32(sA + stage * BS_A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * BS_B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BS_BK / 32; ++kk) {
+            const uint32_t j = static_cast<uint32_t>(kk) << 30;  // scale byte of this K = 32 step
+            bs_mma(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
+                   idesc_mxf4_mxf8(256, t.n_mma, kk), sf_a | j, sf_b | j, (kb | kk) != 0 ? 1u : 0u);
+          }
+          ex_commit<CG>(&empty[stage]);
+          if (++stage == BS_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ex_commit<CG>(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      ex_commit<CG>(drain);
+    }
+    // Both CTAs: every MMA and copy touching this CTA's shared memory or TMEM is done.
+    if (lane == 0) {
+      volatile int never = 0;
+      mbar_wait(drain, 0u, &never, p.fault_site + 5);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const uint32_t acc_empty_leader = map_to_rank(smem_u32(&acc_empty[0]), 0u);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int xbuf = 0;
+    for (int w = pair; w < total; w += npairs) {
+      const ExTile t = bs_decode(w, num_tiles, num_multi, p, false);
+      bool got;
+      if constexpr (PAIRED) {
+        if (threadIdx.x == 64) *epi_ok = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
+        epilogue_bar();
+        got = *epi_ok != 0;
+      } else {
+        got = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6));
+      }
+      if (!got) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc) * BS_ACC_COLS;
+      const int nch = (t.ntok + 31) >> 5;
+      if constexpr (PAIRED) {
+        // warps 0,1 hold g and warps 2,3 hold v for intermediate columns
+        // base + 32 * (q & 1) + lane; g warps form tokens 0-15 of a chunk,
+        // v warps tokens 16-31, after swapping the other half.
+        const bool is_g = q < 2;
+        const int col = t.wt * 128 + static_cast<int>(rank) * 64 + (q & 1) * 32 + lane;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+        const float c = p.situ_c;
+        const float inv_c = 1.0f / c;
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          float r[32];
+          bs_load_chunk(tbase, ch, t.ntok, r);
+          float* X = xch + xbuf * EX_XCH_FLOATS + (q & 1) * 1024;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (is_g)
+              X[i * 32 + lane] = r[16 + i];
+            else
+              X[512 + i * 32 + lane] = r[i];
+          }
+          epilogue_bar();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g = is_g ? r[i] : X[i * 32 + lane];
+            const float v = is_g ? X[512 + i * 32 + lane] : r[16 + i];
+            const int tok = ch * 32 + (is_g ? 0 : 16) + i;
+            if (tok < t.ntok && col < p.out_cols)
+              out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = __float2bfloat16_rn(situ_glu_fast(g, v, c, inv_c));
+          }
+          xbuf ^= 1;
+        }
+      } else {
+        const int col = t.wt * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        float* out = reinterpret_cast<float*>(p.out);
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          float r[32];
+          bs_load_chunk(tbase, ch, t.ntok, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = ch * 32 + i;
+            if (tok < t.ntok && col < p.out_cols) out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = r[i];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncwarp();  // reconverge lanes that skipped the single-thread roles
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    ex_tmem_dealloc<CG>(tmem_base);
+  }
+}
+
+}  // namespace moe

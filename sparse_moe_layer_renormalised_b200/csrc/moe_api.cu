@@ -8,12 +8,16 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
+#include <functional>
 #include <mutex>
 
 #include "backward.cuh"
 #include "combine.cuh"
 #include "gemm_expert.cuh"
 #include "gemm_expert2.cuh"
+#include "gemm_expert_bs.cuh"
+#include "mx8.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -41,7 +45,8 @@ bool dims_ok(const moe_dims* d) {
   if (!(d->situ_c > 0.f) || !std::isfinite(d->situ_c) || !(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps))
     return false;
   if (d->act != MOE_F32 && d->act != MOE_BF16) return false;
-  if (d->routed != MOE_F32 && d->routed != MOE_BF16 && d->routed != MOE_MXFP4) return false;
+  if (d->routed != MOE_F32 && d->routed != MOE_BF16 && d->routed != MOE_MXFP4 && d->routed != MOE_MXFP4_A8)
+    return false;
   if (d->y_out != MOE_F32 && d->y_out != d->act) return false;
   if (d->L % 8 != 0 || d->H % 8 != 0 || d->I % 8 != 0) return false;
   if (d->S > 0 && d->Is % 8 != 0) return false;
@@ -51,9 +56,11 @@ bool dims_ok(const moe_dims* d) {
 
 // Valid dims that this build does not implement.
 bool dims_supported(const moe_dims* d) {
-  if (d->routed == MOE_MXFP4) {
+  if (d->routed == MOE_MXFP4 || d->routed == MOE_MXFP4_A8) {
     // MXFP4 routed weights: bf16 activations; code and scale rows must suit TMA
     // (K/2 and K/32 bytes per row, multiples of 16) for both expert GEMMs.
+    // (The block-scaled path also needs K % 128 and 2-CTA weight tiles, which
+    // these multiples give.)
     if (d->act != MOE_BF16 || d->L % 512 != 0 || d->I % 512 != 0) return false;
   } else if (d->routed != d->act) {
     return false;
@@ -81,14 +88,20 @@ inline size_t act_bytes(const moe_dims& d) { return d.act == MOE_F32 ? 4 : 2; }
 int expert_cg(const moe_dims& d) { return (d.I % 128 == 0 && d.L % 256 == 0) ? 2 : 1; }
 
 // Largest token tile of the grouped expert GEMMs (MMA N = 256 on pairs; a
-// single CTA stages at most 128 token rows; the fp32 path uses 128-row tiles).
-int expert_tile_rows(const moe_dims& d) { return d.act == MOE_BF16 ? 128 * expert_cg(d) : 128; }
+// single CTA stages at most 128 token rows; the fp32 path uses 128-row tiles;
+// the block-scaled path 240, which leaves tensor memory for its scales).
+int expert_tile_rows(const moe_dims& d) {
+  if (d.routed == MOE_MXFP4_A8) return BS_MAX_TILE_ROWS;
+  return d.act == MOE_BF16 ? 128 * expert_cg(d) : 128;
+}
+
+inline bool routed_a8(const moe_dims& d) { return d.routed == MOE_MXFP4_A8; }
 
 
 // ------------------------------------------------------------------------------ workspace
 struct WsLayout {
   size_t scores, topk_idx, topk_w, rank, tile_base, counts, offsets, tile_table, num_m_tiles, perm_token,
-      inv_perm, z, z_perm, h_perm, y_perm, n, h_s, dense_tiles, dense_num, total;
+      inv_perm, z, z_perm, h_perm, y_perm, n, h_s, dense_tiles, dense_num, h_q, sf_z, sf_h, total;
 };
 
 WsLayout ws_layout(const moe_dims& d) {
@@ -121,6 +134,12 @@ WsLayout ws_layout(const moe_dims& d) {
   w.h_s = take(T * static_cast<size_t>(d.S) * d.Is * es);
   w.dense_tiles = take(static_cast<size_t>(cdiv(static_cast<long long>(T), 128) + 1) * 16);
   w.dense_num = take(16);
+  // block-scaled path: E4M3 codes of h and the activation scale tiles (the
+  // codes of the expert-major z rows reuse z_perm)
+  const bool a8 = routed_a8(d);
+  w.h_q = take(a8 ? R * d.I : 0);
+  w.sf_z = take(a8 ? max_m_tiles * (d.L / 128) * 1024 : 0);
+  w.sf_h = take(a8 ? max_m_tiles * (d.I / 128) * 1024 : 0);
   w.total = off;
   return w;
 }
@@ -175,6 +194,37 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed E2M1 codes [rows, K] (K elements, K/2 bytes a row), boxes of 128
+// elements x box_rows rows landing as 16-byte slots of 16 codes and 8 bytes of
+// gap (the shared-memory layout tcgen05.mma kind::mxf8f6f4 reads for 4-bit
+// operands), 128-byte swizzle.  The driver requires a 32-byte aligned base,
+// K % 128 == 0 and a row pitch that is a multiple of 32 bytes.
+bool make_map_e2m1(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows == 0 || K == 0) return false;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K / 2};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// uint8 matrix [rows, cols] with boxes 128 bytes wide x box_rows rows and
+// 128-byte swizzle (E4M3 activation codes as an MMA operand).
+bool make_map_u8_sw128(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -631,6 +681,110 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
   return launch_expert<kEpiF32, false>(cg, mx, maps, p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------------------ block-scaled routed experts
+// Quantises rows of the grouped-GEMM token tiles to MXFP8 (codes [R, K] and
+// scale tiles; see mx8.cuh).  Row r reads src row src_row[r] (or r).
+moe_status stage_quant_mx8(const void* src, long long src_rows, const int32_t* src_row, const int4* table,
+                           const int32_t* n_tiles, int max_tiles, int K, uint8_t* codes, uint8_t* sf, int site,
+                           cudaStream_t s) {
+  const int grid = std::max(1, std::min(max_tiles, 8 * num_sms()));
+  mx8_quant_tiles_kernel<<<grid, MX8_WARPS * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(src), src_rows, src_row,
+                                                          table, n_tiles, 0, K, codes, sf, site);
+  ++g_last_launches;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int EPI, bool PAIRED>
+cudaError_t launch_expert_bs(const BsMaps& maps, const ExParams& p, cudaStream_t s) {
+  auto kern = tc_expert_bs_kernel<EPI, PAIRED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(BS_SMEM));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(BS_THREADS);
+  cfg.dynamicSmemBytes = BS_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int pairs_cache[128] = {};  // per instantiation and device
+  cfg.gridDim = dim3(2 * cluster_pairs(kern, cfg, pairs_cache));
+  return cudaLaunchKernelEx(&cfg, kern, maps, p);
+}
+
+// Bytes of the re-ordered weight scales of the block-scaled kernels.
+size_t tiled_scales_gate_up(const moe_dims& d) {
+  return static_cast<size_t>(d.E) * (d.I / 128) * 2 * (d.L / 128) * 512;
+}
+size_t tiled_scales_down(const moe_dims& d) {
+  return static_cast<size_t>(d.E) * (d.L / 256) * 2 * (d.I / 128) * 512;
+}
+
+// One block-scaled grouped GEMM: paired = gate/up (W_g / W_v over the latent
+// rows, SiTU-GLU -> bf16 h [R, I]); else down (W_o over h -> fp32 [R, L]).
+moe_status stage_expert_bs(const moe_dims& d, bool paired, const moe_weights& w, const uint8_t* act_q,
+                           const uint8_t* act_sf, long long R, const int4* table, const int32_t* n_tiles,
+                           int max_tiles, void* out, int site, cudaStream_t s) {
+  ++g_last_launches;
+  const int K = paired ? d.L : d.I;
+  const int out_rows = paired ? d.I : d.L;  // weight rows per expert
+  BsMaps maps;
+  std::memset(&maps, 0, sizeof maps);
+  const uint64_t wrows = static_cast<uint64_t>(d.E) * out_rows;
+  const size_t sa_bytes = paired ? tiled_scales_gate_up(d) : tiled_scales_down(d);
+  bool ok = true;
+  if (paired)
+    ok = make_map_e2m1(&maps.a0, w.Wg, wrows, K, 64) && make_map_e2m1(&maps.a1, w.Wv, wrows, K, 64) &&
+         make_map_u8(&maps.sa, w.Sgv_tiled, sa_bytes / 16, 16, 16, 32);
+  else
+    ok = make_map_e2m1(&maps.a0, w.Wo, wrows, K, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, 32);
+  for (int i = 0; i < 4 && ok; ++i) ok = make_map_u8_sw128(&maps.b[i], act_q, static_cast<uint64_t>(R), K, 128u >> i);
+  const uint64_t sf_rows = static_cast<uint64_t>(max_tiles) * (K / 128) * 64;
+  ok = ok && make_map_u8(&maps.sb[0], act_sf, sf_rows, 16, 16, 64) && make_map_u8(&maps.sb[1], act_sf, sf_rows, 16, 16, 32);
+  if (!ok) return MOE_ERR_CUDA;
+  ExParams p{};
+  p.tile_table = table;
+  p.num_tiles_dev = n_tiles;
+  p.n_wtiles = paired ? d.I / 128 : d.L / 256;
+  p.w_rows_per_expert = out_rows;
+  p.num_k_blocks = K / BS_BK;
+  p.out = out;
+  p.ldo = out_rows;
+  p.out_cols = out_rows;
+  p.situ_c = d.situ_c;
+  p.fault_site = site;
+  const cudaError_t e = paired ? launch_expert_bs<kEpiSituBF16, true>(maps, p, s) : launch_expert_bs<kEpiF32, false>(maps, p, s);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Buffers of the block-scaled routed-expert sequence.
+struct A8Bufs {
+  uint8_t* xq;   // [R, L] E4M3 codes of the expert-major latent rows
+  uint8_t* sfx;  // their scale tiles
+  void* h;       // [R, I] bf16 SiTU-GLU output
+  uint8_t* hq;   // [R, I] E4M3 codes of h
+  uint8_t* sfh;  // their scale tiles
+};
+
+// The routed experts on the block-scaled path after the latent rows have been
+// quantised: gate/up -> h, h -> MXFP8, down -> y [R, L] fp32.
+moe_status run_routed_a8_after_quant(const moe_dims& d, const moe_weights& w, const A8Bufs& b, long long R,
+                                     const int4* table, const int32_t* n_tiles, int max_tiles, float* y,
+                                     cudaStream_t s, const std::function<void(int, int)>& mark) {
+  moe_status st;
+  mark(MOE_STAGE_EXPERT_GATE_UP, 0);
+  if ((st = stage_expert_bs(d, true, w, b.xq, b.sfx, R, table, n_tiles, max_tiles, b.h, 160, s)) != MOE_OK) return st;
+  mark(MOE_STAGE_EXPERT_GATE_UP, 1);
+  mark(MOE_STAGE_EXPERT_DOWN, 0);
+  if ((st = stage_quant_mx8(b.h, R, nullptr, table, n_tiles, max_tiles, d.I, b.hq, b.sfh, 181, s)) != MOE_OK) return st;
+  st = stage_expert_bs(d, false, w, b.hq, b.sfh, R, table, n_tiles, max_tiles, y, 170, s);
+  mark(MOE_STAGE_EXPERT_DOWN, 1);
+  return st;
+}
+
 // The shared experts' gate/up projection with the SiTU-GLU epilogue.  With
 // bf16 weights it runs on the 2-CTA grouped expert kernel as one "expert"
 // whose S*Is weight rows are W_sg / W_sv (paired row by row) over token tiles
@@ -720,19 +874,31 @@ moe_status stage_output(const moe_dims& d, const moe_weights& w, const void* h_s
 
 // MXFP4 routed weights need their E8M0 scale arrays; other types take none.
 moe_status check_scales(const moe_dims& d, const moe_weights& w) {
+  if (routed_a8(d)) {
+    // block-scaled path: the re-ordered scales (the row-major ones are not
+    // read and may be NULL); the packed codes are read as 4-bit TMA tensors,
+    // which need 32-byte aligned bases
+    if (w.Sgv_tiled == nullptr || w.So_tiled == nullptr || !aligned16(w.Sgv_tiled) || !aligned16(w.So_tiled))
+      return MOE_ERR_INVALID_ARG;
+    const void* codes[] = {w.Wg, w.Wv, w.Wo};
+    for (const void* p : codes)
+      if ((reinterpret_cast<uintptr_t>(p) & 31u) != 0) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+  }
   const bool mx = d.routed == MOE_MXFP4;
   const void* sc[] = {w.Sg, w.Sv, w.So};
   for (const void* p : sc) {
     if (mx && (p == nullptr || !aligned16(p))) return MOE_ERR_INVALID_ARG;
     if (!mx && p != nullptr) return MOE_ERR_INVALID_ARG;
   }
+  if (w.Sgv_tiled != nullptr || w.So_tiled != nullptr) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
 // Workspace of moe_expert_ffn_blocks: h for every row, and a tile table for
 // up to ceil(n_rows / 128) + E * n_blocks tiles.
 struct BlocksWsLayout {
-  size_t h, tile_table, num_tiles, total;
+  size_t h, tile_table, num_tiles, xq, sfx, hq, sfh, total;  // xq .. sfh: block-scaled path only
   int max_tiles;
 };
 
@@ -748,6 +914,12 @@ BlocksWsLayout blocks_ws_layout(const moe_dims& d, long long n_rows, int n_block
   l.h = take(static_cast<size_t>(n_rows) * d.I * act_bytes(d));
   l.tile_table = take(static_cast<size_t>(l.max_tiles) * 16);
   l.num_tiles = take(16);
+  const bool a8 = routed_a8(d);
+  const size_t rows = static_cast<size_t>(n_rows), mt = static_cast<size_t>(l.max_tiles);
+  l.xq = take(a8 ? rows * d.L : 0);
+  l.sfx = take(a8 ? mt * (d.L / 128) * 1024 : 0);
+  l.hq = take(a8 ? rows * d.I : 0);
+  l.sfh = take(a8 ? mt * (d.I / 128) * 1024 : 0);
   l.total = off;
   return l;
 }
@@ -1092,6 +1264,15 @@ moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   const int4* table = at<int4>(ws, L.tile_table);
   const int32_t* n_tiles = at<int32_t>(ws, L.num_m_tiles);
+  if (routed_a8(*d)) {
+    const long long R = d->T * d->k;
+    const int max_tiles = static_cast<int>(cdiv(R, TC_BM) + d->E);
+    const A8Bufs b{at<uint8_t>(ws, L.z_perm), at<uint8_t>(ws, L.sf_z), at<void>(ws, L.h_perm), at<uint8_t>(ws, L.h_q),
+                   at<uint8_t>(ws, L.sf_h)};
+    if ((st = stage_quant_mx8(z_perm, R, nullptr, table, n_tiles, max_tiles, d->L, b.xq, b.sfx, 180, s)) != MOE_OK)
+      return st;
+    return run_routed_a8_after_quant(*d, *w, b, R, table, n_tiles, max_tiles, y_perm, s, [](int, int) {});
+  }
   st = stage_expert_gate_up(*d, *w, z_perm, table, n_tiles, at<void>(ws, L.h_perm), s);
   if (st != MOE_OK) return st;
   return stage_expert_down(*d, *w, at<void>(ws, L.h_perm), table, n_tiles, y_perm, s);
@@ -1171,20 +1352,36 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
   mark(MOE_STAGE_PERMUTE, 0);
   if ((st = stage_permute(*d, idx, L, ws, offsets, nullptr, perm_token, inv_perm, s)) != MOE_OK) return st;
   mark(MOE_STAGE_PERMUTE, 1);
-  mark(MOE_STAGE_GATHER, 0);
-  if ((st = stage_gather(*d, z, at<void>(ws, L.z_perm), perm_token, offsets + d->E, s)) != MOE_OK) return st;
-  mark(MOE_STAGE_GATHER, 1);
   // routed experts
   const int4* table = at<int4>(ws, L.tile_table);
   const int32_t* n_tiles = at<int32_t>(ws, L.num_m_tiles);
-  mark(MOE_STAGE_EXPERT_GATE_UP, 0);
-  if ((st = stage_expert_gate_up(*d, *w, at<void>(ws, L.z_perm), table, n_tiles, at<void>(ws, L.h_perm), s)) != MOE_OK)
-    return st;
-  mark(MOE_STAGE_EXPERT_GATE_UP, 1);
-  mark(MOE_STAGE_EXPERT_DOWN, 0);
-  if ((st = stage_expert_down(*d, *w, at<void>(ws, L.h_perm), table, n_tiles, at<float>(ws, L.y_perm), s)) != MOE_OK)
-    return st;
-  mark(MOE_STAGE_EXPERT_DOWN, 1);
+  if (routed_a8(*d)) {
+    // block-scaled path: the gather writes the MXFP8 codes and scales of the
+    // expert-major z rows; h is quantised in the down stage
+    const long long R = d->T * d->k;
+    const int max_tiles = static_cast<int>(cdiv(R, TC_BM) + d->E);
+    const A8Bufs b{at<uint8_t>(ws, L.z_perm), at<uint8_t>(ws, L.sf_z), at<void>(ws, L.h_perm), at<uint8_t>(ws, L.h_q),
+                   at<uint8_t>(ws, L.sf_h)};
+    mark(MOE_STAGE_GATHER, 0);
+    if ((st = stage_quant_mx8(z, d->T, perm_token, table, n_tiles, max_tiles, d->L, b.xq, b.sfx, 180, s)) != MOE_OK)
+      return st;
+    mark(MOE_STAGE_GATHER, 1);
+    if ((st = run_routed_a8_after_quant(*d, *w, b, R, table, n_tiles, max_tiles, at<float>(ws, L.y_perm), s, mark)) !=
+        MOE_OK)
+      return st;
+  } else {
+    mark(MOE_STAGE_GATHER, 0);
+    if ((st = stage_gather(*d, z, at<void>(ws, L.z_perm), perm_token, offsets + d->E, s)) != MOE_OK) return st;
+    mark(MOE_STAGE_GATHER, 1);
+    mark(MOE_STAGE_EXPERT_GATE_UP, 0);
+    if ((st = stage_expert_gate_up(*d, *w, at<void>(ws, L.z_perm), table, n_tiles, at<void>(ws, L.h_perm), s)) != MOE_OK)
+      return st;
+    mark(MOE_STAGE_EXPERT_GATE_UP, 1);
+    mark(MOE_STAGE_EXPERT_DOWN, 0);
+    if ((st = stage_expert_down(*d, *w, at<void>(ws, L.h_perm), table, n_tiles, at<float>(ws, L.y_perm), s)) != MOE_OK)
+      return st;
+    mark(MOE_STAGE_EXPERT_DOWN, 1);
+  }
   // combine + RMSNorm, then [shared | W_up] output projection
   mark(MOE_STAGE_COMBINE, 0);
   if ((st = stage_combine(*d, at<float>(ws, L.y_perm), inv_perm, tw, w->gamma, a.u, n, s)) != MOE_OK) return st;
@@ -1263,9 +1460,59 @@ moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const 
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   const int4* table = at<int4>(ws, L.tile_table);
   const int32_t* n_tiles = at<int32_t>(ws, L.num_tiles);
+  if (routed_a8(dr)) {
+    const A8Bufs b{at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.sfx), at<void>(ws, L.h), at<uint8_t>(ws, L.hq),
+                   at<uint8_t>(ws, L.sfh)};
+    if ((st = stage_quant_mx8(x_rows, n_rows, nullptr, table, n_tiles, L.max_tiles, d->L, b.xq, b.sfx, 180, s)) !=
+        MOE_OK)
+      return st;
+    return run_routed_a8_after_quant(dr, *w, b, n_rows, table, n_tiles, L.max_tiles, y_rows, s, [](int, int) {});
+  }
   st = stage_expert_gate_up(dr, *w, x_rows, table, n_tiles, at<void>(ws, L.h), s, L.max_tiles);
   if (st != MOE_OK) return st;
   return stage_expert_down(dr, *w, at<void>(ws, L.h), table, n_tiles, y_rows, s, L.max_tiles);
+}
+
+moe_status moe_mx8_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
+                            moe_stream_t stream) {
+  if (rows < 0 || K <= 0 || K % 32 != 0 || rows > 0x7fffffffLL) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || codes == nullptr || scales == nullptr || !aligned16(x) || !aligned16(codes)))
+    return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (rows == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long tiles = cdiv(rows, 128);
+  const int grid = static_cast<int>(std::min<long long>(tiles, 8LL * num_sms()));
+  mx8_quant_tiles_kernel<<<grid, MX8_WARPS * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, nullptr, nullptr,
+                                                          nullptr, rows, K, codes, scales, 182);
+  g_last_launches = 1;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_mx_tiled_scales_size(const moe_dims* d, size_t* gate_up_bytes, size_t* down_bytes) {
+  if (!dims_ok(d) || gate_up_bytes == nullptr || down_bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->L % 512 != 0 || d->I % 512 != 0) return MOE_ERR_UNSUPPORTED;
+  *gate_up_bytes = tiled_scales_gate_up(*d);
+  *down_bytes = tiled_scales_down(*d);
+  return MOE_OK;
+}
+
+moe_status moe_mx_tile_scales(const moe_dims* d, const uint8_t* Sg, const uint8_t* Sv, const uint8_t* So,
+                              uint8_t* Sgv_tiled, uint8_t* So_tiled, moe_stream_t stream) {
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  if (d->L % 512 != 0 || d->I % 512 != 0) return MOE_ERR_UNSUPPORTED;
+  const void* ptrs[] = {Sg, Sv, So, Sgv_tiled, So_tiled};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long n_gu = static_cast<long long>(tiled_scales_gate_up(*d));
+  const long long n_dn = static_cast<long long>(tiled_scales_down(*d));
+  const int grid = 4 * num_sms();
+  mx_tile_weight_scales_kernel<<<grid, 256, 0, s>>>(Sg, Sv, d->I, d->L, 1, n_gu, Sgv_tiled);
+  mx_tile_weight_scales_kernel<<<grid, 256, 0, s>>>(So, nullptr, d->L, d->I, 0, n_dn, So_tiled);
+  g_last_launches = 2;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 size_t moe_backward_workspace_size(const moe_dims* d) {

@@ -36,6 +36,7 @@ import numpy as np
 import torch
 import torch.distributed as dist
 
+from .layer import tile_weight_scales
 from ._binding import (Dims, check, make_weights, moe_combine, moe_expert_ffn_blocks,
                        moe_expert_ffn_blocks_workspace_size, moe_latent_shared, moe_output, moe_permute,
                        moe_router_topk, moe_workspace_size)
@@ -137,6 +138,8 @@ class ExpertParallelMoeLayer:
     dims: the full layer (E = all routed experts).  weights: device tensors
     named as moe_weights' fields; Wg / Wv / Wo (and Sg / Sv / So for MXFP4)
     hold only this rank's experts, bounds[rank] .. bounds[rank+1]-1, in order.
+    With routed = "mxfp4_a8" the dispatched rows stay bf16 and the receiving
+    rank quantises them (moe_expert_ffn_blocks).
     max_tokens sizes the local workspaces."""
 
     def __init__(self, dims: Dims, weights: dict, group=None, max_tokens: int | None = None):
@@ -148,13 +151,16 @@ class ExpertParallelMoeLayer:
         self.e_local = int(self.bounds[self.rank + 1] - self.bounds[self.rank])
         if weights["Wg"].shape[0] != self.e_local:
             raise ValueError(f"rank {self.rank} holds {weights['Wg'].shape[0]} experts, expected {self.e_local}")
-        self.weights = weights
-        self._w = make_weights(**weights)
+        self.local_dims = replace(dims, E=self.e_local)
+        self.weights = dict(weights)
+        if dims.routed == "mxfp4_a8" and "Sgv_tiled" not in weights:
+            # the block-scaled experts read their scales in tiled order, made once per rank
+            self.weights.update(tile_weight_scales(self.local_dims, weights["Sg"], weights["Sv"], weights["So"]))
+        self._w = make_weights(**self.weights)
         self.max_tokens = dims.T if max_tokens is None else max_tokens
         dev = weights["Wr"].device
         self.workspace = torch.empty(moe_workspace_size(replace(dims, T=self.max_tokens)), dtype=torch.uint8,
                                      device=dev)
-        self.local_dims = replace(dims, E=self.e_local)
 
     def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         d = replace(self.dims, T=x.shape[0])

@@ -7,23 +7,40 @@ from dataclasses import replace
 
 import torch
 
-from ._binding import Dims, check, make_aux, make_weights, moe_layer_forward, moe_workspace_size
+from ._binding import (Dims, check, make_aux, make_weights, moe_layer_forward, moe_mx_tile_scales,
+                       moe_mx_tiled_scales_size, moe_workspace_size)
 
 _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def tile_weight_scales(dims: Dims, Sg: torch.Tensor, Sv: torch.Tensor, So: torch.Tensor, stream=None) -> dict:
+    """The routed weights' E8M0 scales in the tiled order of the block-scaled
+    expert kernels (moe_mx_tile_scales): {"Sgv_tiled", "So_tiled"} uint8 device
+    tensors, to pass as weights alongside the codes."""
+    st, n_gu, n_dn = moe_mx_tiled_scales_size(dims)
+    check(st)
+    gu = torch.empty(n_gu, dtype=torch.uint8, device=Sg.device)
+    dn = torch.empty(n_dn, dtype=torch.uint8, device=Sg.device)
+    check(moe_mx_tile_scales(dims, Sg, Sv, So, gu, dn, stream))
+    return {"Sgv_tiled": gu, "So_tiled": dn}
 
 
 class MoeLayer:
     """Weights: dict with Wr, bias, Wdown, Wup, gamma, Wg, Wv, Wo, Wsg, Wsv, Wso
     and, for MXFP4 routed weights, Sg, Sv, So (device tensors in the shapes of
-    include/moe.h).  max_tokens sizes the
+    include/moe.h).  With routed = "mxfp4_a8" (block-scaled MXFP8 x MXFP4
+    experts) the scales are re-ordered once here by moe_mx_tile_scales into
+    Sgv_tiled / So_tiled, which the layer keeps.  max_tokens sizes the
     workspace; each call may use any T <= max_tokens."""
 
     def __init__(self, dims: Dims, weights: dict, max_tokens: int | None = None):
         self.dims = dims
-        self.weights = weights
+        self.weights = dict(weights)
         self.max_tokens = dims.T if max_tokens is None else max_tokens
-        self._w = make_weights(**weights)
         dev = weights["Wr"].device
+        if dims.routed == "mxfp4_a8" and "Sgv_tiled" not in weights:
+            self.weights.update(tile_weight_scales(dims, weights["Sg"], weights["Sv"], weights["So"]))
+        self._w = make_weights(**self.weights)
         nbytes = moe_workspace_size(replace(dims, T=self.max_tokens))
         if nbytes == 0:
             raise ValueError(f"invalid layer dimensions {dims}")

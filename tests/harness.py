@@ -3,6 +3,7 @@ from the seeded generator, oracle references, and the parity metrics."""
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 import torch
@@ -17,6 +18,12 @@ F64 = torch.float64
 # Tolerances (max|y - y_ref| / rms(y_ref)) stated for the layer output.
 TOL_BF16 = 1e-2
 TOL_MXFP4 = 3e-2
+# Block-scaled path: the oracle quantises the same bf16 rows to MXFP8, so both
+# sides multiply the same numbers except where the device's bf16 z or h differs
+# from the oracle's by a rounding step and the E4M3 code of that element
+# changes (one code step is 1/16 - 1/8 of the element); the bar is the MXFP4
+# layer's.
+TOL_MXFP4_A8 = 3e-2
 TOL_F32 = 1e-4
 NEAR_TIE = 1e-4  # key margin below which an index-set difference is allowed
 # Router scores and mixture weights: fp32 on the device from the same bf16 (or
@@ -28,6 +35,10 @@ NEAR_TIE = 1e-4  # key margin below which an index-set difference is allowed
 TOL_SCORES = 1e-4
 TOL_P_REL = 1e-4
 TOL_Z_F32 = 1e-5
+
+
+# Tokens of the K3-size workloads checked against the oracle.
+K3_SAMPLE = int(os.environ.get("MOE_K3_SAMPLE", "512"))
 
 
 def dims_for(cfg, T=None, y_out="f32") -> moe.Dims:

@@ -25,7 +25,7 @@ def _dims(**kw):
 
 def test_library_exports_every_declared_symbol():
     names = _declared()
-    assert len(names) == 18
+    assert len(names) == 21
     lib = ctypes.CDLL(moe.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -62,6 +62,8 @@ FAKE = 1 << 20  # an aligned address; never dereferenced because validation fail
     (dict(y_out="mxfp4"), moe.MOE_ERR_INVALID_ARG),
     (dict(routed="mxfp4"), moe.MOE_ERR_UNSUPPORTED),  # L = 1024 fine, I = 768 not a multiple of 512
     (dict(routed="mxfp4", act="f32", y_out="f32"), moe.MOE_ERR_UNSUPPORTED),
+    (dict(routed="mxfp4_a8"), moe.MOE_ERR_UNSUPPORTED),  # I = 768 not a multiple of 512
+    (dict(routed="mxfp4_a8", I=1024, act="f32", y_out="f32"), moe.MOE_ERR_UNSUPPORTED),
     (dict(H=2056), moe.MOE_ERR_UNSUPPORTED),
     (dict(S=4), moe.MOE_ERR_UNSUPPORTED),
 ])
@@ -154,3 +156,55 @@ def test_stage_entry_points_validate_before_launching():
     assert moe.moe_expert_ffn_blocks(d, w, FAKE, 1000, FAKE, 0, FAKE, FAKE, n) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_expert_ffn_blocks(d, w, FAKE, 1000, FAKE, 4, FAKE, FAKE, n - 1) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_expert_ffn_blocks(d, w, FAKE, -1, FAKE, 4, FAKE, FAKE, n) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_block_scaled_path_validates():
+    """routed = mxfp4_a8 needs the tiled weight scales and 32-byte aligned
+    codes; tiled scales on any other path are rejected; the size query and the
+    tiling and quantiser entries validate on the host."""
+    full = {f: FAKE for f in ("Wr", "bias", "Wdown", "Wup", "gamma", "Wg", "Wv", "Wo", "Wsg", "Wsv", "Wso")}
+    d8 = _dims(I=1024, routed="mxfp4_a8")
+    ws8 = moe.moe_workspace_size(d8)
+    assert ws8 > moe.moe_workspace_size(_dims(I=1024, routed="mxfp4"))  # + E4M3 h and the scale tiles
+    tiled = dict(Sgv_tiled=FAKE, So_tiled=FAKE)
+    call = lambda w: moe.moe_layer_forward(d8, moe.make_weights(**w), FAKE, FAKE, None, FAKE, ws8, 0)  # noqa: E731
+    assert call(full) == moe.MOE_ERR_INVALID_ARG                                  # no tiled scales
+    assert call({**full, **tiled, "So_tiled": FAKE + 8}) == moe.MOE_ERR_INVALID_ARG  # misaligned
+    assert call({**full, **tiled, "Wv": FAKE + 16}) == moe.MOE_ERR_INVALID_ARG       # codes not 32-byte aligned
+    dm = _dims(I=1024, routed="mxfp4")
+    wsm = moe.moe_workspace_size(dm)
+    wm = moe.make_weights(**{**full, "Sg": FAKE, "Sv": FAKE, "So": FAKE, **tiled})
+    assert moe.moe_layer_forward(dm, wm, FAKE, FAKE, None, FAKE, wsm, 0) == moe.MOE_ERR_INVALID_ARG
+    # sizes of the tiled scales equal those of the row-major ones
+    k3 = _dims(H=7168, L=3584, E=896, k=16, I=3072, routed="mxfp4_a8")
+    st, gu, dn = moe.moe_mx_tiled_scales_size(k3)
+    assert st == moe.MOE_OK and gu == 896 * 3072 * 3584 // 16 and dn == 896 * 3584 * 3072 // 32
+    assert moe.moe_mx_tiled_scales_size(_dims())[0] == moe.MOE_ERR_UNSUPPORTED
+    assert moe.moe_mx_tile_scales(k3, FAKE, None, FAKE, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_mx_tile_scales(k3, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    # the stand-alone quantiser
+    assert moe.moe_mx8_quantize(FAKE, 4, 48, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG   # K % 32
+    assert moe.moe_mx8_quantize(FAKE + 8, 4, 64, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_mx8_quantize(None, 4, 64, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_mx8_quantize(None, 0, 64, None, None, 0) == moe.MOE_OK               # nothing to do
+
+
+def test_structs_keep_their_tensors_alive():
+    """make_weights / make_aux / make_grads hold the tensors whose addresses
+    they carry, so a tensor built for the call is not freed (and its memory
+    reused) while the struct is in use."""
+    import gc
+    import weakref
+
+    import torch
+
+    for make, field in ((moe.make_weights, "Sgv_tiled"), (moe.make_aux, "u"), (moe.make_grads, "dx")):
+        t = torch.zeros(4)
+        ref = weakref.ref(t)
+        s = make(**{field: t})
+        del t
+        gc.collect()
+        assert ref() is not None
+        del s
+        gc.collect()
+        assert ref() is None

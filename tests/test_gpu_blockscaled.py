@@ -1,0 +1,175 @@
+"""Block-scaled routed experts (MXFP4 weights x MXFP8 inputs on tcgen05.mma
+kind::mxf8f6f4) against the oracle: the MXFP8 quantiser bit for bit, the
+weight-scale tiling index by index, the expert GEMMs and the whole layer to
+the stated bars.  The oracle quantises the same bf16 inputs by the same rule
+(OCP MX v1.0 MXFP8, E4M3 with the shared-scale rule), so the device and the
+oracle multiply the same numbers; the bars cover accumulation order only."""
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+import sparse_moe_layer_renormalised_b200 as moe
+from harness import TOL_MXFP4_A8, compare_layer, dims_for, make_device_layer, parity, run_layer
+from oracle import inputs as oin
+from sparse_moe_layer_renormalised_b200.layer import tile_weight_scales
+
+pytestmark = pytest.mark.gpu
+F64 = torch.float64
+
+
+def _no_fault():
+    st, code = moe.moe_device_error()
+    assert st == moe.MOE_OK and code == 0, f"device fault {code}"
+
+
+def _quantiser_input(rows: int, K: int, seed: int) -> torch.Tensor:
+    """bf16 rows whose 32-blocks span many binades, with the quantiser's
+    special cases planted: an all-zero block (with a -0), a block whose
+    largest value saturates (1.9375 * 2^e -> 496 units -> 448), bf16
+    subnormals, and values near the bf16 maximum."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(rows, K, generator=g, dtype=torch.float64)
+    binade = torch.randint(-30, 30, (rows, K // 32, 1), generator=g).to(F64)
+    x = (x.reshape(rows, K // 32, 32) * torch.exp2(binade)).reshape(rows, K)
+    x[0, :32] = 0.0
+    x[0, 5] = -0.0
+    if K >= 64:
+        x[0, 32:64] = 0.25
+        x[0, 40] = -1.9375
+    if K >= 96:
+        x[0, 64:96] = torch.linspace(-3e-39, 3e-39, 32, dtype=F64)  # bf16 subnormals
+    if rows > 1 and K >= 64:
+        x[1, 32:64] = torch.linspace(-3.0e38, 3.0e38, 32, dtype=F64)
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (300, 1024), (1000, 3584), (129, 3072)])
+def test_mx8_quantize_bit_exact(rows, K):
+    x = _quantiser_input(rows, K, rows + K)
+    codes = torch.empty(rows, K, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(rows, K // 32, dtype=torch.uint8, device="cuda")
+    assert moe.moe_mx8_quantize(x.cuda(), rows, K, codes, scales) == moe.MOE_OK
+    torch.cuda.synchronize()
+    _no_fault()
+    ref_codes, ref_scales = oracle.mx8_quantize(x.to(F64))
+    got_c, got_s = codes.cpu().numpy(), scales.cpu().numpy()
+    assert np.array_equal(got_s, ref_scales), int((got_s != ref_scales).sum())
+    assert np.array_equal(got_c, ref_codes), int((got_c != ref_codes).sum())
+
+
+def test_mx8_quantize_rejects_bad_arguments():
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    c = torch.empty(4, 64, dtype=torch.uint8, device="cuda")
+    s = torch.empty(4, 2, dtype=torch.uint8, device="cuda")
+    assert moe.moe_mx8_quantize(x, 4, 48, c, s) == moe.MOE_ERR_INVALID_ARG  # K not a multiple of 32
+    assert moe.moe_mx8_quantize(None, 4, 64, c, s) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_mx8_quantize(x, 0, 64, None, None) == moe.MOE_OK
+
+
+def test_tile_scales_layout():
+    """moe_mx_tile_scales against a host re-indexing of the row-major scales by
+    the layout include/moe.h states (atom byte 16*(m%32) + 4*(m/32) + j)."""
+    cfg = gen.CONFIGS["mxfp4a8-small"]
+    d = dims_for(cfg)
+    w = gen.device_layer(cfg, "cuda", with_x=False)
+    t = tile_weight_scales(d, w["Sg"], w["Sv"], w["So"])
+    torch.cuda.synchronize()
+    E, I, L = cfg.E, cfg.I, cfg.L
+    Sg, Sv, So = (w[n].cpu().numpy() for n in ("Sg", "Sv", "So"))
+    j = np.arange(512)
+    m = (j >> 4) + 32 * ((j >> 2) & 3)
+    kb = j & 3
+    gu = t["Sgv_tiled"].cpu().numpy().reshape(E, I // 128, 2, L // 128, 512)
+    e, wt, c, ch, jj = np.meshgrid(np.arange(E), np.arange(I // 128), np.arange(2), np.arange(L // 128), j,
+                                   indexing="ij")
+    mm = m[jj]
+    row = wt * 128 + c * 64 + (mm % 64)
+    col = 4 * ch + kb[jj]
+    want = np.where(mm < 64, Sg[e, row, col], Sv[e, row, col])
+    assert np.array_equal(gu, want)
+    dn = t["So_tiled"].cpu().numpy().reshape(E, L // 256, 2, I // 128, 512)
+    e, wt, c, ch, jj = np.meshgrid(np.arange(E), np.arange(L // 256), np.arange(2), np.arange(I // 128), j,
+                                   indexing="ij")
+    assert np.array_equal(dn, So[e, wt * 256 + c * 128 + m[jj], 4 * ch + kb[jj]])
+
+
+def _routing(T, E, k, skew, seed):
+    g = torch.Generator().manual_seed(seed)
+    logits = torch.randn(T, E, generator=g)
+    if skew:  # a few experts take most tokens (several 240-row tiles each)
+        logits = logits + 3.0 * (torch.arange(E, dtype=torch.float32) + 1.0) ** -0.3
+    return torch.topk(logits, k, dim=1).indices.to(torch.int32)
+
+
+@pytest.mark.parametrize("T,skew", [(300, False), (40, False), (1024, True), (1, False)])
+def test_expert_ffn_a8(T, skew):
+    """Routed experts on the block-scaled path against the oracle, which
+    quantises the same bf16 rows (z, then h) and decodes the same weight bits.
+    The skewed case gives experts several token tiles; T = 1 a 16-wide MMA."""
+    cfg = gen.CONFIGS["mxfp4a8-small"].with_(T=T)
+    E, k, L = cfg.E, cfg.k, cfg.L
+    d = dims_for(cfg, T=T)
+    w = gen.device_layer(cfg, "cuda", with_x=False)
+    idx = _routing(T, E, k, skew, 31 + T)
+    counts, offsets, _, _ = oracle.permute(idx.numpy(), E)
+    R = T * k
+    z_perm = torch.randn(R, L, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    y_perm = torch.full((R, L), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(moe.moe_workspace_size(d), dtype=torch.uint8, device="cuda")
+    wts = moe.make_weights(Wg=w["Wg"], Wv=w["Wv"], Wo=w["Wo"], **tile_weight_scales(d, w["Sg"], w["Sv"], w["So"]))
+    off = torch.as_tensor(offsets, dtype=torch.int32).cuda()
+    assert moe.moe_expert_ffn(d, wts, z_perm.cuda(), off, y_perm, ws) == moe.MOE_OK
+    torch.cuda.synchronize()
+    _no_fault()
+    if skew:
+        assert int(np.max(counts)) > 2 * 240  # several tiles for the largest expert
+    zf = z_perm.to(F64)
+    ref = torch.empty(R, L, dtype=F64)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if a == b:
+            continue
+        Wg, Wv, Wo = oin.expert_weights(cfg, e)
+        ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wv, Wo, cfg.situ_c, oracle.bf16_round, act_mx8=True)
+    assert parity(y_perm.cpu().to(F64), ref) <= TOL_MXFP4_A8
+
+
+def test_a8_layer_all_tokens():
+    """The whole layer with block-scaled routed experts, every token against the oracle."""
+    cfg = gen.CONFIGS["mxfp4a8-small"]
+    layer, w = make_device_layer(cfg)
+    y, aux = run_layer(layer, w["x"])
+    m = compare_layer(cfg, np.arange(cfg.T), y, aux, TOL_MXFP4_A8)
+    print(f"\n[mxfp4a8-small] " + " ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}" for k, v in m.items()))
+
+
+def test_a8_layer_matches_mxfp4_up_to_activation_rounding():
+    """Same weights and selection: the block-scaled layer differs from the
+    bf16-activation MXFP4 layer by the MXFP8 rounding of the expert inputs,
+    a few per cent of rms (the oracle's own distance between the two, about
+    4% of rms(y) at this shape), not more."""
+    c8 = gen.CONFIGS["mxfp4a8-small"]
+    c4 = gen.CONFIGS["mxfp4-small"]
+    l8, w = make_device_layer(c8)
+    y8, _ = run_layer(l8, w["x"])
+    l4 = moe.MoeLayer(dims_for(c4), {k: v for k, v in w.items() if k != "x"})
+    y4, _ = run_layer(l4, w["x"])
+    d = (y8 - y4).double()
+    rel_rms = (d.pow(2).mean().sqrt() / y4.double().pow(2).mean().sqrt()).item()
+    assert 1e-3 < rel_rms < 0.1, rel_rms
+
+
+@pytest.mark.slow
+def test_k3_a8_sampled():
+    """K3 shape, block-scaled routed experts at the full T = 8192, seeded sample
+    of tokens against the oracle quantising and decoding the same bits."""
+    from harness import K3_SAMPLE
+
+    cfg = gen.CONFIGS["mxfp4-a8"]
+    layer, w = make_device_layer(cfg)
+    y, aux = run_layer(layer, w["x"])
+    tokens = gen.sample_tokens(cfg, min(K3_SAMPLE, cfg.T))
+    m = compare_layer(cfg, tokens, y, aux, TOL_MXFP4_A8)
+    print(f"\n[mxfp4-a8] " + " ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}" for k, v in m.items()))

@@ -16,6 +16,7 @@ import sparse_moe_layer_renormalised_b200 as moe
 from harness import TOL_BF16, dims_for, oracle_forward, parity
 from oracle import inputs as oin
 from sparse_moe_layer_renormalised_b200 import expert_parallel as ep
+from sparse_moe_layer_renormalised_b200.layer import tile_weight_scales
 
 pytestmark = pytest.mark.gpu
 F64 = torch.float64
@@ -26,7 +27,7 @@ def _no_fault():
     assert st == moe.MOE_OK and code == 0, f"device fault {code}"
 
 
-@pytest.mark.parametrize("name,lo,hi", [("mid", 40, 104), ("mxfp4-small", 0, 64)])
+@pytest.mark.parametrize("name,lo,hi", [("mid", 40, 104), ("mxfp4-small", 0, 64), ("mxfp4a8-small", 8, 40)])
 def test_expert_ffn_blocks_three_sources(name, lo, hi):
     """Rows of experts lo..hi-1 from three 'sources' (each expert-major), as
     an expert-parallel rank receives them; every row against the oracle."""
@@ -43,10 +44,13 @@ def test_expert_ffn_blocks_three_sources(name, lo, hi):
     offs = np.stack(blocks).astype(np.int32)
     expert_of_row = np.concatenate([np.repeat(np.arange(lo, hi), np.diff(b)) for b in blocks])
     x = torch.randn(rows, cfg.L, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
-    names = ("Wg", "Wv", "Wo") + (("Sg", "Sv", "So") if cfg.routed == "mxfp4" else ())
+    mx = cfg.routed in ("mxfp4", "mxfp4_a8")
+    names = ("Wg", "Wv", "Wo") + (("Sg", "Sv", "So") if mx else ())
     wl = {n: w[n][lo:hi].contiguous() for n in names}
     d = moe.Dims(T=rows, H=cfg.H, L=cfg.L, E=E_loc, k=1, I=cfg.I, S=cfg.S, Is=cfg.Is, act=cfg.act,
                  routed=cfg.routed)
+    if cfg.routed == "mxfp4_a8":
+        wl.update(tile_weight_scales(d, wl.pop("Sg"), wl.pop("Sv"), wl.pop("So")))
     ws = torch.empty(moe.moe_expert_ffn_blocks_workspace_size(d, rows, 3), dtype=torch.uint8, device="cuda")
     y = torch.full((rows, cfg.L), float("nan"), dtype=torch.float32, device="cuda")
     assert moe.moe_expert_ffn_blocks(d, moe.make_weights(**wl), x.cuda(), rows, torch.from_numpy(offs).cuda(), 3, y,
@@ -57,7 +61,8 @@ def test_expert_ffn_blocks_three_sources(name, lo, hi):
     xf = x.to(F64)
     for e in np.unique(expert_of_row):
         r = torch.as_tensor(np.nonzero(expert_of_row == e)[0])
-        ref[r] = oracle.expert_forward(xf[r], *oin.expert_weights_raw(cfg, int(e)), cfg.situ_c, oracle.bf16_round)
+        ref[r] = oracle.expert_forward(xf[r], *oin.expert_weights_raw(cfg, int(e)), cfg.situ_c, oracle.bf16_round,
+                                       act_mx8=cfg.routed == "mxfp4_a8")
     assert parity(y.cpu().to(F64), ref) <= 1e-2
 
 

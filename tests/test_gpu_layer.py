@@ -1,5 +1,4 @@
 """The whole layer through moe_layer_forward against the oracle (GPU)."""
-import os
 
 import numpy as np
 import pytest
@@ -7,7 +6,7 @@ import torch
 
 import gen
 import sparse_moe_layer_renormalised_b200 as moe
-from harness import (TOL_BF16, TOL_F32, TOL_MXFP4, compare_layer, make_device_layer, moe_inputs_rows, oracle_forward,
+from harness import (K3_SAMPLE, TOL_BF16, TOL_F32, TOL_MXFP4, compare_layer, make_device_layer, moe_inputs_rows, oracle_forward,
                      run_layer)
 
 pytestmark = pytest.mark.gpu
@@ -93,7 +92,6 @@ def test_zero_tokens_is_a_no_op(mid_layer):
     assert bool((y == 7.0).all())
 
 
-K3_SAMPLE = int(os.environ.get("MOE_K3_SAMPLE", "512"))
 
 
 @pytest.mark.slow
