@@ -18,12 +18,21 @@ F64 = torch.float64
 # Tolerances (max|y - y_ref| / rms(y_ref)) stated for the layer output.
 TOL_BF16 = 1e-2
 TOL_MXFP4 = 3e-2
-# Block-scaled path: the oracle quantises the same bf16 rows to MXFP8, so both
-# sides multiply the same numbers except where the device's bf16 z or h differs
-# from the oracle's by a rounding step and the E4M3 code of that element
-# changes (one code step is 1/16 - 1/8 of the element); the bar is the MXFP4
-# layer's.
+# Block-scaled path, expert GEMMs on the same bf16 input rows: both sides
+# quantise identical z rows to identical MXFP8 codes, so the error is that of
+# the MXFP4 layer (fp32 accumulation, bf16 h, and an E4M3 code of h flipping
+# where h itself differs by a bf16 step); bar 3e-2.
 TOL_MXFP4_A8 = 3e-2
+# The whole layer on that path: the device's bf16 z (fp32 sum) and the
+# oracle's (fp64 sum) differ by one bf16 step in some elements, and h too.
+# Where such a step (2^-8 relative) crosses an E4M3 rounding boundary (spaced
+# 2^-3 relative), about 1 in 32 of the differing elements, the quantised
+# element moves by a whole E4M3 step (1/16 to 1/8 of it).  A few such flips
+# per row of z and h change g and y by ~1% of rms, and the largest of some 10^6
+# outputs lands near 5 standard deviations: bars 1e-1 on max|d|/rms and 2e-2
+# on rms(d)/rms for y and u.
+TOL_MXFP4_A8_LAYER = 1e-1
+TOL_RMS_A8_LAYER = 2e-2
 TOL_F32 = 1e-4
 NEAR_TIE = 1e-4  # key margin below which an index-set difference is allowed
 # Router scores and mixture weights: fp32 on the device from the same bf16 (or
@@ -113,7 +122,13 @@ def oracle_forward(cfg, tokens, forced_idx=None) -> dict:
     return oracle.layer_forward_streamed(cfg, dense, x, lambda e: oin.expert_weights_raw(cfg, e), forced_idx=forced_idx)
 
 
-def compare_layer(cfg, tokens, y_gpu, aux, tol, ref=None) -> dict:
+def rms_parity(a: torch.Tensor, ref: torch.Tensor) -> float:
+    a = a.to(F64).cpu()
+    ref = ref.to(F64).cpu()
+    return float(torch.sqrt(((a - ref) ** 2).mean()) / torch.sqrt((ref * ref).mean()))
+
+
+def compare_layer(cfg, tokens, y_gpu, aux, tol, ref=None, rms_tol=None) -> dict:
     """Parity of the device layer on the sampled tokens against the oracle.
 
     Index sets must match except for tokens whose oracle key margin (k-th
@@ -173,6 +188,11 @@ def compare_layer(cfg, tokens, y_gpu, aux, tol, ref=None) -> dict:
         assert m["p_rel"] <= TOL_P_REL, f"p: max relative error {m['p_rel']:.3g} > {TOL_P_REL}"
     for key in ("y", "u"):
         assert m[key] <= tol, f"{key}: max|d|/rms = {m[key]:.3g} > {tol}"
+    if rms_tol is not None:
+        m["y_rms"] = rms_parity(y_gpu.cpu()[sel], y_ref)
+        m["u_rms"] = rms_parity(aux["u"].cpu()[sel], u_ref)
+        for key in ("y_rms", "u_rms"):
+            assert m[key] <= rms_tol, f"{key}: rms(d)/rms = {m[key]:.3g} > {rms_tol}"
     # The RMSNorm step: n must be RMSNorm of the device's own u, rounded to the
     # activation type, to within one rounding step of that type.  (Against the
     # oracle's n, per-token normalisation magnifies u's error in tokens whose

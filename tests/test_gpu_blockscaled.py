@@ -2,8 +2,10 @@
 kind::mxf8f6f4) against the oracle: the MXFP8 quantiser bit for bit, the
 weight-scale tiling index by index, the expert GEMMs and the whole layer to
 the stated bars.  The oracle quantises the same bf16 inputs by the same rule
-(OCP MX v1.0 MXFP8, E4M3 with the shared-scale rule), so the device and the
-oracle multiply the same numbers; the bars cover accumulation order only."""
+(OCP MX v1.0 MXFP8, E4M3 with the shared-scale rule): given the same input
+rows the expert GEMMs multiply the same numbers on both sides; in the whole
+layer the device's bf16 z and h can differ from the oracle's by a rounding
+step, which can flip an E4M3 code (bars derived in harness.py)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +13,8 @@ import torch
 import gen
 import oracle
 import sparse_moe_layer_renormalised_b200 as moe
-from harness import TOL_MXFP4_A8, compare_layer, dims_for, make_device_layer, parity, run_layer
+from harness import (TOL_MXFP4_A8, TOL_MXFP4_A8_LAYER, TOL_RMS_A8_LAYER, compare_layer, dims_for, make_device_layer,
+                     parity, run_layer)
 from oracle import inputs as oin
 from sparse_moe_layer_renormalised_b200.layer import tile_weight_scales
 
@@ -137,11 +140,13 @@ def test_expert_ffn_a8(T, skew):
 
 
 def test_a8_layer_all_tokens():
-    """The whole layer with block-scaled routed experts, every token against the oracle."""
+    """The whole layer with block-scaled routed experts, every token against
+    the oracle (bars derived in harness.py: the layer's bf16 z and h differ
+    from the oracle's by a rounding step, which can flip an E4M3 code)."""
     cfg = gen.CONFIGS["mxfp4a8-small"]
     layer, w = make_device_layer(cfg)
     y, aux = run_layer(layer, w["x"])
-    m = compare_layer(cfg, np.arange(cfg.T), y, aux, TOL_MXFP4_A8)
+    m = compare_layer(cfg, np.arange(cfg.T), y, aux, TOL_MXFP4_A8_LAYER, rms_tol=TOL_RMS_A8_LAYER)
     print(f"\n[mxfp4a8-small] " + " ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}" for k, v in m.items()))
 
 
@@ -171,5 +176,5 @@ def test_k3_a8_sampled():
     layer, w = make_device_layer(cfg)
     y, aux = run_layer(layer, w["x"])
     tokens = gen.sample_tokens(cfg, min(K3_SAMPLE, cfg.T))
-    m = compare_layer(cfg, tokens, y, aux, TOL_MXFP4_A8)
+    m = compare_layer(cfg, tokens, y, aux, TOL_MXFP4_A8_LAYER, rms_tol=TOL_RMS_A8_LAYER)
     print(f"\n[mxfp4-a8] " + " ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}" for k, v in m.items()))
