@@ -4,26 +4,33 @@
 //
 //   D[w, t] = sum_k (Wq[w, k] * 2^(sw[w, k/32] - 127)) * (Xq[t, k] * 2^(sx[t, k/32] - 127))
 //
-// Same work decomposition, operand swap and warp roles as gemm_expert.cuh
-// (weight rows are the MMA's M on a 2-CTA pair, M = 256; token rows its N;
-// warp 0 TMA producer, warp 1 TMEM owner and MMA issuer on the even CTA,
-// warps 2-5 epilogue), with these differences:
-//  * a stage covers K = 128: four MMAs of K = 32;
+// Same work decomposition and operand swap as gemm_expert.cuh (weight rows are
+// the MMA's M on a 2-CTA pair, M = 256; token rows its N), with these
+// differences:
+//  * a stage covers K = 256 (two 128-wide halves, 8 MMAs of K = 32).  The MMA
+//    issue is single-threaded and each barrier wait costs it a few hundred
+//    cycles (measured on B200: ~250 cycles per mbarrier check and ~50 per
+//    tcgen05 instruction, against 64 cycles of tensor time for an N = 128
+//    MMA at the fp8 rate), so one wait and one commit per 8 MMAs;
 //  * the weight tile is loaded from the packed E2M1 codes with the TMA type
 //    that spreads 16 codes over 16 bytes of shared memory (8 bytes of codes,
 //    8 bytes of gap), the operand layout this MMA kind reads for 4-bit types;
 //    its completion count is the packed size (64 bytes per row);
 //  * the activation tile is E4M3 codes, one byte each;
-//  * per stage both CTAs also load their weight rows' scale atom (512 bytes)
-//    and the whole token tile's scale atoms (two, 1 KB: each CTA's half of the
-//    accumulator needs the scales of every token column); the MMA thread
-//    copies them to tensor memory with tcgen05.cp (cta_group::2: each CTA
-//    from its own shared memory) ahead of the stage's MMAs.  tcgen05.cp and
-//    tcgen05.mma from one thread execute in issue order, so one scale region
-//    serves every stage;
-//  * token tiles hold at most 240 rows, so two accumulators (2 x 240 fp32
-//    columns) and the scale columns (12) fit the 512 columns of tensor memory.
-// Every wait is bounded.
+//  * per stage both CTAs also load their weight rows' scale atoms (1 KB) and
+//    the whole token tile's scale atoms (2 KB: each CTA's half of the
+//    accumulator needs the scales of every token column).  A copier warp (warp
+//    6 of the even CTA) moves them to tensor memory with tcgen05.cp
+//    (cta_group::2: each CTA from its own shared memory) into one of three scale
+//    buffers and commits to the stage's scale barrier, on which the MMA thread
+//    waits instead of the data barrier; so the MMA thread issues MMAs only;
+//  * token tiles hold at most 208 rows, so two accumulators (2 x 208 fp32
+//    columns) and three scale buffers (3 x 24) fit the 512 columns of tensor
+//    memory; with three, the copier can put stage g's scales in the tensor
+//    pipe's queue ahead of stage g-1's MMAs.
+// Warp roles: 0 TMA producer (both CTAs), 1 TMEM owner and MMA issuer (even
+// CTA), 2-5 epilogue (both CTAs), 6 scale copier (even CTA).  Every wait is
+// bounded.
 #pragma once
 
 #include "gemm_expert.cuh"
@@ -31,28 +38,32 @@
 
 namespace moe {
 
-constexpr int BS_BK = 128;                         // K elements per stage: 4 MMAs of K = 32
-constexpr uint32_t BS_A_BYTES = 128 * BS_BK;       // 128 weight rows, one byte slot per E2M1 code
+constexpr int BS_BK = 256;                         // K elements per stage: two halves of 128, 8 MMAs of K = 32
+constexpr uint32_t BS_HALF_BYTES = 128 * 128;      // a 128-row x 128-element half tile (one byte per code slot)
+constexpr uint32_t BS_A_BYTES = 2 * BS_HALF_BYTES;  // 128 weight rows
 constexpr uint32_t BS_A_TX = 128 * BS_BK / 2;      // bytes the A tile's TMA completes (packed codes)
-constexpr uint32_t BS_B_BYTES = 128 * BS_BK;       // up to 128 token rows of E4M3 codes per CTA
-constexpr uint32_t BS_SFA_BYTES = 512;             // scale atom: 128 weight rows x 4 k-blocks
-constexpr uint32_t BS_SFB_BYTES = 1024;            // token rows 0-127 and 128-255
-constexpr int BS_STAGES = 6;
-constexpr int BS_MAX_TILE_ROWS = 240;              // largest token tile (MMA N)
+constexpr uint32_t BS_B_BYTES = 2 * BS_HALF_BYTES;  // up to 128 token rows of E4M3 codes per CTA
+constexpr uint32_t BS_SFA_BYTES = 1024;            // two scale atoms (128 weight rows x 4 k-blocks each)
+constexpr uint32_t BS_SFB_BYTES = 2048;            // two K halves x (token rows 0-127, 128-255)
+constexpr int BS_STAGES = 3;
+constexpr int BS_MAX_TILE_ROWS = 208;              // largest token tile (MMA N)
 constexpr uint32_t BS_ACC_COLS = BS_MAX_TILE_ROWS;
-constexpr uint32_t BS_SF_COL = 2 * BS_ACC_COLS;    // SFA in columns 480-483, SFB in 484-491
-constexpr int BS_THREADS = 192;
+constexpr uint32_t BS_SF_COL = 2 * BS_ACC_COLS;    // three scale buffers of 24 columns from here
+constexpr int BS_SF_BUFS = 3;
+constexpr uint32_t BS_SF_BUF_COLS = 24;            // SFA half 0 / 1 at +0 / +4, SFB half 0 / 1 at +8 / +16
+constexpr int BS_THREADS = 224;
+constexpr int BS_COPY_WARP = 6;
 constexpr uint32_t BS_STAGE_BYTES = BS_A_BYTES + BS_B_BYTES + BS_SFA_BYTES + BS_SFB_BYTES;
 constexpr size_t BS_SMEM = 1024 + static_cast<size_t>(BS_STAGES) * BS_STAGE_BYTES + EX_XCH_BYTES + 512;
-static_assert(BS_SF_COL + 12 <= 2 * EX_ACC_COLS, "tensor memory columns");
+static_assert(BS_SF_COL + BS_SF_BUFS * BS_SF_BUF_COLS <= 2 * EX_ACC_COLS, "tensor memory columns");
 static_assert(BS_SMEM <= 232448, "shared memory per CTA");
 
 struct BsMaps {
   CUtensorMap a0;    // E2M1 codes, 16 per 16-byte slot: PAIRED W_g [E*I, L] (64-row boxes), else W_o [E*L, I] (128-row)
   CUtensorMap a1;    // PAIRED: W_v, as a0
-  CUtensorMap sa;    // weight scale tiles as [n, 16] bytes, 32-row (512-byte) boxes
+  CUtensorMap sa;    // weight scale tiles as [n, 16] bytes, 64-row (two atoms, 1 KB) boxes
   CUtensorMap b[4];  // E4M3 activation codes [R, K]: 128-byte wide boxes of 128, 64, 32, 16 rows, 128-byte swizzle
-  CUtensorMap sb[2]; // activation scale tiles as [n, 16] bytes: 64-row (both atoms) and 32-row boxes
+  CUtensorMap sb;    // activation scale tiles as [n, 16] bytes, 128-row (two K chunks x two atoms, 2 KB) boxes
 };
 
 // Shared-memory descriptor of a scale atom for tcgen05.cp: 32 rows of 16
@@ -142,10 +153,12 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   float* xch = reinterpret_cast<float*>(sSB + BS_STAGES * BS_SFB_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + EX_XCH_BYTES);
   uint64_t* empty = full + BS_STAGES;
-  uint64_t* acc_full = empty + BS_STAGES;
+  uint64_t* sf_full = empty + BS_STAGES;  // the stage's scales are in tensor memory (even CTA)
+  uint64_t* acc_full = sf_full + BS_STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* copy_drain = drain + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(copy_drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_ok = abort + 1;
 
@@ -160,12 +173,14 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
     for (int s = 0; s < BS_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 4 * CG);
     }
     mbar_init(drain, 1);
+    mbar_init(copy_drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -174,8 +189,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
     if (PAIRED) tma_prefetch_desc(&maps.a1);
     tma_prefetch_desc(&maps.sa);
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&maps.b[i]);
-    tma_prefetch_desc(&maps.sb[0]);
-    tma_prefetch_desc(&maps.sb[1]);
+    tma_prefetch_desc(&maps.sb);
   }
   if (warp == 1) ex_tmem_alloc<CG>(tmem_holder);
   tc_fence_before();
@@ -186,6 +200,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   const int num_tiles = p.num_tiles_dev[0];
   const int num_multi = p.num_tiles_dev[1];
   const int total = num_tiles * p.n_wtiles;
+  const int n_stages = p.num_k_blocks;  // stages of K = 256 per item
+  const int nkb128 = 2 * p.num_k_blocks;  // 128-wide K chunks per row (scale-tile indexing)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (both CTAs)
@@ -201,32 +217,36 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
         const int bsel = rows_cta > 64 ? 0 : rows_cta > 32 ? 1 : rows_cta > 16 ? 2 : 3;
         const int brows = 128 >> bsel;
         const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
-        const bool two_atoms = t.n_mma > 128;
-        const uint32_t bytes = static_cast<uint32_t>(CG) * (BS_A_TX + static_cast<uint32_t>(brows) * BS_BK +
-                                                            BS_SFA_BYTES + (two_atoms ? 1024u : 512u));
+        const uint32_t bytes = static_cast<uint32_t>(CG) * (BS_A_TX + 2u * static_cast<uint32_t>(brows) * 128u +
+                                                            BS_SFA_BYTES + BS_SFB_BYTES);
         const int wrow = t.expert * p.w_rows_per_expert + (PAIRED ? t.wt * 128 : t.wt * 256) +
                          static_cast<int>(rank) * (PAIRED ? 64 : 128);
         // 16-byte rows of the scale tiles: 32 per atom
-        const int sa_row0 = ((t.expert * p.n_wtiles + t.wt) * 2 + static_cast<int>(rank)) * p.num_k_blocks * 32;
-        const int sb_row0 = t.tt * p.num_k_blocks * 64;
-        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        const int sa_row0 = ((t.expert * p.n_wtiles + t.wt) * 2 + static_cast<int>(rank)) * nkb128 * 32;
+        const int sb_row0 = t.tt * nkb128 * 64;
+        for (int kb = 0; kb < n_stages; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort, p.fault_site + 1)) {
             ok = false;
             break;
           }
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-          const int kc = kb * BS_BK;
           uint8_t* a_dst = sA + stage * BS_A_BYTES;
-          if (kExL2Hints && !t.multi) {
-            ex_tma_load_hint<CG>(a_dst, &maps.a0, &full[stage], kc, wrow, pol_w);
-            if (PAIRED) ex_tma_load_hint<CG>(a_dst + BS_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
-          } else {
-            ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
-            if (PAIRED) ex_tma_load<CG>(a_dst + BS_A_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
+          uint8_t* b_dst = sB + stage * BS_B_BYTES;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kc = kb * BS_BK + h * 128;
+            uint8_t* ah = a_dst + h * BS_HALF_BYTES;
+            if (kExL2Hints && !t.multi) {
+              ex_tma_load_hint<CG>(ah, &maps.a0, &full[stage], kc, wrow, pol_w);
+              if (PAIRED) ex_tma_load_hint<CG>(ah + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
+            } else {
+              ex_tma_load<CG>(ah, &maps.a0, &full[stage], kc, wrow);
+              if (PAIRED) ex_tma_load<CG>(ah + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
+            }
+            ex_tma_load_hint<CG>(b_dst + h * BS_HALF_BYTES, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
           }
-          ex_tma_load<CG>(sSA + stage * BS_SFA_BYTES, &maps.sa, &full[stage], 0, sa_row0 + kb * 32);
-          ex_tma_load_hint<CG>(sB + stage * BS_B_BYTES, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
-          ex_tma_load<CG>(sSB + stage * BS_SFB_BYTES, &maps.sb[two_atoms ? 0 : 1], &full[stage], 0, sb_row0 + kb * 64);
+          ex_tma_load<CG>(sSA + stage * BS_SFA_BYTES, &maps.sa, &full[stage], 0, sa_row0 + kb * 64);
+          ex_tma_load<CG>(sSB + stage * BS_SFB_BYTES, &maps.sb, &full[stage], 0, sb_row0 + kb * 128);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == BS_STAGES) {
@@ -248,32 +268,37 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
     if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t g = 0;  // stages consumed so far
+      uint32_t sf_buf = 0;  // scale buffer of stage g (g mod BS_SF_BUFS)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const uint32_t sf_a = tmem_base + BS_SF_COL, sf_b = sf_a + 4u;
       for (int w = pair; w < total && ok; w += npairs) {
         const ExTile t = bs_decode(w, num_tiles, num_multi, p, false);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort, p.fault_site + 3)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * BS_ACC_COLS;
-        for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort, p.fault_site + 4)) {
+        const uint32_t idesc0 = idesc_mxf4_mxf8(256, t.n_mma, 0);
+        for (int kb = 0; kb < n_stages; ++kb, ++g) {
+          if (!mbar_wait(&sf_full[stage], phase, abort, p.fault_site + 4)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          bs_copy_sf(sf_a, sf_atom_desc(smem_u32(sSA + stage * BS_SFA_BYTES)));
-          bs_copy_sf(sf_b, sf_atom_desc(smem_u32(sSB + stage * BS_SFB_BYTES)));
-          if (t.n_mma > 128) bs_copy_sf(sf_b + 4u, sf_atom_desc(smem_u32(sSB + stage * BS_SFB_BYTES + 512)));
+          const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * BS_SF_BUF_COLS;
+          if (++sf_buf == BS_SF_BUFS) sf_buf = 0;
           const uint32_t a_addr = smem_u32(sA + stage * BS_A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * BS_B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BS_BK / 32; ++kk) {
-            const uint32_t j = static_cast<uint32_t>(kk) << 30;  // scale byte of this K = 32 step
-            bs_mma(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
-                   idesc_mxf4_mxf8(256, t.n_mma, kk), sf_a | j, sf_b | j, (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t j = static_cast<uint32_t>(kk);  // scale byte of this K = 32 step
+              const uint32_t id = idesc0 | (j << 4) | (j << 29);
+              bs_mma(d_tmem, sw128_kmajor_desc(a_addr + h * BS_HALF_BYTES + kk * 32),
+                     sw128_kmajor_desc(b_addr + h * BS_HALF_BYTES + kk * 32), id, (sf + 4u * h) | (j << 30),
+                     (sf + 8u + 8u * h) | (j << 30), (kb | h | kk) != 0 ? 1u : 0u);
+            }
           ex_commit<CG>(&empty[stage]);
           if (++stage == BS_STAGES) {
             stage = 0;
@@ -289,10 +314,66 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
       }
       ex_commit<CG>(drain);
     }
-    // Both CTAs: every MMA and copy touching this CTA's shared memory or TMEM is done.
+    // Both CTAs: every MMA touching this CTA's shared memory or TMEM is done.
     if (lane == 0) {
       volatile int never = 0;
       mbar_wait(drain, 0u, &never, p.fault_site + 5);
+    }
+    __syncwarp();
+  } else if (warp == BS_COPY_WARP) {
+    // ------------------------------------------------------------------ scale copier (even CTA)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t g = 0;
+      int prev2_stage = 0;        // stage of g - BS_SF_BUFS (its MMAs used the same scale buffer)
+      uint32_t prev2_phase = 0;
+      uint32_t sf_buf = 0;
+      bool ok = true;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const ExTile t = bs_decode(w, num_tiles, num_multi, p, false);
+        const bool two_atoms = t.n_mma > 128;
+        for (int kb = 0; kb < n_stages; ++kb, ++g) {
+          if (!mbar_wait(&full[stage], phase, abort, p.fault_site + 7)) {
+            ok = false;
+            break;
+          }
+          if (g >= static_cast<uint32_t>(BS_SF_BUFS)) {
+            if (!mbar_wait(&empty[prev2_stage], prev2_phase, abort, p.fault_site + 8)) {
+              ok = false;
+              break;
+            }
+            if (++prev2_stage == BS_STAGES) {
+              prev2_stage = 0;
+              prev2_phase ^= 1u;
+            }
+          }
+          tc_fence_after();
+          const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * BS_SF_BUF_COLS;
+          if (++sf_buf == BS_SF_BUFS) sf_buf = 0;
+          const uint8_t* sa = sSA + stage * BS_SFA_BYTES;
+          const uint8_t* sb = sSB + stage * BS_SFB_BYTES;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            bs_copy_sf(sf + 4u * h, sf_atom_desc(smem_u32(sa + h * 512)));
+            bs_copy_sf(sf + 8u + 8u * h, sf_atom_desc(smem_u32(sb + h * 1024)));
+            if (two_atoms) bs_copy_sf(sf + 12u + 8u * h, sf_atom_desc(smem_u32(sb + h * 1024 + 512)));
+          }
+          // the MMA thread waits on this instead of full[]: data and scales are in place
+          asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           smem_u32(&sf_full[stage]))
+                       : "memory");
+          if (++stage == BS_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(copy_drain))
+                   : "memory");
+      volatile int never = 0;
+      mbar_wait(copy_drain, 0u, &never, p.fault_site + 9);
     }
     __syncwarp();
   } else {

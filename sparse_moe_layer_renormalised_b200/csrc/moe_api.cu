@@ -736,14 +736,16 @@ moe_status stage_expert_bs(const moe_dims& d, bool paired, const moe_weights& w,
   const uint64_t wrows = static_cast<uint64_t>(d.E) * out_rows;
   const size_t sa_bytes = paired ? tiled_scales_gate_up(d) : tiled_scales_down(d);
   bool ok = true;
+  // scale tiles as 16-byte rows: weight boxes of two atoms (two 128-wide K
+  // chunks, 1 KB), activation boxes of two chunks x two atoms (2 KB)
   if (paired)
     ok = make_map_e2m1(&maps.a0, w.Wg, wrows, K, 64) && make_map_e2m1(&maps.a1, w.Wv, wrows, K, 64) &&
-         make_map_u8(&maps.sa, w.Sgv_tiled, sa_bytes / 16, 16, 16, 32);
+         make_map_u8(&maps.sa, w.Sgv_tiled, sa_bytes / 16, 16, 16, 64);
   else
-    ok = make_map_e2m1(&maps.a0, w.Wo, wrows, K, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, 32);
+    ok = make_map_e2m1(&maps.a0, w.Wo, wrows, K, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, 64);
   for (int i = 0; i < 4 && ok; ++i) ok = make_map_u8_sw128(&maps.b[i], act_q, static_cast<uint64_t>(R), K, 128u >> i);
   const uint64_t sf_rows = static_cast<uint64_t>(max_tiles) * (K / 128) * 64;
-  ok = ok && make_map_u8(&maps.sb[0], act_sf, sf_rows, 16, 16, 64) && make_map_u8(&maps.sb[1], act_sf, sf_rows, 16, 16, 32);
+  ok = ok && make_map_u8(&maps.sb, act_sf, sf_rows, 16, 16, 128);
   if (!ok) return MOE_ERR_CUDA;
   ExParams p{};
   p.tile_table = table;
