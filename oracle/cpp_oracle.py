@@ -36,7 +36,7 @@ class oc_dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("L", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("S", ctypes.c_int32), ("Is", ctypes.c_int32),
                 ("situ_c", ctypes.c_double), ("rms_eps", ctypes.c_double), ("mode", ctypes.c_int32),
-                ("routed_act_mx8", ctypes.c_int32)]
+                ("routed_act", ctypes.c_int32)]
 
 
 class oc_weights(ctypes.Structure):
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.oc_e4m3_decode.argtypes = [vp, i64, vp]
         L.oc_e4m3_encode.argtypes = [vp, i64, vp]
         L.oc_mx8_quantize.argtypes = [vp, i64, i64, vp, vp]
+        L.oc_e2m1_encode.argtypes = [vp, i64, vp]
+        L.oc_mx4_quantize.argtypes = [vp, i64, i64, vp, vp]
         L.oc_combine.argtypes = [vp, vp, i64, i64, i64, vp]
         L.oc_rms_norm.argtypes = [vp, vp, i64, i64, f64, vp]
         L.oc_shared_experts.argtypes = [vp, i64, i64, i64, i64, pm, pm, pm, f64, i32, vp]
@@ -180,6 +182,7 @@ def f32_to_f64(a) -> torch.Tensor:
 
 
 E2M1_VALUES = _py.E2M1_VALUES
+routed_act = _py.routed_act  # a name mapping, no arithmetic
 
 
 def mxfp4_dequant(codes, scales) -> torch.Tensor:
@@ -257,21 +260,24 @@ def _linear(a: torch.Tensor, W) -> torch.Tensor:
     return out
 
 
-def expert_forward(z_rows: torch.Tensor, Wg, Wv, Wo, c: float, rnd, act_mx8: bool = False):
+_ACT_CODE = {None: 0, "mxfp8": 1, "mxfp4": 2}
+
+
+def expert_forward(z_rows: torch.Tensor, Wg, Wv, Wo, c: float, rnd, act: str | None = None):
     """g = W_g z, v = W_v z, h = rnd(SiTU-GLU(g, v)), y = W_o h (fp64); with
-    act_mx8 the rows of z and of h (after rnd) are first replaced by their
-    MXFP8 values."""
+    act ("mxfp8" / "mxfp4") the rows of z and of h (after rnd) are first
+    replaced by their values in that format."""
     mode = _mode_of(rnd)
     if mode is None:  # a caller-supplied rounding function: the same steps, one call each
-        zq = mx8_round(z_rows) if act_mx8 else z_rows
+        zq = act_round(act, z_rows)
         h = rnd(situ_glu(_linear(zq, Wg), _linear(zq, Wv), c))
-        return _linear(mx8_round(h) if act_mx8 else h, Wo)
+        return _linear(act_round(act, h), Wo)
     z = _f64(z_rows)
     keep: list = []
     mg, mv, mo = _mat(Wg, keep), _mat(Wv, keep), _mat(Wo, keep)
     y = torch.empty(z.shape[0], mo.rows, dtype=F64)
     lib().oc_expert_forward(_ptr(z), z.shape[0], z.shape[1], ctypes.byref(mg), ctypes.byref(mv), ctypes.byref(mo),
-                            float(c), mode, 1 if act_mx8 else 0, _ptr(y))
+                            float(c), mode, _ACT_CODE[act], _ptr(y))
     return y
 
 
@@ -306,6 +312,37 @@ def mx8_round(v) -> torch.Tensor:
     """The values of the MXFP8 encoding of rows v [R, K] (fp64)."""
     codes, scales = mx8_quantize(v)
     return mx8_dequant(codes, scales)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    """fp64 values -> nearest E2M1 codes, one per byte (ties to even,
+    saturating to +-6)."""
+    v = _f64(v)
+    out = np.empty(tuple(v.shape), dtype=np.uint8)
+    lib().oc_e2m1_encode(_ptr(v), v.numel(), out.ctypes.data)
+    return out
+
+
+def mx4_quantize(v) -> tuple[np.ndarray, np.ndarray]:
+    """Rows of fp64 values [R, K] -> MXFP4 (packed codes [R, K/2] uint8, E8M0
+    scale bytes [R, K/32] uint8)."""
+    v = _f64(v)
+    R, K = v.shape
+    codes = np.empty((R, K // 2), dtype=np.uint8)
+    scales = np.empty((R, K // 32), dtype=np.uint8)
+    lib().oc_mx4_quantize(_ptr(v), R, K, codes.ctypes.data, scales.ctypes.data)
+    return codes, scales
+
+
+def mx4_round(v) -> torch.Tensor:
+    """The values of the MXFP4 encoding of rows v [R, K] (fp64)."""
+    return mxfp4_dequant(*mx4_quantize(v))
+
+
+def act_round(act: str | None, v) -> torch.Tensor:
+    if act is None:
+        return v
+    return {"mxfp8": mx8_round, "mxfp4": mx4_round}[act](v)
 
 
 def mx8_dequant(codes, scales) -> torch.Tensor:
@@ -356,7 +393,7 @@ def _run_layer(cfg, dense: dict, x: torch.Tensor, routed, forced_idx) -> dict:
     keep: list = []
     mode = {"bf16": ROUND_BF16, "f32": ROUND_F32}[cfg.act]
     d = oc_dims(T, cfg.H, cfg.L, cfg.E, cfg.k, cfg.I, cfg.S, cfg.Is, float(cfg.situ_c), float(cfg.rms_eps), mode,
-                1 if getattr(cfg, "routed", None) == "mxfp4_a8" else 0)
+                _ACT_CODE[routed_act(cfg)])
     bias, gamma = _f64(dense["bias"]), _f64(dense["gamma"])
     keep += [bias, gamma]
     shared = [_mat(dense[n], keep) if cfg.S > 0 else _empty_mat() for n in ("Wsg", "Wsv", "Wso")]

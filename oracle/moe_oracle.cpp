@@ -22,8 +22,8 @@
 //     「MXFP4 Quantization-Aware Training」": routed weights served in MXFP4
 //     (format fixed by the OCP Microscaling Formats specification v1.0).
 //     The pages give no activation format; where the routed experts take
-//     MXFP8 inputs (the block-scaled variant) the library's reading is the
-//     same specification's MXFP8 E4M3 with its shared-scale rule (below).
+//     MXFP8 or MXFP4 inputs (the block-scaled variants) the library's reading
+//     is the same specification's formats with their shared-scale rule (below).
 //
 // Readings where the pages are silent (the same in the GPU library):
 //  * SiTU-GLU(g, v) = sigmoid(g) * c*tanh(g/c) * c*tanh(v/c), c = 10;
@@ -189,6 +189,75 @@ void mx8_round_row(const double* v, int64_t K, double* out) {
   for (int64_t k = 0; k < K; ++k) out[k] = e4m3_value(c[k]) * e8m0_value(sc[k / 32]);
 }
 
+// Nearest E2M1 code to v (OCP MX v1.0 FP4 E2M1: sign bit 3, exponent bits 2-1
+// with bias 1, mantissa bit 0; values 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the
+// even code, magnitudes past 6 saturated to 6; the sign of v (of -0 too) kept.
+// Between 2^q and 2^(q+1) (q >= 0) the E2M1 numbers are spaced 2^(q-1); below
+// 2 the spacing is 0.5 (0.5 is the subnormal), so a / spacing is rounded to the
+// nearest even integer (rint) and read back as exponent and mantissa.
+uint8_t e2m1_encode(double v) {
+  const uint8_t sign = std::signbit(v) ? 0x8u : 0u;
+  const double a = std::fabs(v);
+  if (a >= 6.0) return sign | 0x7u;
+  if (a == 0.0) return sign;
+  int e2 = 0;
+  std::frexp(a, &e2);                        // a in [2^(e2-1), 2^e2)
+  int q = std::max(e2 - 1, 0);
+  int units = static_cast<int>(std::rint(std::ldexp(a, 1 - q)));  // a / 2^(q-1)
+  if (q == 0) return sign | static_cast<uint8_t>(units);  // 0 .. 4: codes 0 .. 4 (4 = 2.0)
+  if (units == 4) {                           // carry into the next binade
+    ++q;
+    units = 2;
+  }
+  return sign | static_cast<uint8_t>(((q + 1) << 1) | (units - 2));
+}
+
+// OCP MX v1.0 shared scale of an MXFP4 block: s = floor(log2(max |v|)) - 2 (2 =
+// the largest E2M1 exponent), clamped to [-127, 127]; an all-zero block -127.
+int mx4_block_exponent(const double* v, int64_t n) {
+  double amax = 0.0;
+  for (int64_t i = 0; i < n; ++i) amax = std::max(amax, std::fabs(v[i]));
+  if (amax == 0.0) return -127;
+  int e2 = 0;
+  std::frexp(amax, &e2);
+  return std::max(-127, std::min(127, e2 - 1 - 2));
+}
+
+// One row of K values -> packed E2M1 codes [K/2] (element 2i in the low
+// nibble) and E8M0 scale bytes [K/32].
+void mx4_quantize_row(const double* v, int64_t K, uint8_t* codes, uint8_t* scales) {
+  for (int64_t b = 0; b < K / 32; ++b) {
+    const int s = mx4_block_exponent(v + 32 * b, 32);
+    scales[b] = static_cast<uint8_t>(s + 127);
+    for (int64_t i = 0; i < 32; i += 2) {
+      const uint8_t lo = e2m1_encode(std::ldexp(v[32 * b + i], -s));
+      const uint8_t hi = e2m1_encode(std::ldexp(v[32 * b + i + 1], -s));
+      codes[(32 * b + i) / 2] = static_cast<uint8_t>(lo | (hi << 4));
+    }
+  }
+}
+
+// The values the MXFP4 encoding of a row stands for.
+void mx4_round_row(const double* v, int64_t K, double* out) {
+  std::vector<uint8_t> c(static_cast<size_t>(K / 2)), sc(static_cast<size_t>(K / 32));
+  mx4_quantize_row(v, K, c.data(), sc.data());
+  for (int64_t k = 0; k < K; ++k) {
+    const unsigned code = (k & 1) ? (c[k / 2] >> 4) : (c[k / 2] & 0xFu);
+    out[k] = e2m1_value(code) * e8m0_value(sc[k / 32]);
+  }
+}
+
+// Rounds a row of the expert's GEMM inputs to the activation format of the
+// routed type: 0 none, 1 MXFP8, 2 MXFP4.
+void act_round_row(int act, const double* v, int64_t K, double* out) {
+  if (act == 1)
+    mx8_round_row(v, K, out);
+  else if (act == 2)
+    mx4_round_row(v, K, out);
+  else
+    std::memcpy(out, v, sizeof(double) * K);
+}
+
 double sigmoid(double t) { return 1.0 / (1.0 + std::exp(-t)); }
 
 double situ_glu(double g, double v, double c) {
@@ -301,25 +370,26 @@ void linear(const double* a, int64_t R, int64_t K, const oc_mat& W, double* out)
 
 // y[n, L] = W_o SiTU-GLU(W_g z, W_v z), h stored with `mode` ([K3-896]
 // "K3のエキスパートは896個の小型LLMではない"; SiTU-GLU from [K3-report]).
-// act_mx8: the expert's two GEMM inputs (the rows of z, and h after its
-// storage rounding) are first replaced row by row by their MXFP8 values.
+// act (the routed experts' input format: 0 as stored, 1 MXFP8, 2 MXFP4): the
+// expert's two GEMM inputs (the rows of z, and h after its storage rounding)
+// are first replaced row by row by their values in that format.
 void expert(const double* z, int64_t n, int64_t L, const oc_mat& Wg, const oc_mat& Wv, const oc_mat& Wo, double c,
-            int mode, int act_mx8, double* y) {
+            int mode, int act, double* y) {
   const int64_t I = Wg.rows;
   std::vector<double> zq;
-  if (act_mx8) {
+  if (act != 0) {
     zq.resize(static_cast<size_t>(n * L));
-    for (int64_t r = 0; r < n; ++r) mx8_round_row(z + r * L, L, &zq[r * L]);
+    for (int64_t r = 0; r < n; ++r) act_round_row(act, z + r * L, L, &zq[r * L]);
     z = zq.data();
   }
   std::vector<double> g(static_cast<size_t>(n * I)), v(static_cast<size_t>(n * I));
   linear(z, n, L, Wg, g.data());
   linear(z, n, L, Wv, v.data());
   for (int64_t i = 0; i < n * I; ++i) g[i] = store(situ_glu(g[i], v[i], c), mode);
-  if (act_mx8)
+  if (act != 0)
     for (int64_t r = 0; r < n; ++r) {
       std::vector<double> row(g.begin() + r * I, g.begin() + (r + 1) * I);
-      mx8_round_row(row.data(), I, &g[r * I]);
+      act_round_row(act, row.data(), I, &g[r * I]);
     }
   linear(g.data(), n, I, Wo, y);
 }
@@ -432,8 +502,18 @@ int oc_permute(const int64_t* idx, int64_t T, int64_t k, int64_t E, int64_t* cou
 }
 
 void oc_expert_forward(const double* z, int64_t n, int64_t L, const oc_mat* Wg, const oc_mat* Wv, const oc_mat* Wo,
-                       double c, int mode, int act_mx8, double* y) {
-  expert(z, n, L, *Wg, *Wv, *Wo, c, mode, act_mx8, y);
+                       double c, int mode, int act, double* y) {
+  expert(z, n, L, *Wg, *Wv, *Wo, c, mode, act, y);
+}
+
+// E2M1 codes (one per byte, low nibble) <-> values; rows of values -> packed
+// MXFP4 codes [rows, K/2] and E8M0 scale bytes [rows, K/32].
+void oc_e2m1_encode(const double* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e2m1_encode(v[i]);
+}
+
+void oc_mx4_quantize(const double* v, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales) {
+  for (int64_t r = 0; r < rows; ++r) mx4_quantize_row(v + r * K, K, codes + r * (K / 2), scales + r * (K / 32));
 }
 
 // E4M3 codes -> values; values -> nearest E4M3 codes (ties to even,
@@ -492,7 +572,7 @@ typedef struct {
   int32_t H, L, E, k, I, S, Is;
   double situ_c, rms_eps;
   int32_t mode;  // storage rounding of z, h, shared h, n
-  int32_t routed_act_mx8;  // 1: the routed experts take MXFP8 inputs (block-scaled variant)
+  int32_t routed_act;  // the routed experts' input format: 0 as stored, 1 MXFP8, 2 MXFP4 (block-scaled variants)
 } oc_dims;
 
 typedef struct {
@@ -571,7 +651,7 @@ int oc_layer_forward(const oc_dims* d, const oc_weights* w, const double* x, con
     zr.assign(static_cast<size_t>(n * L), 0.0);
     yr.assign(static_cast<size_t>(n * L), 0.0);
     for (int64_t r = 0; r < n; ++r) std::memcpy(&zr[r * L], o->z + (pe[r] / k) * L, sizeof(double) * L);
-    expert(zr.data(), n, L, Wg, Wv, Wo, d->situ_c, d->mode, d->routed_act_mx8, yr.data());
+    expert(zr.data(), n, L, Wg, Wv, Wo, d->situ_c, d->mode, d->routed_act, yr.data());
     for (int64_t r = 0; r < n; ++r) std::memcpy(&y_slots[pe[r] * L], &yr[r * L], sizeof(double) * L);
   }
   oc_combine(y_slots.data(), o->p, T, k, L, o->u);

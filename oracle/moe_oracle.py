@@ -19,9 +19,9 @@ Sources (web pages; cited by title and section):
    non-linearity and puts smooth caps on both the linear and the up branch.
 [K3-QAT] ai-tech-express.jp article, section "量子化を前提とした学習「MXFP4
    Quantization-Aware Training」": routed weights are served in MXFP4.  The
-   pages name no activation format; for the block-scaled variant, whose routed
-   experts take MXFP8 inputs, the reading is OCP MX v1.0's MXFP8 (E4M3) with
-   that specification's shared-scale rule.
+   pages name no activation format; for the block-scaled variants, whose routed
+   experts take MXFP8 or MXFP4 inputs, the reading is OCP MX v1.0's MXFP8
+   (E4M3) or MXFP4 (E2M1) with that specification's shared-scale rule.
 
 Readings where the pages are silent (each is also listed in the design notes):
   * SiTU-GLU is taken as  h = sigmoid(g) * c*tanh(g/c) * c*tanh(v/c),  c = 10:
@@ -57,6 +57,11 @@ __all__ = [
     "mx8_quantize",
     "mx8_dequant",
     "mx8_round",
+    "e2m1_encode",
+    "mx4_quantize",
+    "mx4_round",
+    "routed_act",
+    "act_round",
     "sigmoid",
     "router_scores",
     "select_experts",
@@ -212,6 +217,67 @@ def mx8_round(v) -> torch.Tensor:
     return mx8_dequant(*mx8_quantize(v))
 
 
+def e2m1_encode(v) -> np.ndarray:
+    """Nearest E2M1 code (one per byte, 0..15) to each fp64 value, ties to the
+    even code, magnitudes beyond 6 (the largest E2M1) saturated to 6; -0 keeps
+    its sign.
+
+    The E2M1 numbers are spaced 0.5 below 2 (0.5 is the subnormal) and
+    2^(q-1) between 2^q and 2^(q+1) for q = 1, 2, so rounding is
+    round_half_even(a / spacing) spacing units."""
+    v = torch.as_tensor(v).to(F64)
+    neg = torch.signbit(v)
+    a = torch.clamp(v.abs(), max=6.0)
+    _, ex = torch.frexp(a)                   # a in [2^(ex-1), 2^ex)
+    q = torch.clamp(ex.to(torch.int64) - 1, min=0)
+    units = torch.round(torch.ldexp(a, (1 - q).to(torch.int64)))   # half to even
+    # q = 0: units 0..4 are the codes 0..4 (4 = 2.0); q >= 1: units 2..4, 4 carries
+    carry = (q >= 1) & (units >= 4)
+    q = torch.where(carry, q + 1, q)
+    units = torch.where(carry, units / 2, units).to(torch.int64)
+    code = torch.where(q == 0, units, ((q + 1) << 1) | (units - 2))
+    code = torch.where(neg, code | 8, code)
+    return code.to(torch.uint8).numpy()
+
+
+def mx4_quantize(v) -> tuple[np.ndarray, np.ndarray]:
+    """Rows of fp64 values [R, K] (K a multiple of 32) -> OCP MXFP4: per block
+    of 32 along K the shared scale 2^s, s = floor(log2(max |v|)) - 2 (2 = the
+    largest E2M1 exponent) clamped to [-127, 127] (an all-zero block takes
+    -127), and the E2M1 codes of v / 2^s, two per byte (element 2i in the low
+    nibble).  Returns (codes [R, K/2], scale bytes s + 127 [R, K/32])."""
+    v = torch.as_tensor(v).to(F64)
+    R, K = v.shape
+    blocks = v.reshape(R, K // 32, 32)
+    amax = blocks.abs().amax(dim=2)
+    _, ex = torch.frexp(amax)
+    s = torch.clamp(ex.to(torch.int64) - 1 - 2, min=-127, max=127)
+    s = torch.where(amax == 0, torch.full_like(s, -127), s)
+    scaled = torch.ldexp(blocks, (-s)[:, :, None].expand(R, K // 32, 32))
+    nib = e2m1_encode(scaled.reshape(R, K))
+    codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    return codes, (s + 127).to(torch.uint8).numpy()
+
+
+def mx4_round(v) -> torch.Tensor:
+    """The values the MXFP4 encoding of rows v stands for."""
+    return mxfp4_dequant(*mx4_quantize(v))
+
+
+def routed_act(cfg) -> str | None:
+    """The input format of the routed experts' GEMMs: "mxfp8" for the
+    block-scaled MXFP4 x MXFP8 variant, "mxfp4" for MXFP4 x MXFP4, else None
+    (the stored activations)."""
+    return {"mxfp4_a8": "mxfp8", "mxfp4_a4": "mxfp4"}.get(getattr(cfg, "routed", None))
+
+
+def act_round(act: str | None, v) -> torch.Tensor:
+    """Rows v replaced by their values in the activation format act."""
+    if act is None:
+        return v
+    return {"mxfp8": mx8_round, "mxfp4": mx4_round}[act](v)
+
+
 # ----------------------------------------------------------------------------------------------
 # Router: s = Sigmoid(W_r x), bias for selection only, renormalised unbiased scores
 # ([K3-896] section "ルーターは計算の割当器"; [K3-2axis] fixed bias + ordinary top-k)
@@ -301,18 +367,17 @@ def situ_glu(g: torch.Tensor, v: torch.Tensor, c: float) -> torch.Tensor:
 
 
 def expert_forward(z_rows: torch.Tensor, Wg: torch.Tensor, Wv: torch.Tensor, Wo: torch.Tensor, c: float, rnd,
-                   act_mx8: bool = False):
+                   act: str | None = None):
     """One GLU expert on latent rows: g = W_g z, v = W_v z, h = SiTU-GLU(g, v)
-    (stored, so rounded by rnd), y = W_o h (fp64, not rounded).  act_mx8 (the
-    block-scaled variant): the rows of z, and of h after rnd, are replaced by
-    their MXFP8 values before they enter the products."""
-    if act_mx8:
-        z_rows = mx8_round(z_rows)
+    (stored, so rounded by rnd), y = W_o h (fp64, not rounded).  act ("mxfp8"
+    or "mxfp4", the block-scaled variants): the rows of z, and of h after rnd,
+    are replaced by their values in that format before they enter the
+    products."""
+    z_rows = act_round(act, z_rows)
     g = z_rows @ Wg.T
     v = z_rows @ Wv.T
     h = rnd(situ_glu(g, v, c))
-    if act_mx8:
-        h = mx8_round(h)
+    h = act_round(act, h)
     return h @ Wo.T
 
 
@@ -378,7 +443,7 @@ def layer_forward(cfg, w: dict, x: torch.Tensor, forced_idx=None) -> dict:
     for e in torch.unique(idx).tolist():
         t, j = torch.nonzero(idx == e, as_tuple=True)
         y_slots[t, j] = expert_forward(z[t], w["Wg"][e], w["Wv"][e], w["Wo"][e], cfg.situ_c, rnd,
-                                       act_mx8=getattr(cfg, "routed", None) == "mxfp4_a8")
+                                       act=routed_act(cfg))
     out = _finish(x, z, idx, p, y_slots, w, cfg, rnd)
     out.update({"s": s, "idx": idx, "p": p, "margin": margin})
     return out
@@ -402,7 +467,7 @@ def layer_forward_streamed(cfg, dense: dict, x: torch.Tensor, expert_weights, fo
     for e in torch.unique(idx).tolist():
         t, j = torch.nonzero(idx == e, as_tuple=True)
         Wg, Wv, Wo = expert_weights(e)
-        y_slots[t, j] = expert_forward(z[t], Wg, Wv, Wo, cfg.situ_c, rnd, act_mx8=getattr(cfg, "routed", None) == "mxfp4_a8")
+        y_slots[t, j] = expert_forward(z[t], Wg, Wv, Wo, cfg.situ_c, rnd, act=routed_act(cfg))
     out = _finish(x, z, idx, p, y_slots, dense, cfg, rnd)
     out.update({"s": s, "idx": idx, "p": p, "margin": margin})
     return out

@@ -135,7 +135,7 @@ def test_expert_ffn_a8(T, skew):
         if a == b:
             continue
         Wg, Wv, Wo = oin.expert_weights(cfg, e)
-        ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wv, Wo, cfg.situ_c, oracle.bf16_round, act_mx8=True)
+        ref[a:b] = oracle.expert_forward(zf[a:b], Wg, Wv, Wo, cfg.situ_c, oracle.bf16_round, act="mxfp8")
     assert parity(y_perm.cpu().to(F64), ref) <= TOL_MXFP4_A8
 
 

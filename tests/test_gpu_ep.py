@@ -62,7 +62,7 @@ def test_expert_ffn_blocks_three_sources(name, lo, hi):
     for e in np.unique(expert_of_row):
         r = torch.as_tensor(np.nonzero(expert_of_row == e)[0])
         ref[r] = oracle.expert_forward(xf[r], *oin.expert_weights_raw(cfg, int(e)), cfg.situ_c, oracle.bf16_round,
-                                       act_mx8=cfg.routed == "mxfp4_a8")
+                                       act=oracle.routed_act(cfg))
     assert parity(y.cpu().to(F64), ref) <= 1e-2
 
 

@@ -155,7 +155,7 @@ def test_cpp_and_torch_mx8_agree_bit_for_bit():
 
 
 def test_expert_forward_mx8_rounds_both_inputs(O):
-    """act_mx8: the expert sees the MXFP8 values of its z rows and of h.  With
+    """act="mxfp8": the expert sees the MXFP8 values of its z rows and of h.  With
     z already MXFP8-exact the gate/up inputs are unchanged, so the result is
     W_o applied to mx8_round(h); with an identity-like W_o that is h's MXFP8
     rounding itself, which differs from the unquantised expert."""
@@ -165,11 +165,107 @@ def test_expert_forward_mx8_rounds_both_inputs(O):
     Wg = torch.randn(I, L, generator=g, dtype=F64) / 8
     Wv = torch.randn(I, L, generator=g, dtype=F64) / 8
     Wo = torch.eye(L, I, dtype=F64)
-    y8 = O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round, act_mx8=True)
+    y8 = O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round, act="mxfp8")
     h = O.bf16_round(O.situ_glu(z @ Wg.T, z @ Wv.T, 10.0))
     assert torch.equal(y8, O.mx8_round(h))
     y = O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round)
     assert torch.equal(y, h) and not torch.equal(y, y8)
+
+
+def _e2m1_table():
+    """Code -> value of the 16 E2M1 codes, from the OCP table (golden file)."""
+    tab = {int(r[0]): float(r[1]) for r in read_golden("e2m1_ocp_mx.txt")}
+    return np.array([tab[c] for c in range(16)])
+
+
+def test_e2m1_encode_is_the_nearest_code_ties_to_even(O):
+    """Brute force over the OCP table: every value maps to the code whose value
+    is nearest (magnitudes beyond 6 to +-6), a tie going to the even code; the
+    sign is kept, -0 included.  Midpoints of every neighbour pair are in the
+    sample, so a wrong tie rule or spacing fails."""
+    tab = _e2m1_table()
+    mags = tab[:8]
+    mids = (mags[:-1] + mags[1:]) / 2
+    rng = np.random.default_rng(21)
+    v = np.concatenate([mags, mids, np.nextafter(mids, 0), np.nextafter(mids, 10), rng.uniform(0, 9, 5000),
+                        [6.5, 7.0, 100.0, 1e300]])
+    v = np.concatenate([v, -v])
+    got = O.e2m1_encode(torch.from_numpy(v))
+    for x, c in zip(v, got):
+        a = min(abs(x), 6.0)
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        want = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert c == (want | (8 if np.signbit(x) else 0)), (x, c)
+    assert list(O.e2m1_encode(torch.tensor([0.0, -0.0], dtype=F64))) == [0, 8]
+    assert np.array_equal(O.e2m1_encode(torch.from_numpy(tab[np.r_[0:8, 9:16]])), np.r_[0:8, 9:16])
+
+
+def test_mx4_scale_rule_closed_forms(O):
+    """OCP MX v1.0 shared scale of an MXFP4 block, s = floor(log2 max|v|) - 2,
+    clamped to the E8M0 range; codes of v / 2^s packed two per byte, the even
+    element in the low nibble."""
+    def q(block):
+        c, s = O.mx4_quantize(torch.tensor([block], dtype=F64))
+        return c[0], int(s[0, 0])
+
+    c, s = q([1.0] * 32)                      # s = -2: 1 -> 4, code 6
+    assert s == 125 and set(c) == {0x66}
+    c, s = q([7.0] + [0.0] * 31)              # s = 0: 7 saturates to 6 (code 7)
+    assert s == 127 and c[0] == 0x07 and set(c[1:]) == {0}
+    c, s = q([0.0] * 32)                      # all-zero block: the lowest scale
+    assert s == 0 and set(c) == {0}
+    c, s = q([-3.0, 0.75] + [0.0] * 30)       # max 3 -> s = -1: -6 (code 15), 1.5 (code 3)
+    assert s == 126 and c[0] == (3 << 4) | 15
+    c, s = q([0.0, 6.0 * 2.0**100] + [0.0] * 30)  # s = 100: 6 in the high nibble
+    assert s == 227 and c[0] == 0x70
+    c, s = q([2.0**-130] + [0.0] * 31)        # clamped at -127: 2^-130 * 2^127 = 0.125 rounds to 0
+    assert s == 0 and set(c) == {0}
+    v = torch.tensor([[0.2] * 16 + [5.0] * 16], dtype=F64)  # s = 0: 0.2 -> 0 (nearest of 0, 0.5)
+    assert O.mx4_round(v)[0, 0].item() == 0.0 and O.mx4_round(v)[0, 16].item() == 4.0
+
+
+def test_mx4_round_is_the_nearest_block_value_and_idempotent(O):
+    """Each element of mx4_round(x) is, brute force, the nearest of the 15
+    values +-E2M1 * 2^s of its block to x (ties to the even code), and
+    quantising the result again changes nothing."""
+    g = torch.Generator().manual_seed(22)
+    x = torch.randn(16, 128, generator=g, dtype=F64) * torch.exp2(torch.randint(-20, 20, (16, 4), generator=g)
+                                                                   .to(F64)).repeat_interleave(32, dim=1)
+    r = O.mx4_round(x)
+    assert torch.equal(O.mx4_round(r), r)
+    _, s = O.mx4_quantize(x)
+    tab = _e2m1_table()
+    for i in range(x.shape[0]):
+        for k in range(x.shape[1]):
+            sc = 2.0 ** (int(s[i, k // 32]) - 127)
+            cand = tab * sc
+            d = np.abs(cand - x[i, k].item())
+            best = np.flatnonzero(d == d.min())
+            best = [b for b in best if b % 2 == 0] or list(best)
+            assert r[i, k].item() in cand[best], (i, k)
+
+
+def test_cpp_and_torch_mx4_agree_bit_for_bit():
+    x = torch.randn(200, 1024, generator=torch.Generator().manual_seed(23), dtype=F64).to(torch.bfloat16).to(F64)
+    x = x * torch.exp2(torch.randint(-40, 40, (200, 1), generator=torch.Generator().manual_seed(24)).to(F64))
+    a = oracle.mx4_quantize(x)
+    b = oracle.torch_ref.mx4_quantize(x)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_expert_forward_mx4_rounds_both_inputs(O):
+    """act="mxfp4": as for MXFP8, with the MXFP4 values of z and of h."""
+    g = torch.Generator().manual_seed(25)
+    L, I, n = 64, 64, 5
+    z = O.mx4_round(torch.randn(n, L, generator=g, dtype=F64))
+    Wg = torch.randn(I, L, generator=g, dtype=F64) / 8
+    Wv = torch.randn(I, L, generator=g, dtype=F64) / 8
+    Wo = torch.eye(L, I, dtype=F64)
+    y4 = O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round, act="mxfp4")
+    h = O.bf16_round(O.situ_glu(z @ Wg.T, z @ Wv.T, 10.0))
+    assert torch.equal(y4, O.mx4_round(h))
+    assert not torch.equal(y4, O.expert_forward(z, Wg, Wv, Wo, 10.0, O.bf16_round, act="mxfp8"))
 
 
 def test_sigmoid_matches_scipy(O):
