@@ -5,12 +5,14 @@ One step = one moe_layer_forward over one batch of T synthetic tokens (all
 stages: router, top-k, latent projection, shared experts, permute, routed
 experts, combine + RMSNorm, output projection).
 
-The default run measures four K3-shape workloads, one after the other:
+The default run measures five K3-shape workloads, one after the other:
   prefill   T=16384, bf16, Zipf(0.8) expert load  -> the headline line
   decode    T=256, bf16, bias N(0, 0.05)           -> "decode" sub-object
   mxfp4     T=8192, MXFP4 routed weights           -> "mxfp4" sub-object
   mxfp4-a8  T=8192, the same MXFP4 weights, expert inputs quantised to MXFP8,
             block-scaled tensor-core MMA           -> "mxfp4-a8" sub-object
+  mxfp4-a4  T=8192, the same MXFP4 weights, expert inputs quantised to MXFP4,
+            all-4-bit block-scaled MMA             -> "mxfp4-a4" sub-object
 (H=7168, L=3584, 896 experts top-16, I=3072, 2 shared experts, Is=3072).
 Each line carries its own device time, stage times, roofline, end-to-end
 number, near-tie count and an oracle sample (parity and CPU baseline).
@@ -66,8 +68,9 @@ def dims_for(cfg, y_out: str) -> moe.Dims:
 def workload_name(cfg) -> str:
     load = "Zipf(0.8) expert load" if cfg.bias == "zipf" else "bias N(0,0.05)"
     w = {"mxfp4": "MXFP4 routed weights",
-         "mxfp4_a8": "MXFP4 routed weights x MXFP8 expert inputs (block-scaled MMA)"}.get(cfg.routed,
-                                                                                         f"{cfg.act} weights")
+         "mxfp4_a8": "MXFP4 routed weights x MXFP8 expert inputs (block-scaled MMA)",
+         "mxfp4_a4": "MXFP4 routed weights x MXFP4 expert inputs (all-4-bit block-scaled MMA)"}.get(
+        cfg.routed, f"{cfg.act} weights")
     return (f"{cfg.name}: Stable LatentMoE layer T={cfg.T}, H={cfg.H}, L={cfg.L}, E={cfg.E} top-{cfg.k}, "
             f"I={cfg.I}, {cfg.S} shared (Is={cfg.Is}), {w}, {load}")
 
@@ -141,7 +144,7 @@ def barrier(world: int) -> None:
 
 # ----------------------------------------------------------------------------------- roofline
 def routed_weight_bytes_per_element(cfg) -> float:
-    if cfg.routed in ("mxfp4", "mxfp4_a8"):
+    if cfg.routed in ("mxfp4", "mxfp4_a8", "mxfp4_a4"):
         return 0.53125  # 4 bits + one E8M0 byte per 32
     return 2.0 if cfg.routed == "bf16" else 4.0
 
@@ -155,7 +158,8 @@ def stage_work(cfg, offsets: np.ndarray, T: int) -> dict:
     touched = int((counts > 0).sum())
     wbytes = 2 * cfg.I * cfg.L * routed_weight_bytes_per_element(cfg)
     flops = 2.0 * R * cfg.L * 2 * cfg.I
-    act_in = 1.03125 if cfg.routed == "mxfp4_a8" else 2.0  # MXFP8 rows: E4M3 + E8M0/32
+    # MXFP8 rows: E4M3 + E8M0/32; MXFP4 rows: E2M1 + E8M0/32
+    act_in = {"mxfp4_a8": 1.03125, "mxfp4_a4": 0.53125}.get(cfg.routed, 2.0)
     bytes_ = touched * wbytes + R * cfg.L * act_in + R * cfg.I * 2
     return {"flops": flops, "bytes": bytes_, "touched_experts": touched}
 
@@ -177,8 +181,8 @@ def gate_up_kernel(cfg) -> str:
     of moe_api.cu's use_two_tile: bf16 weights whose tiles divide evenly take
     the two-weight-tile kernel when the average expert has fewer than 64 rows,
     or as MOE_EXPERT_KERNEL forces; MXFP4 takes the one-tile kernel)."""
-    if cfg.routed == "mxfp4_a8":
-        return "tc_expert_bs_kernel<3, 1>"
+    if cfg.routed in ("mxfp4_a8", "mxfp4_a4"):
+        return f"tc_expert_bs_kernel<3, 1, {1 if cfg.routed == 'mxfp4_a4' else 0}>"
     cg = 2 if (cfg.I % 128 == 0 and cfg.L % 256 == 0) else 1
     env = os.environ.get("MOE_EXPERT_KERNEL", "")
     two = cfg.routed == "bf16" and cfg.I % (128 * cg) == 0 and (
@@ -199,6 +203,12 @@ def gate_up_roofline(cfg, offsets, stage_ms: dict, peaks: dict) -> dict:
         tensor_peak = 2.0 * peaks["bf16_tflops_sustained"]
         tsrc = (f"{peaks['source']} sustained bf16 x 2 (nominal fp8/bf16 ratio): the MMA kind is kind::mxf8f6f4 "
                 "with E2M1 weights and E4M3 activations")
+    elif cfg.routed == "mxfp4_a4":
+        # kind::mxf4 runs at the fp4 rate: the measured bf16 peak times the
+        # nominal fp4 / bf16 ratio (9 / 2.25 PFLOP/s dense)
+        tensor_peak = 4.0 * peaks["bf16_tflops_sustained"]
+        tsrc = (f"{peaks['source']} sustained bf16 x 4 (nominal fp4/bf16 ratio): the MMA kind is kind::mxf4 "
+                "with E2M1 weights and activations")
     else:
         tensor_peak = peaks["bf16_tflops_sustained"]
         tsrc = f"{peaks['source']} sustained bf16 (the MMA kind is kind::f16 with bf16 operands)"
@@ -223,7 +233,8 @@ def gate_up_roofline(cfg, offsets, stage_ms: dict, peaks: dict) -> dict:
         if rec.get("kernel") == kname:
             traffic = rec.get("dram_bytes_per_launch")
     kern = kname + {"mxfp4": " (2-CTA grouped gate/up, SiTU epilogue, MXFP4 weights decoded to bf16 in shared memory)",
-                    "mxfp4_a8": " (2-CTA grouped gate/up, SiTU epilogue, block-scaled MXFP4 x MXFP8 MMA)"}.get(
+                    "mxfp4_a8": " (2-CTA grouped gate/up, SiTU epilogue, block-scaled MXFP4 x MXFP8 MMA)",
+                    "mxfp4_a4": " (2-CTA grouped gate/up, SiTU epilogue, block-scaled MXFP4 x MXFP4 MMA)"}.get(
         cfg.routed, " (2-CTA grouped gate/up, SiTU epilogue)")
     return {"kernel": f"{kern} = stage expert_gate_up", "bound": bound, "achieved": round(achieved, 1),
             "peak": peak, "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": src,
@@ -437,7 +448,7 @@ def oracle_sample(cfg, layer, x, n_tokens: int, seed_offset: int = 0) -> tuple[d
               "differences_without_near_tie": int((differ & ~near).sum()), "near_tie_tokens": int(near.sum()),
               "max_abs_dy_over_rms": round(float((y_dev - ref["y"]).abs().max()) / rms, 6),
               "max_rms_dy_over_rms": round(float((y_dev - ref["y"]).pow(2).mean().sqrt()) / rms, 6),
-              "tolerance": {"mxfp4": 3e-2, "mxfp4_a8": 1e-1}.get(cfg.routed, 1e-2),
+              "tolerance": {"mxfp4": 3e-2, "mxfp4_a8": 1e-1, "mxfp4_a4": 0.5}.get(cfg.routed, 1e-2),
               "oracle": "fp64 C++ oracle (oracle/moe_oracle.cpp), storage-faithful bf16 rounding"}
     cpu = {"value": round(len(tokens) / oracle_s, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
            "kind": "oracle",
@@ -584,7 +595,7 @@ def run_ours(args, rank, world, local_rank):
     out.update({k: v for k, v in line.items() if k not in ("value", "unit", "ms_per_step")})
     out["qb_update"] = measure_qb(cfg, dev, stream, peaks)
 
-    extra = [] if args.no_extra_lines or args.config != "prefill" else ["decode", "mxfp4", "mxfp4-a8"]
+    extra = [] if args.no_extra_lines or args.config != "prefill" else ["decode", "mxfp4", "mxfp4-a8", "mxfp4-a4"]
     for name in extra:
         sub = gen.CONFIGS[name]
         if name == "decode":
@@ -596,7 +607,7 @@ def run_ours(args, rank, world, local_rank):
             xs = x[: sub.T].contiguous()
             out["decode"] = workload_line(sub, lay, xs, args, world, rank, local_rank, peaks, headline=False)
             del lay, xs, w
-        elif name == "mxfp4-a8":
+        elif name in ("mxfp4-a8", "mxfp4-a4"):
             # the MXFP4 workload's weights and x (same seed and shapes), routed
             # experts on the block-scaled path
             del layer

@@ -23,8 +23,9 @@ class LayerConfig:
     S: int  # shared experts
     Is: int  # shared-expert intermediate
     act: str = "bf16"  # activations / dense weights: "f32" or "bf16"
-    # routed-expert weights: "f32", "bf16", "mxfp4", or "mxfp4_a8" (MXFP4
-    # weights with the experts' inputs quantised to MXFP8: the block-scaled path)
+    # routed-expert weights: "f32", "bf16", "mxfp4", "mxfp4_a8" or "mxfp4_a4"
+    # (MXFP4 weights with the experts' inputs quantised to MXFP8 / MXFP4: the
+    # block-scaled paths)
     routed: str = "bf16"
     bias: str = "normal"  # "normal" (N(0, bias_std)) or "zipf"
     bias_std: float = 0.05
@@ -81,6 +82,14 @@ CONFIGS: dict[str, LayerConfig] = {
                                  routed="mxfp4_a8"),
     "mxfp4a8-e64": LayerConfig("mxfp4a8-e64", T=1024, H=7168, L=3584, E=64, k=16, I=3072, S=2, Is=3072, bias="zipf",
                                routed="mxfp4_a8", oracle_tokens=64),
+    # All-4-bit variant: MXFP4 routed weights x MXFP4 expert inputs, the same
+    # three sizes.
+    "mxfp4-a4": LayerConfig("mxfp4-a4", T=8192, H=7168, L=3584, E=896, k=16, I=3072, S=2, Is=3072,
+                            routed="mxfp4_a4", oracle_tokens=512),
+    "mxfp4a4-small": LayerConfig("mxfp4a4-small", T=1024, H=2048, L=1024, E=64, k=8, I=1024, S=2, Is=1024,
+                                 routed="mxfp4_a4"),
+    "mxfp4a4-e64": LayerConfig("mxfp4a4-e64", T=1024, H=7168, L=3584, E=64, k=16, I=3072, S=2, Is=3072, bias="zipf",
+                               routed="mxfp4_a4", oracle_tokens=64),
 }
 
 # Tensor ids: the second half of the Philox key of each input tensor.
@@ -145,5 +154,5 @@ def tensor_dtype(cfg: LayerConfig, name: str) -> str:
     if name in ("bias", "gamma"):
         return "f32"
     if name in ("Wg", "Wv", "Wo"):
-        return "mxfp4" if cfg.routed == "mxfp4_a8" else cfg.routed
+        return "mxfp4" if cfg.routed in ("mxfp4_a8", "mxfp4_a4") else cfg.routed
     return cfg.act

@@ -60,6 +60,13 @@
  *    read in the tiled order of moe_mx_tile_scales (moe_weights.Sgv_tiled,
  *    So_tiled); Wg, Wv and Wo must be 32-byte aligned.  Same dims rules as
  *    MOE_MXFP4.
+ *  - MOE_BF16 / MOE_MXFP4_A4  as MOE_MXFP4_A8 with the expert inputs quantised
+ *    to OCP MXFP4 instead: per block of 32 the E8M0 scale 2^s,
+ *    s = floor(log2(max |v|)) - 2 clamped to [-127, 127] (-127 for an all-zero
+ *    block), and E2M1 codes round-to-nearest-even(v / 2^s) saturated to +-6,
+ *    two per byte (the even element in the low nibble).  Both expert GEMMs run
+ *    on tcgen05.mma kind::mxf4 (both operands 4-bit); same scale tiles,
+ *    alignment and dims rules as MOE_MXFP4_A8.
  * Stored activations (z, expert h, shared h, n) are held in the activation type;
  * y_perm, u and the router scores are fp32.
  */
@@ -90,7 +97,7 @@ typedef enum {
   MOE_ERR_DEVICE = 4       /* moe_device_error only: a kernel recorded a device-side fault */
 } moe_status;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP4 = 2, MOE_MXFP4_A8 = 3 } moe_dtype;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP4 = 2, MOE_MXFP4_A8 = 3, MOE_MXFP4_A4 = 4 } moe_dtype;
 
 /* Layer shape and numerics.  K3 values: H=7168, L=3584, E=896, k=16, I=3072,
  * S=2, Is=3072 (dimension table of the page cited above). */
@@ -129,7 +136,7 @@ typedef struct {
   const void* Wsg;     /* [S, Is, H] shared gate projections */
   const void* Wsv;     /* [S, Is, H] shared up projections */
   const void* Wso;     /* [S, H, Is] shared down projections */
-  /* MOE_MXFP4_A8 only (NULL otherwise): the E8M0 scales of W_g / W_v and of
+  /* MOE_MXFP4_A8 / MOE_MXFP4_A4 only (NULL otherwise): the E8M0 scales of W_g / W_v and of
    * W_o in the tiled order written by moe_mx_tile_scales (Sg, Sv, So are not
    * read on that path and may be NULL). */
   const uint8_t* Sgv_tiled;
@@ -200,8 +207,8 @@ MOE_API moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, const
  *   h = SiTU-GLU(z_perm[r] . Wg[e]^T, z_perm[r] . Wv[e]^T)   (stored in act type)
  *   y_perm[r] = h . Wo[e]^T                                    (fp32 [T*k, L])
  * Only w->Wg, w->Wv, w->Wo (and for MXFP4 w->Sg, w->Sv, w->So; for
- * MOE_MXFP4_A8 w->Sgv_tiled, w->So_tiled, with z_perm and h quantised to
- * MXFP8 first) are read.
+ * MOE_MXFP4_A8 / MOE_MXFP4_A4 w->Sgv_tiled, w->So_tiled, with z_perm and h
+ * quantised to MXFP8 / MXFP4 first) are read.
  * Workspace: moe_workspace_size(d) bytes. */
 MOE_API moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z_perm,
                           const int32_t* expert_offsets, float* y_perm, void* ws, size_t ws_bytes,
@@ -253,7 +260,9 @@ MOE_API moe_status moe_output(const moe_dims* d, const moe_weights* w, const voi
  *    call (e.g. one rank's partition); other weight fields are not read.
  *  - Workspace: moe_expert_ffn_blocks_workspace_size(d, n_rows, n_blocks)
  *    bytes, 256-byte aligned.  Offsets outside [0, n_rows] are recorded as a
- *    device fault (moe_device_error) and their segment is skipped.
+ *    device fault (moe_device_error) and their segment is skipped.  After the
+ *    call the workspace begins with h [n_rows, I] in the activation type (the
+ *    stored SiTU-GLU rows, before any quantisation), for inspection.
  * d->T and d->k are not used. */
 MOE_API size_t moe_expert_ffn_blocks_workspace_size(const moe_dims* d, int64_t n_rows, int32_t n_blocks);
 MOE_API moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const void* x_rows, int64_t n_rows,
@@ -359,7 +368,16 @@ MOE_API moe_status moe_layer_backward(const moe_dims* d, const moe_weights* w, c
 MOE_API moe_status moe_mx8_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
                                     moe_stream_t stream);
 
-/* Weight scales for the block-scaled routed experts (routed = MOE_MXFP4_A8).
+/* The activation quantiser of the MXFP4-input path (routed = MOE_MXFP4_A4),
+ * on its own: rows of x [rows, K] bf16 -> OCP MXFP4 codes [rows, K/2] (E2M1,
+ * two per byte, the even element in the low nibble) and E8M0 scale bytes
+ * [rows, K/32] (row-major), by the rule stated at MOE_MXFP4_A4 above.  Same
+ * argument rules as moe_mx8_quantize. */
+MOE_API moe_status moe_mx4_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
+                                    moe_stream_t stream);
+
+/* Weight scales for the block-scaled routed experts (routed = MOE_MXFP4_A8 or
+ * MOE_MXFP4_A4).
  * The block-scaled MMA takes its scales from tensor memory, loaded from
  * shared memory in 512-byte atoms of 128 rows x 4 blocks of 32 along K (byte
  * 16*(m%32) + 4*(m/32) + j = row m, block j); moe_mx_tile_scales re-orders the

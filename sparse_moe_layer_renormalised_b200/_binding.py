@@ -17,8 +17,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE = 0, 1, 2, 3, 4
-MOE_F32, MOE_BF16, MOE_MXFP4, MOE_MXFP4_A8 = 0, 1, 2, 3
-_DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "mxfp4": MOE_MXFP4, "mxfp4_a8": MOE_MXFP4_A8}
+MOE_F32, MOE_BF16, MOE_MXFP4, MOE_MXFP4_A8, MOE_MXFP4_A4 = 0, 1, 2, 3, 4
+_DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "mxfp4": MOE_MXFP4, "mxfp4_a8": MOE_MXFP4_A8, "mxfp4_a4": MOE_MXFP4_A4}
+# routed types whose experts run on the block-scaled MMA (tiled weight scales)
+BLOCK_SCALED = ("mxfp4_a8", "mxfp4_a4")
 
 EXPORTED = (
     "moe_workspace_size",
@@ -42,6 +44,7 @@ EXPORTED = (
     "moe_mx_tiled_scales_size",
     "moe_mx_tile_scales",
     "moe_mx8_quantize",
+    "moe_mx4_quantize",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -134,6 +137,7 @@ def lib() -> ctypes.CDLL:
         L.moe_mx_tiled_scales_size.argtypes = [pd, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
         L.moe_mx_tile_scales.argtypes = [pd, vp, vp, vp, vp, vp, vp]
         L.moe_mx8_quantize.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
+        L.moe_mx4_quantize.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
         for f in EXPORTED:
             if f not in ("moe_workspace_size", "moe_status_str", "moe_expert_ffn_blocks_workspace_size",
                          "moe_backward_workspace_size"):
@@ -330,6 +334,10 @@ def moe_mx_tile_scales(d, Sg, Sv, So, Sgv_tiled, So_tiled, stream=None) -> int:
 
 def moe_mx8_quantize(x, rows: int, K: int, codes, scales, stream=None) -> int:
     return lib().moe_mx8_quantize(_ptr(x), int(rows), int(K), _ptr(codes), _ptr(scales), _stream(stream))
+
+
+def moe_mx4_quantize(x, rows: int, K: int, codes, scales, stream=None) -> int:
+    return lib().moe_mx4_quantize(_ptr(x), int(rows), int(K), _ptr(codes), _ptr(scales), _stream(stream))
 
 
 def moe_selftest_wait_timeout(limit_ms: int, waited_ns, stream=None) -> int:

@@ -1,6 +1,7 @@
 // Block-scaled grouped routed-expert GEMM for sm_100a: MXFP4 weights times
-// MXFP8 activations on tcgen05.mma kind::mxf8f6f4 (the tensor cores apply
-// both operands' E8M0 block scales; no decode pass).
+// MXFP8 activations on tcgen05.mma kind::mxf8f6f4, or times MXFP4
+// activations on kind::mxf4 (template flag A4); the tensor cores apply both
+// operands' E8M0 block scales, no decode pass.
 //
 //   D[w, t] = sum_k (Wq[w, k] * 2^(sw[w, k/32] - 127)) * (Xq[t, k] * 2^(sx[t, k/32] - 127))
 //
@@ -28,13 +29,18 @@
 //    columns) and three scale buffers (3 x 24) fit the 512 columns of tensor
 //    memory; with three, the copier can put stage g's scales in the tensor
 //    pipe's queue ahead of stage g-1's MMAs.
+// With A4 both operands are packed E2M1 codes (two per byte, the even
+// element in the low nibble), which kind::mxf4 reads as they are: a stage's
+// K = 256 is one 128-byte wide box per operand (plain byte TMA, 128-byte
+// swizzle) and 4 MMAs of K = 64, each taking two scale bytes (j = 0 or 2) of
+// the same scale columns; stages are half the size, so there are five.
 // Warp roles: 0 TMA producer (both CTAs), 1 TMEM owner and MMA issuer (even
 // CTA), 2-5 epilogue (both CTAs), 6 scale copier (even CTA).  Every wait is
 // bounded.
 #pragma once
 
 #include "gemm_expert.cuh"
-#include "mx8.cuh"
+#include "mx_quant.cuh"
 
 namespace moe {
 
@@ -53,16 +59,27 @@ constexpr int BS_SF_BUFS = 3;
 constexpr uint32_t BS_SF_BUF_COLS = 24;            // SFA half 0 / 1 at +0 / +4, SFB half 0 / 1 at +8 / +16
 constexpr int BS_THREADS = 224;
 constexpr int BS_COPY_WARP = 6;
-constexpr uint32_t BS_STAGE_BYTES = BS_A_BYTES + BS_B_BYTES + BS_SFA_BYTES + BS_SFB_BYTES;
-constexpr size_t BS_SMEM = 1024 + static_cast<size_t>(BS_STAGES) * BS_STAGE_BYTES + EX_XCH_BYTES + 512;
 static_assert(BS_SF_COL + BS_SF_BUFS * BS_SF_BUF_COLS <= 2 * EX_ACC_COLS, "tensor memory columns");
-static_assert(BS_SMEM <= 232448, "shared memory per CTA");
+
+// Stage geometry of the two activation formats.
+template <bool A4>
+struct BsStage {
+  static constexpr uint32_t A_BYTES = A4 ? BS_HALF_BYTES : BS_A_BYTES;  // packed codes: 128 rows x 128 bytes
+  static constexpr uint32_t B_BYTES = A4 ? BS_HALF_BYTES : BS_B_BYTES;
+  static constexpr int STAGES = A4 ? 5 : BS_STAGES;
+  static constexpr uint32_t BYTES = A_BYTES + B_BYTES + BS_SFA_BYTES + BS_SFB_BYTES;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * BYTES + EX_XCH_BYTES + 512;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+  static_assert(STAGES >= BS_SF_BUFS, "the scale copier's reuse wait assumes a stage per scale buffer at least");
+};
 
 struct BsMaps {
-  CUtensorMap a0;    // E2M1 codes, 16 per 16-byte slot: PAIRED W_g [E*I, L] (64-row boxes), else W_o [E*L, I] (128-row)
+  CUtensorMap a0;    // E2M1 codes (A8: 16 per 16-byte slot; A4: packed bytes, 128-byte wide boxes):
+                     //   PAIRED W_g [E*I, L] (64-row boxes), else W_o [E*L, I] (128-row)
   CUtensorMap a1;    // PAIRED: W_v, as a0
   CUtensorMap sa;    // weight scale tiles as [n, 16] bytes, 64-row (two atoms, 1 KB) boxes
-  CUtensorMap b[4];  // E4M3 activation codes [R, K]: 128-byte wide boxes of 128, 64, 32, 16 rows, 128-byte swizzle
+  CUtensorMap b[4];  // activation codes (A8: E4M3 [R, K]; A4: packed E2M1 [R, K/2] bytes): 128-byte
+                     //   wide boxes of 128, 64, 32, 16 rows, 128-byte swizzle
   CUtensorMap sb;    // activation scale tiles as [n, 16] bytes, 128-row (two K chunks x two atoms, 2 KB) boxes
 };
 
@@ -85,6 +102,13 @@ __host__ __device__ constexpr uint32_t idesc_mxf4_mxf8(int M, int N, int j) {
          (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(j) << 29);
 }
 
+// kind::mxf4 with A = B = E2M1 (format 1 in [7, 10) and [10, 13)), E8M0
+// scales, K = 64 per MMA: scale bytes j and j + 1 (j = 0 or 2) of the column.
+__host__ __device__ constexpr uint32_t idesc_mxf4_mxf4(int M, int N, int j) {
+  return (static_cast<uint32_t>(j) << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(j) << 29);
+}
+
 // 32 rows x 128 bits of shared memory -> tensor memory lanes 0-31 of every
 // lane quarter (4 columns from taddr), in both CTAs of the pair.
 __device__ __forceinline__ void bs_copy_sf(uint32_t taddr, uint64_t sdesc) {
@@ -98,6 +122,17 @@ __device__ __forceinline__ void bs_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// As bs_mma, one 256 x N x 64 step of kind::mxf4 (two 32-blocks per scale).
+__device__ __forceinline__ void bs_mma4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                        uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
@@ -140,21 +175,23 @@ __device__ __forceinline__ ExTile bs_decode(int w, int num_tiles, int num_multi,
   return t;
 }
 
-template <int EPI, bool PAIRED>
+template <int EPI, bool PAIRED, bool A4>
 __global__ void __launch_bounds__(BS_THREADS, 1)
     tc_expert_bs_kernel(const __grid_constant__ BsMaps maps, const ExParams p) {
   constexpr int CG = 2;
+  using G = BsStage<A4>;
+  constexpr int kStages = G::STAGES;
   extern __shared__ uint8_t bs_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bs_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + BS_STAGES * BS_A_BYTES;
-  uint8_t* sSA = sB + BS_STAGES * BS_B_BYTES;
-  uint8_t* sSB = sSA + BS_STAGES * BS_SFA_BYTES;
-  float* xch = reinterpret_cast<float*>(sSB + BS_STAGES * BS_SFB_BYTES);
+  uint8_t* sB = sA + kStages * G::A_BYTES;
+  uint8_t* sSA = sB + kStages * G::B_BYTES;
+  uint8_t* sSB = sSA + kStages * BS_SFA_BYTES;
+  float* xch = reinterpret_cast<float*>(sSB + kStages * BS_SFB_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + EX_XCH_BYTES);
-  uint64_t* empty = full + BS_STAGES;
-  uint64_t* sf_full = empty + BS_STAGES;  // the stage's scales are in tensor memory (even CTA)
-  uint64_t* acc_full = sf_full + BS_STAGES;
+  uint64_t* empty = full + kStages;
+  uint64_t* sf_full = empty + kStages;  // the stage's scales are in tensor memory (even CTA)
+  uint64_t* acc_full = sf_full + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint64_t* copy_drain = drain + 1;
@@ -170,7 +207,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   const int npairs = static_cast<int>(gridDim.x >> 1);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < BS_STAGES; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_full[s], 1);
@@ -217,8 +254,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
         const int bsel = rows_cta > 64 ? 0 : rows_cta > 32 ? 1 : rows_cta > 16 ? 2 : 3;
         const int brows = 128 >> bsel;
         const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
-        const uint32_t bytes = static_cast<uint32_t>(CG) * (BS_A_TX + 2u * static_cast<uint32_t>(brows) * 128u +
-                                                            BS_SFA_BYTES + BS_SFB_BYTES);
+        const uint32_t b_tx = (A4 ? 1u : 2u) * static_cast<uint32_t>(brows) * 128u;
+        const uint32_t bytes = static_cast<uint32_t>(CG) * (BS_A_TX + b_tx + BS_SFA_BYTES + BS_SFB_BYTES);
         const int wrow = t.expert * p.w_rows_per_expert + (PAIRED ? t.wt * 128 : t.wt * 256) +
                          static_cast<int>(rank) * (PAIRED ? 64 : 128);
         // 16-byte rows of the scale tiles: 32 per atom
@@ -230,8 +267,20 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             break;
           }
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-          uint8_t* a_dst = sA + stage * BS_A_BYTES;
-          uint8_t* b_dst = sB + stage * BS_B_BYTES;
+          uint8_t* a_dst = sA + stage * G::A_BYTES;
+          uint8_t* b_dst = sB + stage * G::B_BYTES;
+          if constexpr (A4) {
+            // one 128-byte (256-code) wide box per operand; x in bytes
+            const int kc = kb * 128;
+            if (kExL2Hints && !t.multi) {
+              ex_tma_load_hint<CG>(a_dst, &maps.a0, &full[stage], kc, wrow, pol_w);
+              if (PAIRED) ex_tma_load_hint<CG>(a_dst + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
+            } else {
+              ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
+              if (PAIRED) ex_tma_load<CG>(a_dst + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
+            }
+            ex_tma_load_hint<CG>(b_dst, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
+          } else
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int kc = kb * BS_BK + h * 128;
@@ -249,7 +298,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
           ex_tma_load<CG>(sSB + stage * BS_SFB_BYTES, &maps.sb, &full[stage], 0, sb_row0 + kb * 128);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == BS_STAGES) {
+          if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -259,7 +308,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
       // load of the pair to land before the pair may exit.
       if (leader) {
         volatile int never = 0;
-        for (int s = 0; s < BS_STAGES; ++s)
+        for (int s = 0; s < kStages; ++s)
           if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_parity >> s) & 1u, &never, p.fault_site + 2);
       }
     }
@@ -278,7 +327,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort, p.fault_site + 3)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * BS_ACC_COLS;
-        const uint32_t idesc0 = idesc_mxf4_mxf8(256, t.n_mma, 0);
+        const uint32_t idesc0 = A4 ? idesc_mxf4_mxf4(256, t.n_mma, 0) : idesc_mxf4_mxf8(256, t.n_mma, 0);
         for (int kb = 0; kb < n_stages; ++kb, ++g) {
           if (!mbar_wait(&sf_full[stage], phase, abort, p.fault_site + 4)) {
             ok = false;
@@ -287,8 +336,20 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
           tc_fence_after();
           const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * BS_SF_BUF_COLS;
           if (++sf_buf == BS_SF_BUFS) sf_buf = 0;
-          const uint32_t a_addr = smem_u32(sA + stage * BS_A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * BS_B_BYTES);
+          const uint32_t a_addr = smem_u32(sA + stage * G::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * G::B_BYTES);
+          if constexpr (A4) {
+            // MMA kk covers K = 64 kk .. 64 kk + 63: 32-blocks 2kk, 2kk + 1, i.e.
+            // scale bytes 2 (kk % 2), +1 of the atoms of K chunk kk / 2
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t j = 2u * static_cast<uint32_t>(kk & 1);
+              const uint32_t h = static_cast<uint32_t>(kk >> 1);
+              bs_mma4(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
+                      idesc0 | (j << 4) | (j << 29), (sf + 4u * h) | (j << 30), (sf + 8u + 8u * h) | (j << 30),
+                      (kb | kk) != 0 ? 1u : 0u);
+            }
+          } else
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -300,7 +361,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
                      (sf + 8u + 8u * h) | (j << 30), (kb | h | kk) != 0 ? 1u : 0u);
             }
           ex_commit<CG>(&empty[stage]);
-          if (++stage == BS_STAGES) {
+          if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -343,7 +404,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
               ok = false;
               break;
             }
-            if (++prev2_stage == BS_STAGES) {
+            if (++prev2_stage == kStages) {
               prev2_stage = 0;
               prev2_phase ^= 1u;
             }
@@ -363,7 +424,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
           asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                            smem_u32(&sf_full[stage]))
                        : "memory");
-          if (++stage == BS_STAGES) {
+          if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }

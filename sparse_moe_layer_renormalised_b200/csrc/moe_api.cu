@@ -17,7 +17,7 @@
 #include "gemm_expert.cuh"
 #include "gemm_expert2.cuh"
 #include "gemm_expert_bs.cuh"
-#include "mx8.cuh"
+#include "mx_quant.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -45,7 +45,8 @@ bool dims_ok(const moe_dims* d) {
   if (!(d->situ_c > 0.f) || !std::isfinite(d->situ_c) || !(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps))
     return false;
   if (d->act != MOE_F32 && d->act != MOE_BF16) return false;
-  if (d->routed != MOE_F32 && d->routed != MOE_BF16 && d->routed != MOE_MXFP4 && d->routed != MOE_MXFP4_A8)
+  if (d->routed != MOE_F32 && d->routed != MOE_BF16 && d->routed != MOE_MXFP4 && d->routed != MOE_MXFP4_A8 &&
+      d->routed != MOE_MXFP4_A4)
     return false;
   if (d->y_out != MOE_F32 && d->y_out != d->act) return false;
   if (d->L % 8 != 0 || d->H % 8 != 0 || d->I % 8 != 0) return false;
@@ -56,7 +57,7 @@ bool dims_ok(const moe_dims* d) {
 
 // Valid dims that this build does not implement.
 bool dims_supported(const moe_dims* d) {
-  if (d->routed == MOE_MXFP4 || d->routed == MOE_MXFP4_A8) {
+  if (d->routed == MOE_MXFP4 || d->routed == MOE_MXFP4_A8 || d->routed == MOE_MXFP4_A4) {
     // MXFP4 routed weights: bf16 activations; code and scale rows must suit TMA
     // (K/2 and K/32 bytes per row, multiples of 16) for both expert GEMMs.
     // (The block-scaled path also needs K % 128 and 2-CTA weight tiles, which
@@ -89,13 +90,17 @@ int expert_cg(const moe_dims& d) { return (d.I % 128 == 0 && d.L % 256 == 0) ? 2
 
 // Largest token tile of the grouped expert GEMMs (MMA N = 256 on pairs; a
 // single CTA stages at most 128 token rows; the fp32 path uses 128-row tiles;
-// the block-scaled path 240, which leaves tensor memory for its scales).
+// the block-scaled paths 208, which leaves tensor memory for their scales).
 int expert_tile_rows(const moe_dims& d) {
-  if (d.routed == MOE_MXFP4_A8) return BS_MAX_TILE_ROWS;
+  if (d.routed == MOE_MXFP4_A8 || d.routed == MOE_MXFP4_A4) return BS_MAX_TILE_ROWS;
   return d.act == MOE_BF16 ? 128 * expert_cg(d) : 128;
 }
 
-inline bool routed_a8(const moe_dims& d) { return d.routed == MOE_MXFP4_A8; }
+// Block-scaled routed experts (MXFP8 or MXFP4 inputs); a4: the MXFP4 one.
+inline bool routed_bs(const moe_dims& d) { return d.routed == MOE_MXFP4_A8 || d.routed == MOE_MXFP4_A4; }
+inline bool routed_a4(const moe_dims& d) { return d.routed == MOE_MXFP4_A4; }
+// Bytes of one row of K activation codes in the block-scaled input format.
+inline size_t bs_code_bytes(const moe_dims& d, size_t K) { return routed_a4(d) ? K / 2 : K; }
 
 
 // ------------------------------------------------------------------------------ workspace
@@ -134,12 +139,12 @@ WsLayout ws_layout(const moe_dims& d) {
   w.h_s = take(T * static_cast<size_t>(d.S) * d.Is * es);
   w.dense_tiles = take(static_cast<size_t>(cdiv(static_cast<long long>(T), 128) + 1) * 16);
   w.dense_num = take(16);
-  // block-scaled path: E4M3 codes of h and the activation scale tiles (the
+  // block-scaled paths: the codes of h and the activation scale tiles (the
   // codes of the expert-major z rows reuse z_perm)
-  const bool a8 = routed_a8(d);
-  w.h_q = take(a8 ? R * d.I : 0);
-  w.sf_z = take(a8 ? max_m_tiles * (d.L / 128) * 1024 : 0);
-  w.sf_h = take(a8 ? max_m_tiles * (d.I / 128) * 1024 : 0);
+  const bool bs = routed_bs(d);
+  w.h_q = take(bs ? R * bs_code_bytes(d, d.I) : 0);
+  w.sf_z = take(bs ? max_m_tiles * (d.L / 128) * 1024 : 0);
+  w.sf_h = take(bs ? max_m_tiles * (d.I / 128) * 1024 : 0);
   w.total = off;
   return w;
 }
@@ -682,26 +687,29 @@ moe_status stage_expert_down(const moe_dims& d, const moe_weights& w, const void
 }
 
 // ------------------------------------------------------------------------------ block-scaled routed experts
-// Quantises rows of the grouped-GEMM token tiles to MXFP8 (codes [R, K] and
-// scale tiles; see mx8.cuh).  Row r reads src row src_row[r] (or r).
-moe_status stage_quant_mx8(const void* src, long long src_rows, const int32_t* src_row, const int4* table,
-                           const int32_t* n_tiles, int max_tiles, int K, uint8_t* codes, uint8_t* sf, int site,
-                           cudaStream_t s) {
+// Quantises rows of the grouped-GEMM token tiles to the block-scaled input
+// format of d (MXFP8 codes [R, K] or MXFP4 codes [R, K/2], and scale tiles;
+// see mx_quant.cuh).  Row r reads src row src_row[r] (or r).
+moe_status stage_quant_mx(const moe_dims& d, const void* src, long long src_rows, const int32_t* src_row,
+                          const int4* table, const int32_t* n_tiles, int max_tiles, int K, uint8_t* codes, uint8_t* sf,
+                          int site, cudaStream_t s) {
   const int grid = std::max(1, std::min(max_tiles, 8 * num_sms()));
-  mx8_quant_tiles_kernel<<<grid, MX8_WARPS * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(src), src_rows, src_row,
-                                                          table, n_tiles, 0, K, codes, sf, site);
+  auto kern = routed_a4(d) ? mx_quant_tiles_kernel<true> : mx_quant_tiles_kernel<false>;
+  kern<<<grid, MXQ_WARPS * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(src), src_rows, src_row, table, n_tiles, 0, K,
+                                       codes, sf, site);
   ++g_last_launches;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int EPI, bool PAIRED>
+template <int EPI, bool PAIRED, bool A4>
 cudaError_t launch_expert_bs(const BsMaps& maps, const ExParams& p, cudaStream_t s) {
-  auto kern = tc_expert_bs_kernel<EPI, PAIRED>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(BS_SMEM));
+  auto kern = tc_expert_bs_kernel<EPI, PAIRED, A4>;
+  constexpr size_t smem = BsStage<A4>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(BS_THREADS);
-  cfg.dynamicSmemBytes = BS_SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -737,13 +745,19 @@ moe_status stage_expert_bs(const moe_dims& d, bool paired, const moe_weights& w,
   const size_t sa_bytes = paired ? tiled_scales_gate_up(d) : tiled_scales_down(d);
   bool ok = true;
   // scale tiles as 16-byte rows: weight boxes of two atoms (two 128-wide K
-  // chunks, 1 KB), activation boxes of two chunks x two atoms (2 KB)
+  // chunks, 1 KB), activation boxes of two chunks x two atoms (2 KB).  The
+  // MXFP4-input kernel reads the packed weight codes as plain bytes.
+  const bool a4 = routed_a4(d);
+  auto wmap = [&](CUtensorMap* m, const void* codes, uint32_t box_rows) {
+    return a4 ? make_map_u8_sw128(m, codes, wrows, K / 2, box_rows) : make_map_e2m1(m, codes, wrows, K, box_rows);
+  };
   if (paired)
-    ok = make_map_e2m1(&maps.a0, w.Wg, wrows, K, 64) && make_map_e2m1(&maps.a1, w.Wv, wrows, K, 64) &&
+    ok = wmap(&maps.a0, w.Wg, 64) && wmap(&maps.a1, w.Wv, 64) &&
          make_map_u8(&maps.sa, w.Sgv_tiled, sa_bytes / 16, 16, 16, 64);
   else
-    ok = make_map_e2m1(&maps.a0, w.Wo, wrows, K, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, 64);
-  for (int i = 0; i < 4 && ok; ++i) ok = make_map_u8_sw128(&maps.b[i], act_q, static_cast<uint64_t>(R), K, 128u >> i);
+    ok = wmap(&maps.a0, w.Wo, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, 64);
+  for (int i = 0; i < 4 && ok; ++i)
+    ok = make_map_u8_sw128(&maps.b[i], act_q, static_cast<uint64_t>(R), bs_code_bytes(d, K), 128u >> i);
   const uint64_t sf_rows = static_cast<uint64_t>(max_tiles) * (K / 128) * 64;
   ok = ok && make_map_u8(&maps.sb, act_sf, sf_rows, 16, 16, 128);
   if (!ok) return MOE_ERR_CUDA;
@@ -758,22 +772,27 @@ moe_status stage_expert_bs(const moe_dims& d, bool paired, const moe_weights& w,
   p.out_cols = out_rows;
   p.situ_c = d.situ_c;
   p.fault_site = site;
-  const cudaError_t e = paired ? launch_expert_bs<kEpiSituBF16, true>(maps, p, s) : launch_expert_bs<kEpiF32, false>(maps, p, s);
+  cudaError_t e;
+  if (a4)
+    e = paired ? launch_expert_bs<kEpiSituBF16, true, true>(maps, p, s) : launch_expert_bs<kEpiF32, false, true>(maps, p, s);
+  else
+    e = paired ? launch_expert_bs<kEpiSituBF16, true, false>(maps, p, s)
+               : launch_expert_bs<kEpiF32, false, false>(maps, p, s);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // Buffers of the block-scaled routed-expert sequence.
-struct A8Bufs {
-  uint8_t* xq;   // [R, L] E4M3 codes of the expert-major latent rows
+struct BsBufs {
+  uint8_t* xq;   // codes of the expert-major latent rows ([R, L] E4M3 or [R, L/2] packed E2M1)
   uint8_t* sfx;  // their scale tiles
   void* h;       // [R, I] bf16 SiTU-GLU output
-  uint8_t* hq;   // [R, I] E4M3 codes of h
+  uint8_t* hq;   // codes of h
   uint8_t* sfh;  // their scale tiles
 };
 
-// The routed experts on the block-scaled path after the latent rows have been
-// quantised: gate/up -> h, h -> MXFP8, down -> y [R, L] fp32.
-moe_status run_routed_a8_after_quant(const moe_dims& d, const moe_weights& w, const A8Bufs& b, long long R,
+// The routed experts on a block-scaled path after the latent rows have been
+// quantised: gate/up -> h, h -> MXFP8 / MXFP4, down -> y [R, L] fp32.
+moe_status run_routed_bs_after_quant(const moe_dims& d, const moe_weights& w, const BsBufs& b, long long R,
                                      const int4* table, const int32_t* n_tiles, int max_tiles, float* y,
                                      cudaStream_t s, const std::function<void(int, int)>& mark) {
   moe_status st;
@@ -781,7 +800,8 @@ moe_status run_routed_a8_after_quant(const moe_dims& d, const moe_weights& w, co
   if ((st = stage_expert_bs(d, true, w, b.xq, b.sfx, R, table, n_tiles, max_tiles, b.h, 160, s)) != MOE_OK) return st;
   mark(MOE_STAGE_EXPERT_GATE_UP, 1);
   mark(MOE_STAGE_EXPERT_DOWN, 0);
-  if ((st = stage_quant_mx8(b.h, R, nullptr, table, n_tiles, max_tiles, d.I, b.hq, b.sfh, 181, s)) != MOE_OK) return st;
+  if ((st = stage_quant_mx(d, b.h, R, nullptr, table, n_tiles, max_tiles, d.I, b.hq, b.sfh, 181, s)) != MOE_OK)
+    return st;
   st = stage_expert_bs(d, false, w, b.hq, b.sfh, R, table, n_tiles, max_tiles, y, 170, s);
   mark(MOE_STAGE_EXPERT_DOWN, 1);
   return st;
@@ -876,7 +896,7 @@ moe_status stage_output(const moe_dims& d, const moe_weights& w, const void* h_s
 
 // MXFP4 routed weights need their E8M0 scale arrays; other types take none.
 moe_status check_scales(const moe_dims& d, const moe_weights& w) {
-  if (routed_a8(d)) {
+  if (routed_bs(d)) {
     // block-scaled path: the re-ordered scales (the row-major ones are not
     // read and may be NULL); the packed codes are read as 4-bit TMA tensors,
     // which need 32-byte aligned bases
@@ -916,12 +936,12 @@ BlocksWsLayout blocks_ws_layout(const moe_dims& d, long long n_rows, int n_block
   l.h = take(static_cast<size_t>(n_rows) * d.I * act_bytes(d));
   l.tile_table = take(static_cast<size_t>(l.max_tiles) * 16);
   l.num_tiles = take(16);
-  const bool a8 = routed_a8(d);
+  const bool bs = routed_bs(d);
   const size_t rows = static_cast<size_t>(n_rows), mt = static_cast<size_t>(l.max_tiles);
-  l.xq = take(a8 ? rows * d.L : 0);
-  l.sfx = take(a8 ? mt * (d.L / 128) * 1024 : 0);
-  l.hq = take(a8 ? rows * d.I : 0);
-  l.sfh = take(a8 ? mt * (d.I / 128) * 1024 : 0);
+  l.xq = take(bs ? rows * bs_code_bytes(d, d.L) : 0);
+  l.sfx = take(bs ? mt * (d.L / 128) * 1024 : 0);
+  l.hq = take(bs ? rows * bs_code_bytes(d, d.I) : 0);
+  l.sfh = take(bs ? mt * (d.I / 128) * 1024 : 0);
   l.total = off;
   return l;
 }
@@ -1179,6 +1199,24 @@ moe_status run_backward(const moe_dims& d, const moe_weights& w, const void* x, 
 }
 
 }  // namespace
+// MXFP8 / MXFP4 quantisation of row-major bf16 rows (row-major scales).
+moe_status mx_quantize_rows(bool fp4, const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
+                            moe_stream_t stream, int site) {
+  if (rows < 0 || K <= 0 || K % 32 != 0 || rows > 0x7fffffffLL) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || codes == nullptr || scales == nullptr || !aligned16(x) || !aligned16(codes)))
+    return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (rows == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long tiles = cdiv(rows, 128);
+  const int grid = static_cast<int>(std::min<long long>(tiles, 8LL * num_sms()));
+  auto kern = fp4 ? mx_quant_tiles_kernel<true> : mx_quant_tiles_kernel<false>;
+  kern<<<grid, MXQ_WARPS * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, nullptr, nullptr, nullptr, rows, K,
+                                       codes, scales, site);
+  g_last_launches = 1;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -1266,14 +1304,14 @@ moe_status moe_expert_ffn(const moe_dims* d, const moe_weights* w, const void* z
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   const int4* table = at<int4>(ws, L.tile_table);
   const int32_t* n_tiles = at<int32_t>(ws, L.num_m_tiles);
-  if (routed_a8(*d)) {
+  if (routed_bs(*d)) {
     const long long R = d->T * d->k;
     const int max_tiles = static_cast<int>(cdiv(R, TC_BM) + d->E);
-    const A8Bufs b{at<uint8_t>(ws, L.z_perm), at<uint8_t>(ws, L.sf_z), at<void>(ws, L.h_perm), at<uint8_t>(ws, L.h_q),
+    const BsBufs b{at<uint8_t>(ws, L.z_perm), at<uint8_t>(ws, L.sf_z), at<void>(ws, L.h_perm), at<uint8_t>(ws, L.h_q),
                    at<uint8_t>(ws, L.sf_h)};
-    if ((st = stage_quant_mx8(z_perm, R, nullptr, table, n_tiles, max_tiles, d->L, b.xq, b.sfx, 180, s)) != MOE_OK)
+    if ((st = stage_quant_mx(*d, z_perm, R, nullptr, table, n_tiles, max_tiles, d->L, b.xq, b.sfx, 180, s)) != MOE_OK)
       return st;
-    return run_routed_a8_after_quant(*d, *w, b, R, table, n_tiles, max_tiles, y_perm, s, [](int, int) {});
+    return run_routed_bs_after_quant(*d, *w, b, R, table, n_tiles, max_tiles, y_perm, s, [](int, int) {});
   }
   st = stage_expert_gate_up(*d, *w, z_perm, table, n_tiles, at<void>(ws, L.h_perm), s);
   if (st != MOE_OK) return st;
@@ -1357,18 +1395,18 @@ moe_status moe_layer_forward(const moe_dims* d, const moe_weights* w, const void
   // routed experts
   const int4* table = at<int4>(ws, L.tile_table);
   const int32_t* n_tiles = at<int32_t>(ws, L.num_m_tiles);
-  if (routed_a8(*d)) {
-    // block-scaled path: the gather writes the MXFP8 codes and scales of the
-    // expert-major z rows; h is quantised in the down stage
+  if (routed_bs(*d)) {
+    // block-scaled paths: the gather writes the MXFP8 / MXFP4 codes and
+    // scales of the expert-major z rows; h is quantised in the down stage
     const long long R = d->T * d->k;
     const int max_tiles = static_cast<int>(cdiv(R, TC_BM) + d->E);
-    const A8Bufs b{at<uint8_t>(ws, L.z_perm), at<uint8_t>(ws, L.sf_z), at<void>(ws, L.h_perm), at<uint8_t>(ws, L.h_q),
+    const BsBufs b{at<uint8_t>(ws, L.z_perm), at<uint8_t>(ws, L.sf_z), at<void>(ws, L.h_perm), at<uint8_t>(ws, L.h_q),
                    at<uint8_t>(ws, L.sf_h)};
     mark(MOE_STAGE_GATHER, 0);
-    if ((st = stage_quant_mx8(z, d->T, perm_token, table, n_tiles, max_tiles, d->L, b.xq, b.sfx, 180, s)) != MOE_OK)
+    if ((st = stage_quant_mx(*d, z, d->T, perm_token, table, n_tiles, max_tiles, d->L, b.xq, b.sfx, 180, s)) != MOE_OK)
       return st;
     mark(MOE_STAGE_GATHER, 1);
-    if ((st = run_routed_a8_after_quant(*d, *w, b, R, table, n_tiles, max_tiles, at<float>(ws, L.y_perm), s, mark)) !=
+    if ((st = run_routed_bs_after_quant(*d, *w, b, R, table, n_tiles, max_tiles, at<float>(ws, L.y_perm), s, mark)) !=
         MOE_OK)
       return st;
   } else {
@@ -1462,13 +1500,13 @@ moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const 
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   const int4* table = at<int4>(ws, L.tile_table);
   const int32_t* n_tiles = at<int32_t>(ws, L.num_tiles);
-  if (routed_a8(dr)) {
-    const A8Bufs b{at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.sfx), at<void>(ws, L.h), at<uint8_t>(ws, L.hq),
+  if (routed_bs(dr)) {
+    const BsBufs b{at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.sfx), at<void>(ws, L.h), at<uint8_t>(ws, L.hq),
                    at<uint8_t>(ws, L.sfh)};
-    if ((st = stage_quant_mx8(x_rows, n_rows, nullptr, table, n_tiles, L.max_tiles, d->L, b.xq, b.sfx, 180, s)) !=
+    if ((st = stage_quant_mx(dr, x_rows, n_rows, nullptr, table, n_tiles, L.max_tiles, d->L, b.xq, b.sfx, 180, s)) !=
         MOE_OK)
       return st;
-    return run_routed_a8_after_quant(dr, *w, b, n_rows, table, n_tiles, L.max_tiles, y_rows, s, [](int, int) {});
+    return run_routed_bs_after_quant(dr, *w, b, n_rows, table, n_tiles, L.max_tiles, y_rows, s, [](int, int) {});
   }
   st = stage_expert_gate_up(dr, *w, x_rows, table, n_tiles, at<void>(ws, L.h), s, L.max_tiles);
   if (st != MOE_OK) return st;
@@ -1477,18 +1515,12 @@ moe_status moe_expert_ffn_blocks(const moe_dims* d, const moe_weights* w, const 
 
 moe_status moe_mx8_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
                             moe_stream_t stream) {
-  if (rows < 0 || K <= 0 || K % 32 != 0 || rows > 0x7fffffffLL) return MOE_ERR_INVALID_ARG;
-  if (rows > 0 && (x == nullptr || codes == nullptr || scales == nullptr || !aligned16(x) || !aligned16(codes)))
-    return MOE_ERR_INVALID_ARG;
-  g_last_launches = 0;
-  if (rows == 0) return MOE_OK;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const long long tiles = cdiv(rows, 128);
-  const int grid = static_cast<int>(std::min<long long>(tiles, 8LL * num_sms()));
-  mx8_quant_tiles_kernel<<<grid, MX8_WARPS * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, nullptr, nullptr,
-                                                          nullptr, rows, K, codes, scales, 182);
-  g_last_launches = 1;
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return mx_quantize_rows(false, x, rows, K, codes, scales, stream, 182);
+}
+
+moe_status moe_mx4_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
+                            moe_stream_t stream) {
+  return mx_quantize_rows(true, x, rows, K, codes, scales, stream, 183);
 }
 
 moe_status moe_mx_tiled_scales_size(const moe_dims* d, size_t* gate_up_bytes, size_t* down_bytes) {

@@ -1,16 +1,22 @@
-// MXFP8 activations and scale-factor tiles for the block-scaled expert GEMMs.
+// MXFP8 / MXFP4 activations and scale-factor tiles for the block-scaled
+// expert GEMMs.
 //
-// Format (OCP Microscaling Formats v1.0, the format family of the routed
+// Formats (OCP Microscaling Formats v1.0, the format family of the routed
 // weights on page "ai-tech-express.jp" on K3, section "量子化を前提とした学習
 // 「MXFP4 Quantization-Aware Training」"; the pages give no activation format,
-// MXFP8 E4M3 is the library's reading): a row is cut into blocks of 32
-// consecutive elements along K; a block holds one E8M0 scale X = 2^s and 32
-// E4M3 codes q with value q * X.  The scale follows the spec's rule:
-//   s = floor(log2(max_i |v_i|)) - 8        (8 = largest E4M3 exponent)
+// MXFP8 E4M3 or MXFP4 E2M1 is the library's reading): a row is cut into
+// blocks of 32 consecutive elements along K; a block holds one E8M0 scale
+// X = 2^s and 32 element codes q with value q * X.  The scale follows the
+// spec's rule:
+//   s = floor(log2(max_i |v_i|)) - emax     (emax = largest element exponent:
+//                                            8 for E4M3, 2 for E2M1)
 // clamped to [-127, 127] (an all-zero block gets s = -127), and
-//   q_i = E4M3(v_i / X), rounded to nearest even, saturated to +-448.
-// Inputs are bf16, so v / X is exact in fp32 and the one rounding is the
-// conversion instruction's.
+//   q_i = element(v_i / X), rounded to nearest even, saturated to the
+//         largest finite element (+-448 for E4M3, +-6 for E2M1).
+// Inputs are bf16, so v / X is exact in fp32 (or below the smallest element
+// step, where it rounds to a signed zero either way) and the one rounding is
+// the conversion instruction's.  E4M3 codes take a byte each; E2M1 codes two
+// to a byte, the even element in the low nibble.
 //
 // Scale-factor tiles: the block-scaled MMA reads scales from tensor memory,
 // where tcgen05.cp puts them from shared memory in 512-byte atoms of 128 rows
@@ -28,7 +34,7 @@
 
 namespace moe {
 
-constexpr int MX8_WARPS = 8;
+constexpr int MXQ_WARPS = 8;
 
 // Byte offset of (tile row i, k-block b) in an activation scale tile.
 __device__ __forceinline__ long long mx8_sf_offset(long long tile, int nkb128, int i, int b) {
@@ -36,22 +42,48 @@ __device__ __forceinline__ long long mx8_sf_offset(long long tile, int nkb128, i
 }
 
 // E8M0 exponent s of a block whose largest |bf16| has bit pattern amax_bits
-// (sign cleared): floor(log2) is the bf16 exponent field - 127 (a subnormal or
-// zero maximum gives a value below -127, which the clamp absorbs).
-__device__ __forceinline__ int mx8_block_exponent(uint32_t amax_bits) {
+// (sign cleared), for elements whose largest exponent is emax: floor(log2) is
+// the bf16 exponent field - 127 (a subnormal or zero maximum gives a value
+// below -127, which the clamp absorbs).
+__device__ __forceinline__ int mx_block_exponent(uint32_t amax_bits, int emax) {
   if (amax_bits == 0u) return -127;
   const int e = static_cast<int>(amax_bits >> 7) - 127;
-  return max(-127, min(127, e - 8));
+  return max(-127, min(127, e - emax));
 }
 
-// 2^-s as fp32 for s in [-127, 119] (normal for every such s).
-__device__ __forceinline__ float mx8_inv_scale(int s) { return __int_as_float((127 - s) << 23); }
+// 2^-s as fp32 for s in [-127, 126] (normal for every such s).
+__device__ __forceinline__ float mx_inv_scale(int s) { return __int_as_float((127 - s) << 23); }
 
 // Two fp32 values -> E4M3 codes (round to nearest even, saturated), lo in the low byte.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Two fp32 values -> E2M1 codes (round to nearest even, saturated), lo in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Quantises 32 bf16 values (4 x uint4) with exponent s into 32 E2M1 codes (one uint4).
+__device__ __forceinline__ void mx4_encode32(const uint4 (&v)[4], float inv, uint4& out) {
+  uint32_t w[4];
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // words 4i .. 4i+3 hold elements 8i .. 8i+7, one byte of codes per word
+    uint32_t acc = 0u;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t a = u[4 * i + b];
+      acc |= e2m1x2(__uint_as_float(a << 16) * inv, __uint_as_float(a & 0xFFFF0000u) * inv) << (8 * b);
+    }
+    w[i] = acc;
+  }
+  out = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // Quantises 32 bf16 values (4 x uint4) with exponent s into 32 E4M3 codes (2 x uint4).
@@ -70,18 +102,20 @@ __device__ __forceinline__ void mx8_encode32(const uint4 (&v)[4], float inv, uin
   out[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// Quantises rows to MXFP8.  With a tile table (tiles != NULL): the rows of
-// the grouped-GEMM token tiles, row r (tile rows row0 .. row0 + ntok - 1)
-// reading source row src_row[r] (or r when src_row is NULL), scales written
-// into the tile's scale atoms.  Without one: rows 0 .. n_rows - 1 (src_row
-// ignored), scales row-major [n_rows, K/32].  Codes go to codes [r, K].  One
-// warp per row; lane j handles the blocks j, j + 32, ...  Source rows outside
+// Quantises rows to MXFP8 (FP4 = false) or MXFP4 (FP4 = true).  With a tile
+// table (tiles != NULL): the rows of the grouped-GEMM token tiles, row r
+// (tile rows row0 .. row0 + ntok - 1) reading source row src_row[r] (or r
+// when src_row is NULL), scales written into the tile's scale atoms.
+// Without one: rows 0 .. n_rows - 1 (src_row ignored), scales row-major
+// [n_rows, K/32].  Codes go to codes [r, K] (FP4: [r, K/2]).  One warp per
+// row; lane j handles the blocks j, j + 32, ...  Source rows outside
 // [0, src_rows) record `site` in the fault flag and are skipped.
-__global__ void __launch_bounds__(MX8_WARPS * 32)
-    mx8_quant_tiles_kernel(const __nv_bfloat16* __restrict__ src, long long src_rows,
-                           const int32_t* __restrict__ src_row, const int4* __restrict__ tiles,
-                           const int32_t* __restrict__ num_tiles, long long n_rows, int K,
-                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int site) {
+template <bool FP4>
+__global__ void __launch_bounds__(MXQ_WARPS * 32)
+    mx_quant_tiles_kernel(const __nv_bfloat16* __restrict__ src, long long src_rows,
+                          const int32_t* __restrict__ src_row, const int4* __restrict__ tiles,
+                          const int32_t* __restrict__ num_tiles, long long n_rows, int K,
+                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int site) {
   const bool tiled = tiles != nullptr;
   const long long nt = tiled ? num_tiles[0] : (n_rows + 127) / 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -89,7 +123,7 @@ __global__ void __launch_bounds__(MX8_WARPS * 32)
   for (long long t = blockIdx.x; t < nt; t += gridDim.x) {
     const int4 e = tiled ? tiles[t]
                          : make_int4(0, static_cast<int>(t * 128), static_cast<int>(min(128LL, n_rows - t * 128)), 0);
-    for (int i = warp; i < e.z; i += MX8_WARPS) {
+    for (int i = warp; i < e.z; i += MXQ_WARPS) {
       const long long r = static_cast<long long>(e.y) + i;
       const long long sr = tiled && src_row != nullptr ? static_cast<long long>(src_row[r]) : r;
       if (sr < 0 || sr >= src_rows) {
@@ -97,7 +131,7 @@ __global__ void __launch_bounds__(MX8_WARPS * 32)
         continue;
       }
       const uint4* s4 = reinterpret_cast<const uint4*>(src + sr * K);
-      uint4* c4 = reinterpret_cast<uint4*>(codes + r * K);
+      uint4* c4 = reinterpret_cast<uint4*>(codes + r * (FP4 ? K / 2 : K));
       for (int b = lane; b < nblk; b += 32) {
         uint4 v[4];
 #pragma unroll
@@ -106,11 +140,15 @@ __global__ void __launch_bounds__(MX8_WARPS * 32)
         const uint32_t* u = reinterpret_cast<const uint32_t*>(v);
 #pragma unroll
         for (int j = 0; j < 16; ++j) amax = max(amax, max(u[j] & 0x7FFFu, (u[j] >> 16) & 0x7FFFu));
-        const int sexp = mx8_block_exponent(amax);
-        uint4 q[2];
-        mx8_encode32(v, mx8_inv_scale(sexp), q);
-        c4[2 * b] = q[0];
-        c4[2 * b + 1] = q[1];
+        const int sexp = mx_block_exponent(amax, FP4 ? 2 : 8);
+        if constexpr (FP4) {
+          mx4_encode32(v, mx_inv_scale(sexp), c4[b]);
+        } else {
+          uint4 q[2];
+          mx8_encode32(v, mx_inv_scale(sexp), q);
+          c4[2 * b] = q[0];
+          c4[2 * b + 1] = q[1];
+        }
         sf[tiled ? mx8_sf_offset(t, nkb128, i, b) : r * nblk + b] = static_cast<uint8_t>(sexp + 127);
       }
     }

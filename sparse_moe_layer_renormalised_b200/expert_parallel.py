@@ -37,7 +37,7 @@ import torch
 import torch.distributed as dist
 
 from .layer import tile_weight_scales
-from ._binding import (Dims, check, make_weights, moe_combine, moe_expert_ffn_blocks,
+from ._binding import (BLOCK_SCALED, Dims, check, make_weights, moe_combine, moe_expert_ffn_blocks,
                        moe_expert_ffn_blocks_workspace_size, moe_latent_shared, moe_output, moe_permute,
                        moe_router_topk, moe_workspace_size)
 
@@ -138,7 +138,7 @@ class ExpertParallelMoeLayer:
     dims: the full layer (E = all routed experts).  weights: device tensors
     named as moe_weights' fields; Wg / Wv / Wo (and Sg / Sv / So for MXFP4)
     hold only this rank's experts, bounds[rank] .. bounds[rank+1]-1, in order.
-    With routed = "mxfp4_a8" the dispatched rows stay bf16 and the receiving
+    With a block-scaled routed type ("mxfp4_a8", "mxfp4_a4") the dispatched rows stay bf16 and the receiving
     rank quantises them (moe_expert_ffn_blocks).
     max_tokens sizes the local workspaces."""
 
@@ -153,7 +153,7 @@ class ExpertParallelMoeLayer:
             raise ValueError(f"rank {self.rank} holds {weights['Wg'].shape[0]} experts, expected {self.e_local}")
         self.local_dims = replace(dims, E=self.e_local)
         self.weights = dict(weights)
-        if dims.routed == "mxfp4_a8" and "Sgv_tiled" not in weights:
+        if dims.routed in BLOCK_SCALED and "Sgv_tiled" not in weights:
             # the block-scaled experts read their scales in tiled order, made once per rank
             self.weights.update(tile_weight_scales(self.local_dims, weights["Sg"], weights["Sv"], weights["So"]))
         self._w = make_weights(**self.weights)

@@ -7,7 +7,7 @@ from dataclasses import replace
 
 import torch
 
-from ._binding import (Dims, check, make_aux, make_weights, moe_layer_forward, moe_mx_tile_scales,
+from ._binding import (BLOCK_SCALED, Dims, check, make_aux, make_weights, moe_layer_forward, moe_mx_tile_scales,
                        moe_mx_tiled_scales_size, moe_workspace_size)
 
 _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -28,8 +28,8 @@ def tile_weight_scales(dims: Dims, Sg: torch.Tensor, Sv: torch.Tensor, So: torch
 class MoeLayer:
     """Weights: dict with Wr, bias, Wdown, Wup, gamma, Wg, Wv, Wo, Wsg, Wsv, Wso
     and, for MXFP4 routed weights, Sg, Sv, So (device tensors in the shapes of
-    include/moe.h).  With routed = "mxfp4_a8" (block-scaled MXFP8 x MXFP4
-    experts) the scales are re-ordered once here by moe_mx_tile_scales into
+    include/moe.h).  With routed = "mxfp4_a8" or "mxfp4_a4" (block-scaled
+    MXFP4 weights x MXFP8 / MXFP4 inputs) the scales are re-ordered once here by moe_mx_tile_scales into
     Sgv_tiled / So_tiled, which the layer keeps.  max_tokens sizes the
     workspace; each call may use any T <= max_tokens."""
 
@@ -38,7 +38,7 @@ class MoeLayer:
         self.weights = dict(weights)
         self.max_tokens = dims.T if max_tokens is None else max_tokens
         dev = weights["Wr"].device
-        if dims.routed == "mxfp4_a8" and "Sgv_tiled" not in weights:
+        if dims.routed in BLOCK_SCALED and "Sgv_tiled" not in weights:
             self.weights.update(tile_weight_scales(dims, weights["Sg"], weights["Sv"], weights["So"]))
         self._w = make_weights(**self.weights)
         nbytes = moe_workspace_size(replace(dims, T=self.max_tokens))

@@ -25,7 +25,7 @@ def _dims(**kw):
 
 def test_library_exports_every_declared_symbol():
     names = _declared()
-    assert len(names) == 21
+    assert len(names) == 22
     lib = ctypes.CDLL(moe.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -64,6 +64,8 @@ FAKE = 1 << 20  # an aligned address; never dereferenced because validation fail
     (dict(routed="mxfp4", act="f32", y_out="f32"), moe.MOE_ERR_UNSUPPORTED),
     (dict(routed="mxfp4_a8"), moe.MOE_ERR_UNSUPPORTED),  # I = 768 not a multiple of 512
     (dict(routed="mxfp4_a8", I=1024, act="f32", y_out="f32"), moe.MOE_ERR_UNSUPPORTED),
+    (dict(routed="mxfp4_a4"), moe.MOE_ERR_UNSUPPORTED),  # I = 768 not a multiple of 512
+    (dict(routed="mxfp4_a4", I=1024, act="f32", y_out="f32"), moe.MOE_ERR_UNSUPPORTED),
     (dict(H=2056), moe.MOE_ERR_UNSUPPORTED),
     (dict(S=4), moe.MOE_ERR_UNSUPPORTED),
 ])
@@ -158,14 +160,17 @@ def test_stage_entry_points_validate_before_launching():
     assert moe.moe_expert_ffn_blocks(d, w, FAKE, -1, FAKE, 4, FAKE, FAKE, n) == moe.MOE_ERR_INVALID_ARG
 
 
-def test_block_scaled_path_validates():
-    """routed = mxfp4_a8 needs the tiled weight scales and 32-byte aligned
-    codes; tiled scales on any other path are rejected; the size query and the
-    tiling and quantiser entries validate on the host."""
+@pytest.mark.parametrize("routed", ["mxfp4_a8", "mxfp4_a4"])
+def test_block_scaled_path_validates(routed):
+    """The block-scaled routed types need the tiled weight scales and 32-byte
+    aligned codes; tiled scales on any other path are rejected; the size query
+    and the tiling and quantiser entries validate on the host."""
     full = {f: FAKE for f in ("Wr", "bias", "Wdown", "Wup", "gamma", "Wg", "Wv", "Wo", "Wsg", "Wsv", "Wso")}
-    d8 = _dims(I=1024, routed="mxfp4_a8")
+    d8 = _dims(I=1024, routed=routed)
     ws8 = moe.moe_workspace_size(d8)
-    assert ws8 > moe.moe_workspace_size(_dims(I=1024, routed="mxfp4"))  # + E4M3 h and the scale tiles
+    assert ws8 > moe.moe_workspace_size(_dims(I=1024, routed="mxfp4"))  # + the codes of h and the scale tiles
+    if routed == "mxfp4_a4":  # h's codes take half the bytes of the MXFP8 path's
+        assert ws8 < moe.moe_workspace_size(_dims(I=1024, routed="mxfp4_a8"))
     tiled = dict(Sgv_tiled=FAKE, So_tiled=FAKE)
     call = lambda w: moe.moe_layer_forward(d8, moe.make_weights(**w), FAKE, FAKE, None, FAKE, ws8, 0)  # noqa: E731
     assert call(full) == moe.MOE_ERR_INVALID_ARG                                  # no tiled scales
@@ -176,17 +181,18 @@ def test_block_scaled_path_validates():
     wm = moe.make_weights(**{**full, "Sg": FAKE, "Sv": FAKE, "So": FAKE, **tiled})
     assert moe.moe_layer_forward(dm, wm, FAKE, FAKE, None, FAKE, wsm, 0) == moe.MOE_ERR_INVALID_ARG
     # sizes of the tiled scales equal those of the row-major ones
-    k3 = _dims(H=7168, L=3584, E=896, k=16, I=3072, routed="mxfp4_a8")
+    k3 = _dims(H=7168, L=3584, E=896, k=16, I=3072, routed=routed)
     st, gu, dn = moe.moe_mx_tiled_scales_size(k3)
     assert st == moe.MOE_OK and gu == 896 * 3072 * 3584 // 16 and dn == 896 * 3584 * 3072 // 32
     assert moe.moe_mx_tiled_scales_size(_dims())[0] == moe.MOE_ERR_UNSUPPORTED
     assert moe.moe_mx_tile_scales(k3, FAKE, None, FAKE, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_mx_tile_scales(k3, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
-    # the stand-alone quantiser
-    assert moe.moe_mx8_quantize(FAKE, 4, 48, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG   # K % 32
-    assert moe.moe_mx8_quantize(FAKE + 8, 4, 64, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
-    assert moe.moe_mx8_quantize(None, 4, 64, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
-    assert moe.moe_mx8_quantize(None, 0, 64, None, None, 0) == moe.MOE_OK               # nothing to do
+    # the stand-alone quantisers
+    for q in (moe.moe_mx8_quantize, moe.moe_mx4_quantize):
+        assert q(FAKE, 4, 48, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG   # K % 32
+        assert q(FAKE + 8, 4, 64, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+        assert q(None, 4, 64, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+        assert q(None, 0, 64, None, None, 0) == moe.MOE_OK               # nothing to do
 
 
 def test_structs_keep_their_tensors_alive():

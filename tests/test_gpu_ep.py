@@ -13,7 +13,7 @@ import torch.distributed as dist
 import gen
 import oracle
 import sparse_moe_layer_renormalised_b200 as moe
-from harness import TOL_BF16, dims_for, oracle_forward, parity
+from harness import TOL_BF16, TOL_MXFP4_A4, TOL_RMS_A4, dims_for, oracle_forward, parity, rms_parity
 from oracle import inputs as oin
 from sparse_moe_layer_renormalised_b200 import expert_parallel as ep
 from sparse_moe_layer_renormalised_b200.layer import tile_weight_scales
@@ -27,7 +27,8 @@ def _no_fault():
     assert st == moe.MOE_OK and code == 0, f"device fault {code}"
 
 
-@pytest.mark.parametrize("name,lo,hi", [("mid", 40, 104), ("mxfp4-small", 0, 64), ("mxfp4a8-small", 8, 40)])
+@pytest.mark.parametrize("name,lo,hi", [("mid", 40, 104), ("mxfp4-small", 0, 64), ("mxfp4a8-small", 8, 40),
+                                         ("mxfp4a4-small", 8, 40)])
 def test_expert_ffn_blocks_three_sources(name, lo, hi):
     """Rows of experts lo..hi-1 from three 'sources' (each expert-major), as
     an expert-parallel rank receives them; every row against the oracle."""
@@ -44,12 +45,12 @@ def test_expert_ffn_blocks_three_sources(name, lo, hi):
     offs = np.stack(blocks).astype(np.int32)
     expert_of_row = np.concatenate([np.repeat(np.arange(lo, hi), np.diff(b)) for b in blocks])
     x = torch.randn(rows, cfg.L, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
-    mx = cfg.routed in ("mxfp4", "mxfp4_a8")
+    mx = cfg.routed in ("mxfp4",) + moe.BLOCK_SCALED
     names = ("Wg", "Wv", "Wo") + (("Sg", "Sv", "So") if mx else ())
     wl = {n: w[n][lo:hi].contiguous() for n in names}
     d = moe.Dims(T=rows, H=cfg.H, L=cfg.L, E=E_loc, k=1, I=cfg.I, S=cfg.S, Is=cfg.Is, act=cfg.act,
                  routed=cfg.routed)
-    if cfg.routed == "mxfp4_a8":
+    if cfg.routed in moe.BLOCK_SCALED:
         wl.update(tile_weight_scales(d, wl.pop("Sg"), wl.pop("Sv"), wl.pop("So")))
     ws = torch.empty(moe.moe_expert_ffn_blocks_workspace_size(d, rows, 3), dtype=torch.uint8, device="cuda")
     y = torch.full((rows, cfg.L), float("nan"), dtype=torch.float32, device="cuda")
@@ -63,7 +64,11 @@ def test_expert_ffn_blocks_three_sources(name, lo, hi):
         r = torch.as_tensor(np.nonzero(expert_of_row == e)[0])
         ref[r] = oracle.expert_forward(xf[r], *oin.expert_weights_raw(cfg, int(e)), cfg.situ_c, oracle.bf16_round,
                                        act=oracle.routed_act(cfg))
-    assert parity(y.cpu().to(F64), ref) <= 1e-2
+    if cfg.routed == "mxfp4_a4":  # h's E2M1 codes can flip (bars derived in harness.py)
+        assert parity(y.cpu().to(F64), ref) <= TOL_MXFP4_A4
+        assert rms_parity(y.cpu().to(F64), ref) <= TOL_RMS_A4
+    else:
+        assert parity(y.cpu().to(F64), ref) <= 1e-2
 
 
 def _free_port():
