@@ -30,13 +30,21 @@
 //    memory; with three, the copier can put stage g's scales in the tensor
 //    pipe's queue ahead of stage g-1's MMAs.
 // With A4 both operands are packed E2M1 codes (two per byte, the even
-// element in the low nibble), which kind::mxf4 reads as they are: a stage's
-// K = 256 is one 128-byte wide box per operand (plain byte TMA, 128-byte
-// swizzle) and 4 MMAs of K = 64, each taking two scale bytes (j = 0 or 2) of
-// the same scale columns; stages are half the size, so there are five.
+// element in the low nibble), which kind::mxf4 reads as they are: a 128-byte
+// wide box (plain byte TMA, 128-byte swizzle) holds K = 256, and a stage
+// covers K = 512 in two such slices, 8 MMAs of K = 64, each taking two scale
+// bytes (j = 0 or 2) of one 128-wide K chunk's scale columns.  K = 512 per
+// stage halves the per-stage waits, copies and commits of the single-thread
+// roles against K = 256 (measured on B200: at K = 256 the all-4-bit stage
+// took ~1500 cycles with the tensor pipe 21% busy).  Its token box is at most
+// 104 rows per CTA (the tile's half), so that three stages fit; its four
+// chunks' scales take 48 tensor-memory columns per buffer, so two buffers.
 // Warp roles: 0 TMA producer (both CTAs), 1 TMEM owner and MMA issuer (even
-// CTA), 2-5 epilogue (both CTAs), 6 scale copier (even CTA).  Every wait is
-// bounded.
+// CTA), 2-5 and 7-10 epilogue (both CTAs), 6 scale copier (even CTA).  The
+// two epilogue sets of four warps (one per tensor-memory lane quarter each)
+// drain alternate 32-token chunks of an accumulator: measured on B200, one set
+// left the MMA waiting for accumulators (the SiTU epilogue's latency per chunk
+// exceeded the next item's MMA and load time).  Every wait is bounded.
 #pragma once
 
 #include "gemm_expert.cuh"
@@ -44,43 +52,53 @@
 
 namespace moe {
 
-constexpr int BS_BK = 256;                         // K elements per stage: two halves of 128, 8 MMAs of K = 32
-constexpr uint32_t BS_HALF_BYTES = 128 * 128;      // a 128-row x 128-element half tile (one byte per code slot)
-constexpr uint32_t BS_A_BYTES = 2 * BS_HALF_BYTES;  // 128 weight rows
-constexpr uint32_t BS_A_TX = 128 * BS_BK / 2;      // bytes the A tile's TMA completes (packed codes)
-constexpr uint32_t BS_B_BYTES = 2 * BS_HALF_BYTES;  // up to 128 token rows of E4M3 codes per CTA
-constexpr uint32_t BS_SFA_BYTES = 1024;            // two scale atoms (128 weight rows x 4 k-blocks each)
-constexpr uint32_t BS_SFB_BYTES = 2048;            // two K halves x (token rows 0-127, 128-255)
-constexpr int BS_STAGES = 3;
+constexpr uint32_t BS_SLICE_BYTES = 128 * 128;    // 128 weight rows x one 128-byte wide slice of K
 constexpr int BS_MAX_TILE_ROWS = 208;              // largest token tile (MMA N)
 constexpr uint32_t BS_ACC_COLS = BS_MAX_TILE_ROWS;
-constexpr uint32_t BS_SF_COL = 2 * BS_ACC_COLS;    // three scale buffers of 24 columns from here
-constexpr int BS_SF_BUFS = 3;
-constexpr uint32_t BS_SF_BUF_COLS = 24;            // SFA half 0 / 1 at +0 / +4, SFB half 0 / 1 at +8 / +16
-constexpr int BS_THREADS = 224;
+constexpr uint32_t BS_SF_COL = 2 * BS_ACC_COLS;    // the scale buffers from here
+constexpr int BS_THREADS = 352;
 constexpr int BS_COPY_WARP = 6;
-static_assert(BS_SF_COL + BS_SF_BUFS * BS_SF_BUF_COLS <= 2 * EX_ACC_COLS, "tensor memory columns");
+constexpr int BS_EPI_SET1_WARP = 7;                // warps 7-10: the second epilogue set
 
-// Stage geometry of the two activation formats.
+// Stage geometry.  A stage is two 128-byte wide K slices per operand (A8: K =
+// 128 E4M3 codes, or E2M1 codes spread one per byte, per slice; A4: K = 256
+// packed E2M1 codes per slice), four MMAs per slice, and the scales of its
+// 128-wide K chunks (A8: 2, A4: 4): per chunk one 512-byte atom of the CTA's
+// weight rows and two of the token tile's rows (0-127, 128-255).  In a scale
+// buffer chunk q's weight scales sit at column +4q and its token scales at
+// +SFB_COL + 8q (rows 128-255 at +4 more).
 template <bool A4>
 struct BsStage {
-  static constexpr uint32_t A_BYTES = A4 ? BS_HALF_BYTES : BS_A_BYTES;  // packed codes: 128 rows x 128 bytes
-  static constexpr uint32_t B_BYTES = A4 ? BS_HALF_BYTES : BS_B_BYTES;
-  static constexpr int STAGES = A4 ? 5 : BS_STAGES;
-  static constexpr uint32_t BYTES = A_BYTES + B_BYTES + BS_SFA_BYTES + BS_SFB_BYTES;
+  static constexpr int K = A4 ? 512 : 256;                  // K elements per stage
+  static constexpr int CHUNKS = K / 128;                    // 128-wide K chunks (scale atoms) per stage
+  static constexpr uint32_t A_BYTES = 2 * BS_SLICE_BYTES;   // 128 weight rows
+  static constexpr uint32_t A_TX = 128 * K / 2;             // bytes the A tile's TMA completes (packed codes)
+  static constexpr int B_MAX_ROWS = A4 ? 104 : 128;         // token rows of this CTA's largest box
+  static constexpr uint32_t B_SLICE = B_MAX_ROWS * 128;     // (a multiple of 1024: the swizzle atom)
+  static constexpr uint32_t B_BYTES = 2 * B_SLICE;
+  static constexpr uint32_t SFA_BYTES = CHUNKS * 512;
+  static constexpr uint32_t SFB_BYTES = CHUNKS * 1024;
+  static constexpr int STAGES = 3;
+  static constexpr int SF_BUFS = A4 ? 2 : 3;
+  static constexpr uint32_t SFB_COL = 4 * CHUNKS;
+  static constexpr uint32_t SF_BUF_COLS = 12 * CHUNKS;
+  static constexpr uint32_t BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * BYTES + EX_XCH_BYTES + 512;
   static_assert(SMEM <= 232448, "shared memory per CTA");
-  static_assert(STAGES >= BS_SF_BUFS, "the scale copier's reuse wait assumes a stage per scale buffer at least");
+  static_assert(B_SLICE % 1024 == 0, "token slices start on a swizzle atom");
+  static_assert(2 * B_MAX_ROWS >= BS_MAX_TILE_ROWS, "a CTA's box covers its half of the largest tile");
+  static_assert(BS_SF_COL + SF_BUFS * SF_BUF_COLS <= 2 * EX_ACC_COLS, "tensor memory columns");
+  static_assert(STAGES >= SF_BUFS, "the scale copier's reuse wait assumes a stage per scale buffer at least");
 };
 
 struct BsMaps {
   CUtensorMap a0;    // E2M1 codes (A8: 16 per 16-byte slot; A4: packed bytes, 128-byte wide boxes):
                      //   PAIRED W_g [E*I, L] (64-row boxes), else W_o [E*L, I] (128-row)
   CUtensorMap a1;    // PAIRED: W_v, as a0
-  CUtensorMap sa;    // weight scale tiles as [n, 16] bytes, 64-row (two atoms, 1 KB) boxes
+  CUtensorMap sa;    // weight scale tiles as [n, 16] bytes, boxes of a stage's atoms (SFA_BYTES)
   CUtensorMap b[4];  // activation codes (A8: E4M3 [R, K]; A4: packed E2M1 [R, K/2] bytes): 128-byte
-                     //   wide boxes of 128, 64, 32, 16 rows, 128-byte swizzle
-  CUtensorMap sb;    // activation scale tiles as [n, 16] bytes, 128-row (two K chunks x two atoms, 2 KB) boxes
+                     //   wide boxes of B_MAX_ROWS, 64, 32, 16 rows, 128-byte swizzle
+  CUtensorMap sb;    // activation scale tiles as [n, 16] bytes, boxes of a stage's atoms (SFB_BYTES)
 };
 
 // Shared-memory descriptor of a scale atom for tcgen05.cp: 32 rows of 16
@@ -175,6 +193,18 @@ __device__ __forceinline__ ExTile bs_decode(int w, int num_tiles, int num_multi,
   return t;
 }
 
+// Named barriers of the epilogue: ids 1-4 for the two warps of a column pair
+// (g quarter q, v quarter q + 2) of set es, ids 5-6 for all four warps of a set
+// (aligned barriers: the warp reconverges first).
+__device__ __forceinline__ void bs_pair_bar(int es, int pair_q) {
+  __syncwarp();
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + 2 * es + pair_q) : "memory");
+}
+__device__ __forceinline__ void bs_set_bar(int es) {
+  __syncwarp();
+  asm volatile("bar.sync %0, 128;" ::"r"(5 + es) : "memory");
+}
+
 template <int EPI, bool PAIRED, bool A4>
 __global__ void __launch_bounds__(BS_THREADS, 1)
     tc_expert_bs_kernel(const __grid_constant__ BsMaps maps, const ExParams p) {
@@ -186,8 +216,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + kStages * G::A_BYTES;
   uint8_t* sSA = sB + kStages * G::B_BYTES;
-  uint8_t* sSB = sSA + kStages * BS_SFA_BYTES;
-  float* xch = reinterpret_cast<float*>(sSB + kStages * BS_SFB_BYTES);
+  uint8_t* sSB = sSA + kStages * G::SFA_BYTES;
+  float* xch = reinterpret_cast<float*>(sSB + kStages * G::SFB_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + EX_XCH_BYTES);
   uint64_t* empty = full + kStages;
   uint64_t* sf_full = empty + kStages;  // the stage's scales are in tensor memory (even CTA)
@@ -197,7 +227,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   uint64_t* copy_drain = drain + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(copy_drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* epi_ok = abort + 1;
+  volatile int* epi_ok = abort + 1;  // [2]: accumulator-ready verdict of each epilogue set
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -214,7 +244,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4 * CG);
+      mbar_init(&acc_empty[a], 8 * CG);  // both epilogue sets' warps, in both CTAs
     }
     mbar_init(drain, 1);
     mbar_init(copy_drain, 1);
@@ -238,7 +268,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   const int num_multi = p.num_tiles_dev[1];
   const int total = num_tiles * p.n_wtiles;
   const int n_stages = p.num_k_blocks;  // stages of K = 256 per item
-  const int nkb128 = 2 * p.num_k_blocks;  // 128-wide K chunks per row (scale-tile indexing)
+  const int nkb128 = G::CHUNKS * p.num_k_blocks;  // 128-wide K chunks per row (scale-tile indexing)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (both CTAs)
@@ -252,10 +282,10 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
         const ExTile t = bs_decode(w, num_tiles, num_multi, p, true);
         const int rows_cta = t.n_mma / 2;  // token rows this CTA stages
         const int bsel = rows_cta > 64 ? 0 : rows_cta > 32 ? 1 : rows_cta > 16 ? 2 : 3;
-        const int brows = 128 >> bsel;
+        const int brows = bsel == 0 ? G::B_MAX_ROWS : 128 >> bsel;
         const int tok0 = t.row0 + static_cast<int>(rank) * rows_cta;
-        const uint32_t b_tx = (A4 ? 1u : 2u) * static_cast<uint32_t>(brows) * 128u;
-        const uint32_t bytes = static_cast<uint32_t>(CG) * (BS_A_TX + b_tx + BS_SFA_BYTES + BS_SFB_BYTES);
+        const uint32_t bytes = static_cast<uint32_t>(CG) * (G::A_TX + 2u * static_cast<uint32_t>(brows) * 128u +
+                                                            G::SFA_BYTES + G::SFB_BYTES);
         const int wrow = t.expert * p.w_rows_per_expert + (PAIRED ? t.wt * 128 : t.wt * 256) +
                          static_cast<int>(rank) * (PAIRED ? 64 : 128);
         // 16-byte rows of the scale tiles: 32 per atom
@@ -269,33 +299,23 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* a_dst = sA + stage * G::A_BYTES;
           uint8_t* b_dst = sB + stage * G::B_BYTES;
-          if constexpr (A4) {
-            // one 128-byte (256-code) wide box per operand; x in bytes
-            const int kc = kb * 128;
-            if (kExL2Hints && !t.multi) {
-              ex_tma_load_hint<CG>(a_dst, &maps.a0, &full[stage], kc, wrow, pol_w);
-              if (PAIRED) ex_tma_load_hint<CG>(a_dst + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
-            } else {
-              ex_tma_load<CG>(a_dst, &maps.a0, &full[stage], kc, wrow);
-              if (PAIRED) ex_tma_load<CG>(a_dst + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
-            }
-            ex_tma_load_hint<CG>(b_dst, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
-          } else
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int kc = kb * BS_BK + h * 128;
-            uint8_t* ah = a_dst + h * BS_HALF_BYTES;
+            // slice h: x = 128 E4M3 codes / spread E2M1 codes (A8) or 128
+            // bytes of packed E2M1 codes (A4), 256 per stage either way
+            const int kc = kb * 256 + h * 128;
+            uint8_t* ah = a_dst + h * BS_SLICE_BYTES;
             if (kExL2Hints && !t.multi) {
               ex_tma_load_hint<CG>(ah, &maps.a0, &full[stage], kc, wrow, pol_w);
-              if (PAIRED) ex_tma_load_hint<CG>(ah + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
+              if (PAIRED) ex_tma_load_hint<CG>(ah + BS_SLICE_BYTES / 2, &maps.a1, &full[stage], kc, wrow, pol_w);
             } else {
               ex_tma_load<CG>(ah, &maps.a0, &full[stage], kc, wrow);
-              if (PAIRED) ex_tma_load<CG>(ah + BS_HALF_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
+              if (PAIRED) ex_tma_load<CG>(ah + BS_SLICE_BYTES / 2, &maps.a1, &full[stage], kc, wrow);
             }
-            ex_tma_load_hint<CG>(b_dst + h * BS_HALF_BYTES, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
+            ex_tma_load_hint<CG>(b_dst + h * G::B_SLICE, &maps.b[bsel], &full[stage], kc, tok0, pol_t);
           }
-          ex_tma_load<CG>(sSA + stage * BS_SFA_BYTES, &maps.sa, &full[stage], 0, sa_row0 + kb * 64);
-          ex_tma_load<CG>(sSB + stage * BS_SFB_BYTES, &maps.sb, &full[stage], 0, sb_row0 + kb * 128);
+          ex_tma_load<CG>(sSA + stage * G::SFA_BYTES, &maps.sa, &full[stage], 0, sa_row0 + kb * (G::SFA_BYTES / 16));
+          ex_tma_load<CG>(sSB + stage * G::SFB_BYTES, &maps.sb, &full[stage], 0, sb_row0 + kb * (G::SFB_BYTES / 16));
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -318,7 +338,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t g = 0;  // stages consumed so far
-      uint32_t sf_buf = 0;  // scale buffer of stage g (g mod BS_SF_BUFS)
+      uint32_t sf_buf = 0;  // scale buffer of stage g (g mod SF_BUFS)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -334,31 +354,28 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * BS_SF_BUF_COLS;
-          if (++sf_buf == BS_SF_BUFS) sf_buf = 0;
+          const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * G::SF_BUF_COLS;
+          if (++sf_buf == G::SF_BUFS) sf_buf = 0;
           const uint32_t a_addr = smem_u32(sA + stage * G::A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * G::B_BYTES);
-          if constexpr (A4) {
-            // MMA kk covers K = 64 kk .. 64 kk + 63: 32-blocks 2kk, 2kk + 1, i.e.
-            // scale bytes 2 (kk % 2), +1 of the atoms of K chunk kk / 2
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t j = 2u * static_cast<uint32_t>(kk & 1);
-              const uint32_t h = static_cast<uint32_t>(kk >> 1);
-              bs_mma4(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32),
-                      idesc0 | (j << 4) | (j << 29), (sf + 4u * h) | (j << 30), (sf + 8u + 8u * h) | (j << 30),
-                      (kb | kk) != 0 ? 1u : 0u);
-            }
-          } else
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t j = static_cast<uint32_t>(kk);  // scale byte of this K = 32 step
+              // MMA kk of slice h starts 32 bytes into the slice per step.  A8:
+              // K = 32, the 32-block kk of chunk h (scale byte kk).  A4: K = 64,
+              // 32-blocks 2 (kk % 2), +1 of chunk 2h + kk / 2 (bytes j, j + 1).
+              const uint32_t q = A4 ? 2u * h + (kk >> 1) : static_cast<uint32_t>(h);
+              const uint32_t j = A4 ? 2u * (kk & 1) : static_cast<uint32_t>(kk);
               const uint32_t id = idesc0 | (j << 4) | (j << 29);
-              bs_mma(d_tmem, sw128_kmajor_desc(a_addr + h * BS_HALF_BYTES + kk * 32),
-                     sw128_kmajor_desc(b_addr + h * BS_HALF_BYTES + kk * 32), id, (sf + 4u * h) | (j << 30),
-                     (sf + 8u + 8u * h) | (j << 30), (kb | h | kk) != 0 ? 1u : 0u);
+              const uint64_t ad = sw128_kmajor_desc(a_addr + h * BS_SLICE_BYTES + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(b_addr + h * G::B_SLICE + kk * 32);
+              const uint32_t sfa = (sf + 4u * q) | (j << 30), sfb = (sf + G::SFB_COL + 8u * q) | (j << 30);
+              const uint32_t accum = (kb | h | kk) != 0 ? 1u : 0u;
+              if constexpr (A4)
+                bs_mma4(d_tmem, ad, bd, id, sfa, sfb, accum);
+              else
+                bs_mma(d_tmem, ad, bd, id, sfa, sfb, accum);
             }
           ex_commit<CG>(&empty[stage]);
           if (++stage == kStages) {
@@ -387,7 +404,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t g = 0;
-      int prev2_stage = 0;        // stage of g - BS_SF_BUFS (its MMAs used the same scale buffer)
+      int prev2_stage = 0;        // stage of g - SF_BUFS (its MMAs used the same scale buffer)
       uint32_t prev2_phase = 0;
       uint32_t sf_buf = 0;
       bool ok = true;
@@ -399,7 +416,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             ok = false;
             break;
           }
-          if (g >= static_cast<uint32_t>(BS_SF_BUFS)) {
+          if (g >= static_cast<uint32_t>(G::SF_BUFS)) {
             if (!mbar_wait(&empty[prev2_stage], prev2_phase, abort, p.fault_site + 8)) {
               ok = false;
               break;
@@ -410,15 +427,15 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             }
           }
           tc_fence_after();
-          const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * BS_SF_BUF_COLS;
-          if (++sf_buf == BS_SF_BUFS) sf_buf = 0;
-          const uint8_t* sa = sSA + stage * BS_SFA_BYTES;
-          const uint8_t* sb = sSB + stage * BS_SFB_BYTES;
+          const uint32_t sf = tmem_base + BS_SF_COL + sf_buf * G::SF_BUF_COLS;
+          if (++sf_buf == G::SF_BUFS) sf_buf = 0;
+          const uint8_t* sa = sSA + stage * G::SFA_BYTES;
+          const uint8_t* sb = sSB + stage * G::SFB_BYTES;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            bs_copy_sf(sf + 4u * h, sf_atom_desc(smem_u32(sa + h * 512)));
-            bs_copy_sf(sf + 8u + 8u * h, sf_atom_desc(smem_u32(sb + h * 1024)));
-            if (two_atoms) bs_copy_sf(sf + 12u + 8u * h, sf_atom_desc(smem_u32(sb + h * 1024 + 512)));
+          for (int q = 0; q < G::CHUNKS; ++q) {
+            bs_copy_sf(sf + 4u * q, sf_atom_desc(smem_u32(sa + q * 512)));
+            bs_copy_sf(sf + G::SFB_COL + 8u * q, sf_atom_desc(smem_u32(sb + q * 1024)));
+            if (two_atoms) bs_copy_sf(sf + G::SFB_COL + 4u + 8u * q, sf_atom_desc(smem_u32(sb + q * 1024 + 512)));
           }
           // the MMA thread waits on this instead of full[]: data and scales are in place
           asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -440,17 +457,20 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int es = warp >= BS_EPI_SET1_WARP ? 1 : 0;  // epilogue set: chunks es, es + 2, ...
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(&acc_empty[0]), 0u);
     int acc = 0;
     uint32_t acc_phase = 0;
-    int xbuf = 0;
     for (int w = pair; w < total; w += npairs) {
       const ExTile t = bs_decode(w, num_tiles, num_multi, p, false);
       bool got;
       if constexpr (PAIRED) {
-        if (threadIdx.x == 64) *epi_ok = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
-        epilogue_bar();
-        got = *epi_ok != 0;
+        // one thread of the set waits; the set's barrier before the write keeps
+        // the previous verdict until every thread has read it
+        bs_set_bar(es);
+        if (lane == 0 && q == (es ? 3 : 2)) epi_ok[es] = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
+        bs_set_bar(es);
+        got = epi_ok[es] != 0;
       } else {
         got = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6));
       }
@@ -459,19 +479,21 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc) * BS_ACC_COLS;
       const int nch = (t.ntok + 31) >> 5;
       if constexpr (PAIRED) {
-        // warps 0,1 hold g and warps 2,3 hold v for intermediate columns
+        // quarters 0,1 hold g and 2,3 hold v for intermediate columns
         // base + 32 * (q & 1) + lane; g warps form tokens 0-15 of a chunk,
-        // v warps tokens 16-31, after swapping the other half.
+        // v warps tokens 16-31, after swapping the other half through this
+        // set's exchange buffer (the two warps of a column pair sync alone).
         const bool is_g = q < 2;
         const int col = t.wt * 128 + static_cast<int>(rank) * 64 + (q & 1) * 32 + lane;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const float c = p.situ_c;
         const float inv_c = 1.0f / c;
+        float* X = xch + es * EX_XCH_FLOATS + (q & 1) * 1024;
 #pragma unroll 1
-        for (int ch = 0; ch < nch; ++ch) {
+        for (int ch = es; ch < nch; ch += 2) {
           float r[32];
           bs_load_chunk(tbase, ch, t.ntok, r);
-          float* X = xch + xbuf * EX_XCH_FLOATS + (q & 1) * 1024;
+          bs_pair_bar(es, q & 1);  // the partner has read the previous chunk's half
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             if (is_g)
@@ -479,7 +501,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             else
               X[512 + i * 32 + lane] = r[i];
           }
-          epilogue_bar();
+          bs_pair_bar(es, q & 1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float g = is_g ? r[i] : X[i * 32 + lane];
@@ -488,13 +510,12 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             if (tok < t.ntok && col < p.out_cols)
               out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = __float2bfloat16_rn(situ_glu_fast(g, v, c, inv_c));
           }
-          xbuf ^= 1;
         }
       } else {
         const int col = t.wt * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
         float* out = reinterpret_cast<float*>(p.out);
 #pragma unroll 1
-        for (int ch = 0; ch < nch; ++ch) {
+        for (int ch = es; ch < nch; ch += 2) {
           float r[32];
           bs_load_chunk(tbase, ch, t.ntok, r);
 #pragma unroll

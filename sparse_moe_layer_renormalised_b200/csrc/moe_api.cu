@@ -744,29 +744,33 @@ moe_status stage_expert_bs(const moe_dims& d, bool paired, const moe_weights& w,
   const uint64_t wrows = static_cast<uint64_t>(d.E) * out_rows;
   const size_t sa_bytes = paired ? tiled_scales_gate_up(d) : tiled_scales_down(d);
   bool ok = true;
-  // scale tiles as 16-byte rows: weight boxes of two atoms (two 128-wide K
-  // chunks, 1 KB), activation boxes of two chunks x two atoms (2 KB).  The
+  // scale tiles as 16-byte rows: per stage one box of the weight atoms (one
+  // per 128-wide K chunk) and one of the token atoms (two per chunk).  The
   // MXFP4-input kernel reads the packed weight codes as plain bytes.
   const bool a4 = routed_a4(d);
+  const uint32_t sfa_rows = (a4 ? BsStage<true>::SFA_BYTES : BsStage<false>::SFA_BYTES) / 16;
+  const uint32_t sfb_rows = (a4 ? BsStage<true>::SFB_BYTES : BsStage<false>::SFB_BYTES) / 16;
+  const uint32_t b_max_rows = a4 ? BsStage<true>::B_MAX_ROWS : BsStage<false>::B_MAX_ROWS;
   auto wmap = [&](CUtensorMap* m, const void* codes, uint32_t box_rows) {
     return a4 ? make_map_u8_sw128(m, codes, wrows, K / 2, box_rows) : make_map_e2m1(m, codes, wrows, K, box_rows);
   };
   if (paired)
     ok = wmap(&maps.a0, w.Wg, 64) && wmap(&maps.a1, w.Wv, 64) &&
-         make_map_u8(&maps.sa, w.Sgv_tiled, sa_bytes / 16, 16, 16, 64);
+         make_map_u8(&maps.sa, w.Sgv_tiled, sa_bytes / 16, 16, 16, sfa_rows);
   else
-    ok = wmap(&maps.a0, w.Wo, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, 64);
+    ok = wmap(&maps.a0, w.Wo, 128) && make_map_u8(&maps.sa, w.So_tiled, sa_bytes / 16, 16, 16, sfa_rows);
   for (int i = 0; i < 4 && ok; ++i)
-    ok = make_map_u8_sw128(&maps.b[i], act_q, static_cast<uint64_t>(R), bs_code_bytes(d, K), 128u >> i);
+    ok = make_map_u8_sw128(&maps.b[i], act_q, static_cast<uint64_t>(R), bs_code_bytes(d, K),
+                           i == 0 ? b_max_rows : 128u >> i);
   const uint64_t sf_rows = static_cast<uint64_t>(max_tiles) * (K / 128) * 64;
-  ok = ok && make_map_u8(&maps.sb, act_sf, sf_rows, 16, 16, 128);
+  ok = ok && make_map_u8(&maps.sb, act_sf, sf_rows, 16, 16, sfb_rows);
   if (!ok) return MOE_ERR_CUDA;
   ExParams p{};
   p.tile_table = table;
   p.num_tiles_dev = n_tiles;
   p.n_wtiles = paired ? d.I / 128 : d.L / 256;
   p.w_rows_per_expert = out_rows;
-  p.num_k_blocks = K / BS_BK;
+  p.num_k_blocks = K / (a4 ? BsStage<true>::K : BsStage<false>::K);
   p.out = out;
   p.ldo = out_rows;
   p.out_cols = out_rows;
