@@ -30,9 +30,10 @@
 // fp32, packed to bf16, all exact) into the same 128-byte-swizzled bf16 A tile
 // the tensor cores read, and the MMA is the ordinary bf16 kind::f16.
 //
-// Warp roles as in gemm_tc.cuh: warp 0 TMA producer, warp 1 TMEM owner and (on
-// the even CTA) MMA issuer, warps 2-5 epilogue, and with MX warps 6-13
-// converters.  Every wait is bounded.
+// Warp roles: warp 0 TMA producer, warp 1 TMEM owner and (on the even CTA)
+// MMA issuer, warps 2-5 the first epilogue set, with MX warps 6-13
+// converters, and the next four warps the second epilogue set (the two sets
+// drain alternate 32-token chunks).  Every wait is bounded.
 #pragma once
 
 #include "activations.cuh"
@@ -47,7 +48,7 @@ constexpr uint32_t EX_B_BYTES = 128 * EX_BK * 2;      // up to 128 token rows pe
 constexpr uint32_t EX_STAGE_BYTES = EX_A_BYTES + EX_B_BYTES;
 constexpr uint32_t EX_ACC_COLS = 256;
 constexpr uint32_t EX_XCH_FLOATS = 2 * 2 * 16 * 32;        // [pair][direction][token][lane]
-constexpr uint32_t EX_XCH_BYTES = 2 * EX_XCH_FLOATS * 4;    // double-buffered, 16 KB
+constexpr uint32_t EX_XCH_BYTES = 2 * EX_XCH_FLOATS * 4;    // one buffer per epilogue set, 16 KB
 constexpr uint32_t EX_CODES_BYTES = 128 * 32;               // MX: E2M1 codes of 128 rows x 64 K
 constexpr uint32_t EX_SCALES_BYTES = 128 * 16;              // MX: E8M0 scales of 128 rows x 8 k-blocks
 constexpr int EX_CONV_WARPS = 8;
@@ -61,7 +62,10 @@ template <bool MX>
 struct ExCfg {
   static constexpr int kStages = MX ? 5 : 6;
   static_assert(!MX || (kStages > EX_CONV_BATCH && 8 % EX_CONV_BATCH == 0), "MX fence batch");
-  static constexpr int kThreads = 192 + (MX ? 32 * EX_CONV_WARPS : 0);
+  // warps: 0 producer, 1 MMA, 2-5 epilogue set 0, (MX) converters, then
+  // epilogue set 1
+  static constexpr int kEpi1Warp = 6 + (MX ? EX_CONV_WARPS : 0);
+  static constexpr int kThreads = 32 * (kEpi1Warp + 4);
   static constexpr uint32_t kStageBytes = EX_STAGE_BYTES + (MX ? EX_CODES_BYTES + EX_SCALES_BYTES : 0u);
   static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + EX_XCH_BYTES + 512;
 };
@@ -106,8 +110,18 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
-// Barrier 1 over the 128 epilogue threads (warps 2-5).
-__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barriers of the two epilogue sets (four warps each, one per
+// tensor-memory lane quarter): ids 1-4 for the two warps of a column pair (g
+// quarter q, v quarter q + 2) of set es, ids 5-6 for all four warps of a set
+// (aligned barriers: the warp reconverges first).
+__device__ __forceinline__ void epi_pair_bar(int es, int pair_q) {
+  __syncwarp();
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + 2 * es + pair_q) : "memory");
+}
+__device__ __forceinline__ void epi_set_bar(int es) {
+  __syncwarp();
+  asm volatile("bar.sync %0, 128;" ::"r"(5 + es) : "memory");
+}
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -302,7 +316,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* epi_ok = abort + 1;  // accumulator-ready verdict shared by the epilogue warps
+  volatile int* epi_ok = abort + 1;  // [2]: accumulator-ready verdict of each epilogue set
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4 * CG);
+      mbar_init(&acc_empty[a], 8 * CG);  // both epilogue sets' warps, in every CTA
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -479,7 +493,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
       mbar_wait(drain, 0u, &never, p.fault_site + 5);
     }
     __syncwarp();
-  } else if (MX && warp >= 6) {
+  } else if (MX && warp >= 6 && warp < 6 + EX_CONV_WARPS) {
     // ------------------------------------------------------------------ MXFP4 converters (both CTAs)
     // thread = one 32-element MX block: row r of the A tile, K half h
     const int ct = threadIdx.x - 192;
@@ -537,21 +551,28 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
+    // Two sets of four warps drain alternate 32-token chunks of an accumulator
+    // (set es: chunks es, es + 2, ...).  Measured on B200 (prefill gate/up):
+    // without the SiTU arithmetic and stores the kernel ran 13% faster, so one
+    // set's drain was on the critical path.
     const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int es = warp >= ExCfg<MX>::kEpi1Warp ? 1 : 0;
     const uint32_t acc_empty_leader =
         CG == 2 ? map_to_rank(smem_u32(&acc_empty[0]), 0u) : smem_u32(&acc_empty[0]);
     int acc = 0;
     uint32_t acc_phase = 0;
-    int xbuf = 0;
     for (int w = pair; w < total; w += npairs) {
       const ExTile t = ex_decode(w, num_tiles, num_multi, p);
       bool got;
       if constexpr (PAIRED) {
-        // One thread waits; the verdict reaches all four warps through the
-        // epilogue barrier, so they always run the same number of barriers.
-        if (threadIdx.x == 64) *epi_ok = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
-        epilogue_bar();
-        got = *epi_ok != 0;
+        // One thread of the set waits; the verdict reaches the set's four warps
+        // through its barrier, so they always run the same number of barriers
+        // (the barrier before the write keeps the previous verdict until every
+        // thread has read it).
+        epi_set_bar(es);
+        if (lane == 0 && q == 2) epi_ok[es] = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
+        epi_set_bar(es);
+        got = epi_ok[es] != 0;
       } else {
         // warp-uniform decision: tcgen05.ld below needs the whole warp
         got = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6));
@@ -561,19 +582,21 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * EX_ACC_COLS);
       const int nch = (t.ntok + 31) >> 5;  // 32-token chunks (uniform over the epilogue warps)
       if constexpr (PAIRED) {
-        // warps 0,1 hold g and warps 2,3 hold v for intermediate columns
+        // quarters 0,1 hold g and 2,3 hold v for intermediate columns
         // base + 32 * (q & 1) + lane; g warps form tokens 0-15 of a chunk,
-        // v warps tokens 16-31, after swapping the other half.
+        // v warps tokens 16-31, after swapping the other half through the
+        // set's exchange buffer (the two warps of a column pair sync alone).
         const bool is_g = q < 2;
         const int col = t.wt * (64 * CG) + static_cast<int>(rank) * 64 + (q & 1) * 32 + lane;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
         const float c = p.situ_c;
         const float inv_c = 1.0f / c;
+        float* X = xch + es * EX_XCH_FLOATS + (q & 1) * 1024;
 #pragma unroll 1
-        for (int ch = 0; ch < nch; ++ch) {
+        for (int ch = es; ch < nch; ch += 2) {
           float r[32];
           tmem_ld32(tbase + ch * 32, r);
-          float* X = xch + xbuf * EX_XCH_FLOATS + (q & 1) * 1024;
+          epi_pair_bar(es, q & 1);  // the partner has read the previous chunk's half
           // direction 0 region carries g (tokens 16-31), direction 1 carries v (tokens 0-15)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -582,7 +605,7 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
             else
               X[512 + i * 32 + lane] = r[i];
           }
-          epilogue_bar();
+          epi_pair_bar(es, q & 1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float g = is_g ? r[i] : X[i * 32 + lane];
@@ -591,13 +614,12 @@ __global__ void __launch_bounds__(ExCfg<MX>::kThreads, 1)
             if (tok < t.ntok && col < p.out_cols)
               out[static_cast<long long>(t.row0 + tok) * p.ldo + col] = __float2bfloat16_rn(situ_glu_fast(g, v, c, inv_c));
           }
-          xbuf ^= 1;
         }
       } else {
         const int col = t.wt * (128 * CG) + static_cast<int>(rank) * 128 + q * 32 + lane;
         float* out = reinterpret_cast<float*>(p.out);
 #pragma unroll 1
-        for (int ch = 0; ch < nch; ++ch) {
+        for (int ch = es; ch < nch; ch += 2) {
           float r[32];
           tmem_ld32(tbase + ch * 32, r);
 #pragma unroll

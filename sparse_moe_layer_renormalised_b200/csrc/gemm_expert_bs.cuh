@@ -193,18 +193,6 @@ __device__ __forceinline__ ExTile bs_decode(int w, int num_tiles, int num_multi,
   return t;
 }
 
-// Named barriers of the epilogue: ids 1-4 for the two warps of a column pair
-// (g quarter q, v quarter q + 2) of set es, ids 5-6 for all four warps of a set
-// (aligned barriers: the warp reconverges first).
-__device__ __forceinline__ void bs_pair_bar(int es, int pair_q) {
-  __syncwarp();
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + 2 * es + pair_q) : "memory");
-}
-__device__ __forceinline__ void bs_set_bar(int es) {
-  __syncwarp();
-  asm volatile("bar.sync %0, 128;" ::"r"(5 + es) : "memory");
-}
-
 template <int EPI, bool PAIRED, bool A4>
 __global__ void __launch_bounds__(BS_THREADS, 1)
     tc_expert_bs_kernel(const __grid_constant__ BsMaps maps, const ExParams p) {
@@ -467,9 +455,9 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
       if constexpr (PAIRED) {
         // one thread of the set waits; the set's barrier before the write keeps
         // the previous verdict until every thread has read it
-        bs_set_bar(es);
+        epi_set_bar(es);
         if (lane == 0 && q == (es ? 3 : 2)) epi_ok[es] = mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6) ? 1 : 0;
-        bs_set_bar(es);
+        epi_set_bar(es);
         got = epi_ok[es] != 0;
       } else {
         got = __all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, abort, p.fault_site + 6));
@@ -493,7 +481,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
         for (int ch = es; ch < nch; ch += 2) {
           float r[32];
           bs_load_chunk(tbase, ch, t.ntok, r);
-          bs_pair_bar(es, q & 1);  // the partner has read the previous chunk's half
+          epi_pair_bar(es, q & 1);  // the partner has read the previous chunk's half
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             if (is_g)
@@ -501,7 +489,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1)
             else
               X[512 + i * 32 + lane] = r[i];
           }
-          bs_pair_bar(es, q & 1);
+          epi_pair_bar(es, q & 1);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float g = is_g ? r[i] : X[i * 32 + lane];
