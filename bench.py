@@ -179,14 +179,13 @@ def layer_bytes(cfg, offsets: np.ndarray, T: int, y_bytes: int) -> float:
 def gate_up_kernel(cfg) -> str:
     """The routed gate/up kernel the library runs for this workload (the rule
     of moe_api.cu's use_two_tile: bf16 weights whose tiles divide evenly take
-    the two-weight-tile kernel when the average expert has fewer than 64 rows,
-    or as MOE_EXPERT_KERNEL forces; MXFP4 takes the one-tile kernel)."""
+    the two-weight-tile kernel unless MOE_EXPERT_KERNEL=one; MXFP4 with bf16
+    inputs takes the one-tile kernel)."""
     if cfg.routed in ("mxfp4_a8", "mxfp4_a4"):
         return f"tc_expert_bs_kernel<3, 1, {1 if cfg.routed == 'mxfp4_a4' else 0}>"
     cg = 2 if (cfg.I % 128 == 0 and cfg.L % 256 == 0) else 1
     env = os.environ.get("MOE_EXPERT_KERNEL", "")
-    two = cfg.routed == "bf16" and cfg.I % (128 * cg) == 0 and (
-        env == "two" or (env != "one" and cfg.T * cfg.k < 64 * cfg.E))
+    two = cfg.routed == "bf16" and cfg.I % (128 * cg) == 0 and env != "one"
     if two:
         return f"tc_expert2_kernel<3, 1, {cg}>"
     return f"tc_expert_kernel<3, 1, {cg}, {1 if cfg.routed == 'mxfp4' else 0}>"

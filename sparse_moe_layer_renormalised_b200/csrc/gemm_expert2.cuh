@@ -22,9 +22,11 @@
 // barrier; commits multicast to both CTAs).  CG = 1: single CTAs, M = 128.
 //
 // Warp roles: 0 TMA producer; 1 TMEM owner and issuer of accumulator 0;
-// 2-5 epilogue; 6 issuer of accumulator 1.  TMEM: accumulator a is columns
-// [256 a, 256 a + 256).  Both accumulators are single-buffered, so an item's
-// MMAs start once the epilogue has drained the previous item's accumulator.
+// 2-5 and 7-10 epilogue (two sets of four warps, one per TMEM lane quarter
+// each, on alternate 32-token chunks); 6 issuer of accumulator 1.  TMEM:
+// accumulator a is columns [256 a, 256 a + 256).  Both accumulators are
+// single-buffered, so an item's MMAs start once the epilogue has drained the
+// previous item's accumulator; the two epilogue sets halve that drain.
 // Every wait is bounded.
 #pragma once
 
@@ -38,7 +40,8 @@ constexpr uint32_t X2_A_BYTES = 128 * EX_BK * 2;  // 128 weight rows x 64 k
 constexpr uint32_t X2_B_BYTES = 128 * EX_BK * 2;  // up to 128 token rows per CTA
 constexpr uint32_t X2_STAGE_BYTES = 2 * X2_A_BYTES + X2_B_BYTES;
 constexpr int X2_STAGES = 4;
-constexpr int X2_THREADS = 224;
+constexpr int X2_THREADS = 352;
+constexpr int X2_EPI1_WARP = 7;  // warps 7-10: the second epilogue set
 constexpr size_t X2_SMEM = 1024 + static_cast<size_t>(X2_STAGES) * X2_STAGE_BYTES + 256;
 
 struct X2Maps {
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(X2_THREADS, 1) tc_expert2_kernel(const __grid_
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4 * CG);
+      mbar_init(&acc_empty[a], 8 * CG);  // both epilogue sets' warps, in every CTA
     }
     mbar_init(drain, 2);
     *abort = 0;
@@ -234,8 +237,9 @@ __global__ void __launch_bounds__(X2_THREADS, 1) tc_expert2_kernel(const __grid_
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
+    // ------------------------------------------------------------------ epilogue (warps 2-5, 7-10, both CTAs)
     const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int es = warp >= X2_EPI1_WARP ? 1 : 0;  // epilogue set: chunks es, es + 2, ...
     const uint32_t acc_empty_leader =
         CG == 2 ? map_to_rank(smem_u32(&acc_empty[0]), 0u) : smem_u32(&acc_empty[0]);
     uint32_t acc_phase = 0;
@@ -263,7 +267,7 @@ __global__ void __launch_bounds__(X2_THREADS, 1) tc_expert2_kernel(const __grid_
         const float c = p.situ_c;
         const float inv_c = 1.0f / c;
 #pragma unroll 1
-        for (int ch = 0; ch < nch; ++ch) {
+        for (int ch = es; ch < nch; ch += 2) {
           float g[32], v[32];
           tmem_ld32(lane_base + ch * 32, g);
           tmem_ld32(lane_base + EX_ACC_COLS + ch * 32, v);
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(X2_THREADS, 1) tc_expert2_kernel(const __grid_
           if (a == 0 || has_second(t.j)) {
             const int col = wrow_local(t.j, a) + q * 32 + lane;
 #pragma unroll 1
-            for (int ch = 0; ch < nch; ++ch) {
+            for (int ch = es; ch < nch; ch += 2) {
               float r[32];
               tmem_ld32(lane_base + a * EX_ACC_COLS + ch * 32, r);
               const long long r0 = static_cast<long long>(t.row0 + ch * 32);

@@ -539,23 +539,20 @@ cudaError_t launch_expert2_inst(const X2Maps& maps, const X2Params& p, cudaStrea
 
 // Which grouped expert kernel runs bf16 weights.  The two-weight-tile kernel
 // (gemm_expert2.cuh) halves the token rows moved per flop and issues MMAs from
-// two threads, but its accumulators are single-buffered; measured on B200 it
-// streams decode-shaped weights (a few rows per expert) 3.5% faster and is 6%
-// slower at the prefill shape (~290 rows per expert), where the one-tile
-// kernel's double-buffered accumulators hide the epilogue.  So it runs when
-// the average expert has fewer than kTwoTileMaxRows rows and its tiles divide
-// evenly.  MOE_EXPERT_KERNEL=one / =two in the environment forces either (both
-// compute the same result; used to compare them).
-constexpr long long kTwoTileMaxRows = 64;
-
+// two threads; its accumulators are single-buffered, and two epilogue warp
+// sets drain them.  Measured on B200 at the K3 shapes it is the faster of the
+// two: prefill (~290 rows per expert) gate/up 14.67 against 15.15 ms and down
+// 7.19 against 7.29 ms, decode (a few rows per expert) 3.5% faster.  So it
+// runs whenever its tiles divide evenly.  MOE_EXPERT_KERNEL=one / =two in the
+// environment forces either (both compute the same result; used to compare
+// them).
 bool use_two_tile(const moe_dims& d, bool paired) {
   if (d.act != MOE_BF16 || d.routed != MOE_BF16) return false;
   const int rows = 128 * expert_cg(d);
   if (paired ? d.I % rows != 0 : d.L % rows != 0) return false;
   const char* env = std::getenv("MOE_EXPERT_KERNEL");
   if (env != nullptr && std::strcmp(env, "one") == 0) return false;
-  if (env != nullptr && std::strcmp(env, "two") == 0) return true;
-  return d.T * d.k < kTwoTileMaxRows * d.E;
+  return true;
 }
 
 moe_status stage_expert2(const moe_dims& d, bool paired, const void* w0, const void* w1, const void* act, int K,
