@@ -376,6 +376,21 @@ MOE_API moe_status moe_mx8_quantize(const void* x, int64_t rows, int32_t K, uint
 MOE_API moe_status moe_mx4_quantize(const void* x, int64_t rows, int32_t K, uint8_t* codes, uint8_t* scales,
                                     moe_stream_t stream);
 
+/* Row gather for the expert-parallel exchange (the pages have no counterpart;
+ * a library facility): dst[r] = src[idx[r]] for r in [0, n), rows of
+ * row_bytes bytes.  The balanced expert-parallel step reorders its
+ * expert-major token rows by destination rank with it before the dispatch
+ * all-to-all, and puts the returned expert outputs back in expert-major
+ * order after the combine all-to-all.
+ *  - src [src_rows, row_bytes] and dst [n, row_bytes]: device, 16-byte
+ *    aligned, row_bytes a multiple of 16; idx [n] int32 device; all owned by
+ *    the caller; src and dst must not overlap.
+ *  - n = 0 is a no-op.  An index outside [0, src_rows) is recorded as a device
+ *    fault (moe_device_error, site code 15) and its row of dst is zero-filled.
+ *  - Enqueued on `stream`; no allocation. */
+MOE_API moe_status moe_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx,
+                                   int64_t n, void* dst, moe_stream_t stream);
+
 /* Weight scales for the block-scaled routed experts (routed = MOE_MXFP4_A8 or
  * MOE_MXFP4_A4).
  * The block-scaled MMA takes its scales from tensor memory, loaded from

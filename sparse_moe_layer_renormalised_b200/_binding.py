@@ -45,6 +45,7 @@ EXPORTED = (
     "moe_mx_tile_scales",
     "moe_mx8_quantize",
     "moe_mx4_quantize",
+    "moe_gather_rows",
 )
 
 MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -138,6 +139,7 @@ def lib() -> ctypes.CDLL:
         L.moe_mx_tile_scales.argtypes = [pd, vp, vp, vp, vp, vp, vp]
         L.moe_mx8_quantize.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
         L.moe_mx4_quantize.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
+        L.moe_gather_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, ctypes.c_int64, vp, vp]
         for f in EXPORTED:
             if f not in ("moe_workspace_size", "moe_status_str", "moe_expert_ffn_blocks_workspace_size",
                          "moe_backward_workspace_size"):
@@ -338,6 +340,11 @@ def moe_mx8_quantize(x, rows: int, K: int, codes, scales, stream=None) -> int:
 
 def moe_mx4_quantize(x, rows: int, K: int, codes, scales, stream=None) -> int:
     return lib().moe_mx4_quantize(_ptr(x), int(rows), int(K), _ptr(codes), _ptr(scales), _stream(stream))
+
+
+def moe_gather_rows(src, src_rows: int, row_bytes: int, idx, n: int, dst, stream=None) -> int:
+    return lib().moe_gather_rows(_ptr(src), int(src_rows), int(row_bytes), _ptr(idx), int(n), _ptr(dst),
+                                 _stream(stream))
 
 
 def moe_selftest_wait_timeout(limit_ms: int, waited_ns, stream=None) -> int:

@@ -1524,6 +1524,22 @@ moe_status moe_mx4_quantize(const void* x, int64_t rows, int32_t K, uint8_t* cod
   return mx_quantize_rows(true, x, rows, K, codes, scales, stream, 183);
 }
 
+moe_status moe_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx, int64_t n,
+                           void* dst, moe_stream_t stream) {
+  if (src_rows < 0 || n < 0 || row_bytes <= 0 || row_bytes % 16 != 0 || row_bytes / 16 > 0x7fffffffLL)
+    return MOE_ERR_INVALID_ARG;
+  if (n > 0x7fffffffLL * GATHER_WARPS) return MOE_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (n == 0) return MOE_OK;
+  if (src == nullptr || idx == nullptr || dst == nullptr || !aligned16(src) || !aligned16(dst))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  gather_rows_idx_kernel<<<static_cast<unsigned>(cdiv(n, GATHER_WARPS)), GATHER_WARPS * 32, 0, s>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), idx, n, src_rows, static_cast<int>(row_bytes / 16));
+  g_last_launches = 1;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_mx_tiled_scales_size(const moe_dims* d, size_t* gate_up_bytes, size_t* down_bytes) {
   if (!dims_ok(d) || gate_up_bytes == nullptr || down_bytes == nullptr) return MOE_ERR_INVALID_ARG;
   if (d->L % 512 != 0 || d->I % 512 != 0) return MOE_ERR_UNSUPPORTED;

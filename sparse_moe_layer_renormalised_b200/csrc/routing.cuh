@@ -15,6 +15,7 @@ constexpr int kFaultExpertRange = 11;     // topk_idx entry outside [0, E)
 constexpr int kFaultDuplicateExpert = 12;  // a token lists the same expert twice
 constexpr int kFaultTokenRange = 13;       // perm_token entry outside [0, T)
 constexpr int kFaultOffsets = 14;          // expert_offsets not monotone / out of range
+constexpr int kFaultRowIndex = 15;         // moe_gather_rows index outside [0, src_rows)
 
 // ------------------------------------------------------------------------------ top-k
 // One warp per token.  Lane l holds experts l, l+32, l+64, ... (E <= 1024).
@@ -338,6 +339,35 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32)
   }
   const uint4* s = src + static_cast<long long>(t) * row_vecs;
   // four 16-byte loads in flight per lane before their stores
+  int i = lane;
+  for (; i + 96 < row_vecs; i += 128) {
+    const uint4 a = s[i], b = s[i + 32], c = s[i + 64], e = s[i + 96];
+    d[i] = a;
+    d[i + 32] = b;
+    d[i + 64] = c;
+    d[i + 96] = e;
+  }
+  for (; i < row_vecs; i += 32) d[i] = s[i];
+}
+
+// dst[r] = src[idx[r]] for r < n, rows of row_vecs 16-byte words (the
+// expert-parallel exchange's reordering of token rows by destination and back).
+// One warp per row; an index outside [0, src_rows) records kFaultRowIndex and
+// zero-fills the row.
+__global__ void __launch_bounds__(GATHER_WARPS * 32)
+    gather_rows_idx_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ idx,
+                           long long n, long long src_rows, int row_vecs) {
+  const long long row = static_cast<long long>(blockIdx.x) * GATHER_WARPS + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n) return;
+  const long long t = idx[row];
+  uint4* d = dst + row * row_vecs;
+  if (t < 0 || t >= src_rows) {
+    if (lane == 0) record_fault(kFaultRowIndex);
+    for (int i = lane; i < row_vecs; i += 32) d[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4* s = src + t * row_vecs;
   int i = lane;
   for (; i + 96 < row_vecs; i += 128) {
     const uint4 a = s[i], b = s[i + 32], c = s[i + 64], e = s[i + 96];

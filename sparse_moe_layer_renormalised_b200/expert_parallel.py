@@ -8,8 +8,18 @@ tokens with all-to-all communication).
 Reading (where the page gives only the idea): experts are partitioned into G
 contiguous ranges, rank g owning experts [bounds[g], bounds[g+1]); every rank
 holds all non-routed weights and runs its own batch of tokens (data parallel
-over tokens).  MoonEP's redundant copies of hot experts and its balanced
-placement are not built.
+over tokens).
+
+Balanced mode (the default; page "Kimi K3 tech-report summary"
+(jiwasawa.github.io), section "Multi-Trillion 規模を支える Infrastructure", the
+MoonEP item: redundant experts planned dynamically so that every rank is
+assigned the same number of tokens, for static compute shapes).  Reading:
+each step the ranks share their per-expert row counts and every rank computes
+the same plan (balanced_plan): rank g runs floor(R/G) or ceil(R/G) of the step's
+R routed rows; a rank whose own experts draw more rows than that hands rows of
+its hottest experts to ranks below their quota, which run those experts as
+redundant copies for the step (their weights travel from the owner with the
+rows).  The static mode (balance=False) sends every row to its expert's owner.
 
 One layer step on rank g (every step of the layer runs in libmoe_b200.so;
 the exchange is torch.distributed all_to_all, NCCL between GPUs):
@@ -19,11 +29,16 @@ the exchange is torch.distributed all_to_all, NCCL between GPUs):
                            pairs with their z rows; the rows bound for rank r
                            are then one contiguous block
   4. exchange plan         per-expert row counts to and from every rank
-  5. dispatch              all_to_all of the z rows
-  6. moe_expert_ffn_blocks this rank's experts over the received rows, one
-                           expert-major block per sending rank
+                           (balanced: all ranks' counts, the plan, and the
+                           redundant experts' weights from their owners)
+  5. dispatch              all_to_all of the z rows (balanced: first ordered
+                           by destination with moe_gather_rows)
+  6. moe_expert_ffn_blocks this rank's experts (balanced: and its redundant
+                           copies) over the received rows, one expert-major
+                           block per sending rank
   7. combine               all_to_all of the fp32 expert outputs back, which
-                           arrive in the sender's own expert-major order
+                           arrive in the sender's send order (balanced: put
+                           back in expert-major order with moe_gather_rows)
   8. moe_combine, moe_output   u, RMSNorm(u), y
 Step 4 reads the expert offsets on the host (the all_to_all needs the row
 counts), the one host synchronisation of the step.
@@ -38,8 +53,8 @@ import torch.distributed as dist
 
 from .layer import tile_weight_scales
 from ._binding import (BLOCK_SCALED, Dims, check, make_weights, moe_combine, moe_expert_ffn_blocks,
-                       moe_expert_ffn_blocks_workspace_size, moe_latent_shared, moe_output, moe_permute,
-                       moe_router_topk, moe_workspace_size)
+                       moe_expert_ffn_blocks_workspace_size, moe_gather_rows, moe_latent_shared, moe_output,
+                       moe_permute, moe_router_topk, moe_workspace_size)
 
 _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
@@ -132,17 +147,189 @@ def combine_rows(rows: torch.Tensor, plan: ExchangePlan, group=None) -> torch.Te
     return out
 
 
+# ------------------------------------------------------------------------------ balanced mode
+@dataclass
+class BalancedPlan:
+    """One step's assignment of the routed rows to ranks.
+
+    The rows of expert e, in global order (sending ranks in rank order, each
+    sender's rows in its own expert-major order), are cut into segments: the
+    owner's first, then one per rank that runs a redundant copy of e."""
+
+    bounds: np.ndarray   # [G + 1] home partition (partition(E, G))
+    quota: np.ndarray    # [G] rows each rank runs: floor(R / G), the first R % G ranks one more
+    segments: list       # [E] lists of (rank, start, count), ordered by start
+    replicas: list       # [G] ascending ids of the experts rank g runs without owning them
+
+    def local_experts(self, g: int) -> np.ndarray:
+        """The experts rank g runs, in its local order: its own, then its
+        redundant copies."""
+        home = np.arange(self.bounds[g], self.bounds[g + 1], dtype=np.int64)
+        return np.concatenate([home, np.asarray(self.replicas[g], np.int64)])
+
+
+def balanced_plan(counts: np.ndarray, bounds: np.ndarray) -> BalancedPlan:
+    """counts [G, E]: rows each rank sends to each expert this step.
+
+    Every rank's load becomes exactly its quota: ranks whose own experts
+    exceed it (donors, in rank order) hand rows of their experts, hottest
+    first (ties to the lower id), to the ranks below it (receivers, in rank
+    order), a receiver taking from one expert until it is full or the
+    donor's excess or the expert's rows are used up.  Each hand-over makes the
+    receiver run a redundant copy of that expert.  Deterministic, so every
+    rank computes the same plan from the same counts."""
+    counts = np.asarray(counts, np.int64)
+    G = len(bounds) - 1
+    C = counts.sum(axis=0)
+    R = int(C.sum())
+    quota = np.full(G, R // G, np.int64)
+    quota[: R % G] += 1
+    home_load = np.array([C[bounds[g]:bounds[g + 1]].sum() for g in range(G)], np.int64)
+    excess = home_load - quota
+    deficit = np.maximum(-excess, 0)
+    receivers = [g for g in range(G) if deficit[g] > 0]
+    keep = C.copy()                     # rows the owner keeps
+    given: list = [[] for _ in range(len(C))]  # per expert: (rank, rows) handed over, in order
+    ri = 0
+    for d in range(G):
+        need = int(excess[d])
+        if need <= 0:
+            continue
+        for e in sorted(range(bounds[d], bounds[d + 1]), key=lambda e: (-C[e], e)):
+            while need > 0 and keep[e] > 0:
+                r = receivers[ri]
+                n = int(min(need, keep[e], deficit[r]))
+                given[e].append((r, n))
+                keep[e] -= n
+                need -= n
+                deficit[r] -= n
+                if deficit[r] == 0:
+                    ri += 1
+            if need == 0:
+                break
+    owner = np.searchsorted(bounds, np.arange(len(C)), side="right") - 1
+    segments, replicas = [], [[] for _ in range(G)]
+    for e in range(len(C)):
+        seg = [(int(owner[e]), 0, int(keep[e]))] if keep[e] > 0 else []
+        start = int(keep[e])
+        for r, n in given[e]:
+            seg.append((r, start, n))
+            replicas[r].append(e)
+            start += n
+        segments.append(seg)
+    return BalancedPlan(bounds=np.asarray(bounds, np.int64), quota=quota, segments=segments,
+                        replicas=[sorted(set(x)) for x in replicas])
+
+
+@dataclass
+class BalancedExchange:
+    """One rank's side of a balanced exchange."""
+
+    send_idx: np.ndarray            # [n_send] rows of the sender's expert-major buffer, in send order
+    send_rows: list                 # [G]
+    recv_rows: list                 # [G]
+    recv_block_offsets: np.ndarray  # [G, n_local + 1] offsets of each source's block, by local expert
+    n_recv: int
+
+
+def _pieces(plan: BalancedPlan, counts: np.ndarray, s: int):
+    """(destination, local expert index there, first row of the piece within
+    the sender's expert-major rows of that expert, rows) for sender s."""
+    local = {g: {int(e): i for i, e in enumerate(plan.local_experts(g))} for g in range(len(plan.quota))}
+    before = counts[:s].sum(axis=0)  # rows of each expert from earlier senders
+    out = []
+    for e in np.nonzero(counts[s])[0]:
+        lo, hi = int(before[e]), int(before[e] + counts[s, e])
+        for g, st, n in plan.segments[e]:
+            a, b = max(lo, st), min(hi, st + n)
+            if a < b:
+                out.append((g, local[g][int(e)], int(e), a - lo, b - a))
+    return out
+
+
+def balanced_exchange(plan: BalancedPlan, counts: np.ndarray, offsets: np.ndarray, rank: int) -> BalancedExchange:
+    """The send order, split sizes and receive blocks of `rank` under the
+    plan; offsets [E + 1] are this rank's expert-major CSR offsets.  Rows
+    bound for one destination are sent together, in the destination's local
+    expert order; a received block (one per source, in rank order) is
+    expert-major in this rank's local order."""
+    counts = np.asarray(counts, np.int64)
+    G = len(plan.quota)
+    n_local = len(plan.local_experts(rank))
+    by_dest = [[] for _ in range(G)]
+    for g, li, e, first, n in _pieces(plan, counts, rank):
+        by_dest[g].append((li, int(offsets[e]) + first, n))
+    idx, send_rows = [], []
+    for g in range(G):
+        pieces = sorted(by_dest[g])
+        send_rows.append(sum(n for _, _, n in pieces))
+        idx += [np.arange(st, st + n, dtype=np.int64) for _, st, n in pieces]
+    send_idx = np.concatenate(idx) if idx else np.zeros(0, np.int64)
+    blocks = np.zeros((G, n_local + 1), np.int64)
+    start = 0
+    for s in range(G):
+        per = np.zeros(n_local, np.int64)
+        for g, li, _, _, n in _pieces(plan, counts, s):
+            if g == rank:
+                per[li] += n
+        blocks[s, 0] = start
+        blocks[s, 1:] = start + np.cumsum(per)
+        start = int(blocks[s, -1])
+    return BalancedExchange(send_idx=send_idx, send_rows=send_rows,
+                            recv_rows=[int(blocks[s, -1] - blocks[s, 0]) for s in range(G)],
+                            recv_block_offsets=blocks, n_recv=start)
+
+
+def gather_counts(offsets: np.ndarray, group=None) -> np.ndarray:
+    """Every rank's per-expert row counts [G, E] (one all_gather)."""
+    c = torch.from_numpy(np.diff(np.asarray(offsets, np.int64)))
+    dev = _comm_device(group)
+    out = [torch.empty_like(c, device=dev) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(out, c.to(dev), group=group)
+    return torch.stack(out).cpu().numpy()
+
+
+def exchange_replica_weights(plan: BalancedPlan, home: dict, group=None) -> dict:
+    """Sends every redundant expert's weights from its owner to the ranks
+    that run it this step.  home: name -> [n_home, ...] tensor of this rank's
+    experts (one slice per expert); returns name -> [len(replicas[rank]), ...]
+    with the slices of this rank's redundant experts in ascending id order."""
+    rank = dist.get_rank(group)
+    G = len(plan.quota)
+    lo = int(plan.bounds[rank])
+    out = {}
+    for name, t in home.items():
+        per = t[0].numel() * t.element_size()
+        flat = t.reshape(t.shape[0], -1).view(torch.uint8) if t.dtype != torch.uint8 else t.reshape(t.shape[0], -1)
+        send, send_sizes = [], []
+        for g in range(G):
+            mine = [e - lo for e in plan.replicas[g] if plan.bounds[rank] <= e < plan.bounds[rank + 1]]
+            send += [flat[i] for i in mine]
+            send_sizes.append(per * len(mine))
+        recv_sizes = [per * sum(1 for e in plan.replicas[rank] if plan.bounds[s] <= e < plan.bounds[s + 1])
+                      for s in range(G)]
+        sbuf = torch.cat(send) if send else torch.zeros(0, dtype=torch.uint8, device=t.device)
+        rbuf = torch.empty(sum(recv_sizes), dtype=torch.uint8, device=t.device)
+        dist.all_to_all_single(rbuf, sbuf.contiguous(), output_split_sizes=recv_sizes, input_split_sizes=send_sizes,
+                               group=group)
+        out[name] = rbuf.view(t.dtype).reshape((len(plan.replicas[rank]),) + tuple(t.shape[1:]))
+    return out
+
+
 class ExpertParallelMoeLayer:
     """One rank's share of an expert-parallel layer.
 
     dims: the full layer (E = all routed experts).  weights: device tensors
     named as moe_weights' fields; Wg / Wv / Wo (and Sg / Sv / So for MXFP4)
     hold only this rank's experts, bounds[rank] .. bounds[rank+1]-1, in order.
-    With a block-scaled routed type ("mxfp4_a8", "mxfp4_a4") the dispatched rows stay bf16 and the receiving
-    rank quantises them (moe_expert_ffn_blocks).
+    With a block-scaled routed type ("mxfp4_a8", "mxfp4_a4") the dispatched
+    rows stay bf16 and the receiving rank quantises them
+    (moe_expert_ffn_blocks).  balance (default True): every rank runs the
+    same number of rows per step, hot experts' rows shared out to redundant
+    copies (module docstring); False: every row goes to its expert's owner.
     max_tokens sizes the local workspaces."""
 
-    def __init__(self, dims: Dims, weights: dict, group=None, max_tokens: int | None = None):
+    def __init__(self, dims: Dims, weights: dict, group=None, max_tokens: int | None = None, balance: bool = True):
         self.dims = dims
         self.group = group
         self.G = dist.get_world_size(group)
@@ -161,6 +348,30 @@ class ExpertParallelMoeLayer:
         dev = weights["Wr"].device
         self.workspace = torch.empty(moe_workspace_size(replace(dims, T=self.max_tokens)), dtype=torch.uint8,
                                      device=dev)
+        self.balance = balance
+        self.last_plan = None
+        if balance:
+            # the routed tensors this path reads, one slice per expert, in
+            # buffers with room behind this rank's experts for redundant copies
+            names = ["Wg", "Wv", "Wo"] + (["Sg", "Sv", "So"] if dims.routed == "mxfp4" else []) + (
+                ["Sgv_tiled", "So_tiled"] if dims.routed in BLOCK_SCALED else [])
+            self._home = {n: self.weights[n].reshape((self.e_local, -1) if n.endswith("_tiled") else
+                                                     tuple(self.weights[n].shape)) for n in names}
+            self._buf = {}
+            self._grow(self.e_local)
+
+    def _grow(self, cap: int) -> None:
+        """Routed-weight buffers for this rank's experts and up to cap
+        redundant copies."""
+        for n, t in self._home.items():
+            b = torch.empty((self.e_local + cap,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+            b[: self.e_local].copy_(t)
+            self._buf[n] = b
+        self._cap = cap
+
+    def _local_weights(self, n_local: int):
+        w = {n: (b[:n_local].reshape(-1) if n.endswith("_tiled") else b[:n_local]) for n, b in self._buf.items()}
+        return make_weights(**w)
 
     def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         d = replace(self.dims, T=x.shape[0])
@@ -180,7 +391,20 @@ class ExpertParallelMoeLayer:
         check(moe_router_topk(d, x, w["Wr"], w["bias"], scores, 0, idx, p, stream))
         check(moe_latent_shared(d, self._w, x, z, h_s, stream))
         check(moe_permute(d, idx, z, offsets, perm_token, inv_perm, z_perm, self.workspace, None, stream))
-        plan = exchange_plan(offsets.cpu().numpy(), self.bounds, self.group)
+        if self.balance:
+            y_perm = self._balanced_experts(d, offsets.cpu().numpy(), z_perm, stream)
+        else:
+            y_perm = self._static_experts(d, offsets.cpu().numpy(), z_perm, stream)
+        n = torch.empty(T, L, dtype=act, device=dev)
+        check(moe_combine(d, y_perm, inv_perm, p, w["gamma"], None, n, stream))
+        y = torch.empty(T, d.H, dtype=_TORCH_DT[d.y_out], device=dev)
+        check(moe_output(d, self._w, h_s, n, y, stream))
+        return y
+
+    def _static_experts(self, d: Dims, offsets: np.ndarray, z_perm: torch.Tensor, stream) -> torch.Tensor:
+        """Every row to its expert's owner and back: y_perm [T k, L] fp32."""
+        dev, L = z_perm.device, d.L
+        plan = exchange_plan(offsets, self.bounds, self.group)
         z_recv = dispatch_rows(z_perm, plan, self.group)
         y_recv = torch.empty(plan.n_recv, L, dtype=torch.float32, device=dev)
         if plan.n_recv > 0:
@@ -189,11 +413,46 @@ class ExpertParallelMoeLayer:
                              dtype=torch.uint8, device=dev)
             check(moe_expert_ffn_blocks(self.local_dims, self._w, z_recv, plan.n_recv, blocks, self.G, y_recv, ws,
                                         None, stream))
-        y_perm = combine_rows(y_recv, plan, self.group)
-        n = torch.empty(T, L, dtype=act, device=dev)
-        check(moe_combine(d, y_perm, inv_perm, p, w["gamma"], None, n, stream))
-        y = torch.empty(T, d.H, dtype=_TORCH_DT[d.y_out], device=dev)
-        check(moe_output(d, self._w, h_s, n, y, stream))
-        return y
+        return combine_rows(y_recv, plan, self.group)
+
+    def _balanced_experts(self, d: Dims, offsets: np.ndarray, z_perm: torch.Tensor, stream) -> torch.Tensor:
+        """The balanced exchange: y_perm [T k, L] fp32 in expert-major order."""
+        dev, L = z_perm.device, d.L
+        counts = gather_counts(offsets, self.group)
+        plan = balanced_plan(counts, self.bounds)
+        self.last_plan = plan
+        ex = balanced_exchange(plan, counts, offsets, self.rank)
+        reps = plan.replicas[self.rank]
+        n_local = self.e_local + len(reps)
+        copies = exchange_replica_weights(plan, self._home, self.group)
+        if len(reps) > self._cap:
+            self._grow(max(len(reps), 2 * self._cap))
+        for n, t in copies.items():
+            self._buf[n][self.e_local:n_local].copy_(t)
+        # rows ordered by destination, dispatched, run, returned, put back
+        n_send = len(ex.send_idx)
+        idx = torch.from_numpy(ex.send_idx.astype(np.int32)).to(dev)
+        z_send = torch.empty_like(z_perm)
+        check(moe_gather_rows(z_perm, z_perm.shape[0], L * z_perm.element_size(), idx, n_send, z_send, stream))
+        z_recv = torch.empty(ex.n_recv, L, dtype=z_perm.dtype, device=dev)
+        dist.all_to_all_single(z_recv, z_send, output_split_sizes=ex.recv_rows, input_split_sizes=ex.send_rows,
+                               group=self.group)
+        y_recv = torch.empty(ex.n_recv, L, dtype=torch.float32, device=dev)
+        if ex.n_recv > 0:
+            ld = replace(d, E=n_local)
+            blocks = torch.from_numpy(ex.recv_block_offsets.astype(np.int32)).to(dev)
+            ws = torch.empty(moe_expert_ffn_blocks_workspace_size(ld, ex.n_recv, self.G), dtype=torch.uint8,
+                             device=dev)
+            check(moe_expert_ffn_blocks(ld, self._local_weights(n_local), z_recv, ex.n_recv, blocks, self.G, y_recv,
+                                        ws, None, stream))
+        y_back = torch.empty(n_send, L, dtype=torch.float32, device=dev)
+        dist.all_to_all_single(y_back, y_recv, output_split_sizes=ex.send_rows, input_split_sizes=ex.recv_rows,
+                               group=self.group)
+        inv = np.empty(n_send, np.int64)
+        inv[ex.send_idx] = np.arange(n_send)
+        inv_t = torch.from_numpy(inv.astype(np.int32)).to(dev)
+        y_perm = torch.empty(n_send, L, dtype=torch.float32, device=dev)
+        check(moe_gather_rows(y_back, n_send, L * 4, inv_t, n_send, y_perm, stream))
+        return y_perm
 
     __call__ = forward

@@ -1,5 +1,7 @@
 """The expert-parallel exchange (dispatch and combine of token rows between
-the ranks that hold the experts) on CPU: gloo ranks, world size 2 and 3.
+the ranks that hold the experts) on CPU: gloo ranks, world sizes 2 to 4, in
+the static mode (rows to their expert's owner) and the balanced mode (equal
+rows per rank, redundant copies of hot experts; see the last section).
 
 Every rank routes its own tokens, orders its (token, slot) pairs expert-major
 (the oracle's stable permutation), and sends each rank the rows of that rank's
@@ -102,3 +104,176 @@ def test_partition_and_plan_tables():
     plan = ep.plan_from_counts(sent, received, 3)
     assert plan.send_rows == [5, 5] and plan.recv_rows == [6, 6] and plan.n_recv == 12
     assert plan.recv_block_offsets.tolist() == [[0, 5, 6, 6], [6, 8, 10, 12]]
+
+
+# ------------------------------------------------------------------------------ balanced mode
+def _row_destinations(plan, counts):
+    """Brute force: the rank that runs each row, per sender, in the sender's
+    expert-major order (global order of expert e's rows: senders in rank
+    order)."""
+    G, E = counts.shape
+    dest = []
+    for s in range(G):
+        d = []
+        for e in range(E):
+            before = int(counts[:s, e].sum())
+            for j in range(int(counts[s, e])):
+                pos = before + j
+                owners = [g for g, st, n in plan.segments[e] if st <= pos < st + n]
+                assert len(owners) == 1, (s, e, j)
+                d.append(owners[0])
+        dest.append(np.array(d, np.int64))
+    return dest
+
+
+def _count_cases():
+    rng = np.random.default_rng(11)
+    cases = []
+    for G, E in [(1, 5), (2, 13), (3, 10), (4, 9), (5, 23), (4, 4)]:
+        w = (np.arange(E) + 1.0) ** -1.2
+        cases.append((G, rng.multinomial(60 * G, w / w.sum(), size=G)))     # Zipf-skewed senders
+        cases.append((G, rng.integers(0, 5, size=(G, E))))                    # small, with zeros
+    hot = np.zeros((3, 7), np.int64)
+    hot[:, 2] = [50, 40, 30]                                                  # one expert holds every row
+    cases += [(3, hot), (4, np.zeros((4, 6), np.int64)), (4, np.eye(4, 6, dtype=np.int64))]  # no rows; R < G
+    return cases
+
+
+@pytest.mark.parametrize("case", range(len(_count_cases())))
+def test_balanced_plan_invariants(case):
+    """Every rank gets floor(R/G) or ceil(R/G) rows (the first R % G one
+    more); each expert's rows are cut into consecutive segments, the owner's
+    first; ranks other than the owner appear only as listed redundant copies;
+    the brute-force destination of every row agrees."""
+    G, counts = _count_cases()[case]
+    E = counts.shape[1]
+    bounds = ep.partition(E, G)
+    plan = ep.balanced_plan(counts, bounds)
+    C, R = counts.sum(axis=0), int(counts.sum())
+    assert plan.quota.tolist() == [R // G + (1 if g < R % G else 0) for g in range(G)]
+    load = np.zeros(G, np.int64)
+    for e in range(E):
+        owner = int(np.searchsorted(bounds, e, side="right") - 1)
+        start = 0
+        for i, (g, st, n) in enumerate(plan.segments[e]):
+            assert st == start and n > 0
+            start += n
+            load[g] += n
+            if g == owner:
+                assert i == 0, "the owner's segment comes first"
+            else:
+                assert e in plan.replicas[g] and not bounds[g] <= e < bounds[g + 1]
+        assert start == C[e]
+    assert load.tolist() == plan.quota.tolist()
+    for g in range(G):
+        assert plan.replicas[g] == sorted(set(plan.replicas[g]))
+        assert all(any(r == g for r, _, _ in plan.segments[e]) for e in plan.replicas[g])
+    dest = _row_destinations(plan, counts)
+    assert np.bincount(np.concatenate(dest + [np.zeros(0, np.int64)]), minlength=G).tolist() == plan.quota.tolist()
+    # a rank already at its quota keeps all its rows and runs no copies
+    home_load = np.array([C[bounds[g]:bounds[g + 1]].sum() for g in range(G)])
+    for g in range(G):
+        if home_load[g] == plan.quota[g]:
+            assert not plan.replicas[g]
+
+
+@pytest.mark.parametrize("case", range(len(_count_cases())))
+def test_balanced_exchange_tables(case):
+    """Each sender's send order is a permutation of its rows, grouped by
+    destination in rank order and, within a destination, by the
+    destination's local expert order; every receiver's blocks match what the
+    senders send it."""
+    G, counts = _count_cases()[case]
+    E = counts.shape[1]
+    bounds = ep.partition(E, G)
+    plan = ep.balanced_plan(counts, bounds)
+    dest = _row_destinations(plan, counts)
+    ex = []
+    for s in range(G):
+        offsets = np.concatenate([[0], np.cumsum(counts[s])])
+        x = ep.balanced_exchange(plan, counts, offsets, s)
+        assert sorted(x.send_idx.tolist()) == list(range(int(counts[s].sum())))
+        expert_of = np.repeat(np.arange(E), counts[s])
+        d_of = dest[s][x.send_idx]
+        assert np.all(np.diff(d_of) >= 0) and np.bincount(d_of, minlength=G).tolist() == x.send_rows
+        for g in range(G):
+            local = {int(e): i for i, e in enumerate(plan.local_experts(g))}
+            sel = x.send_idx[d_of == g]
+            li = np.array([local[int(e)] for e in expert_of[sel]], np.int64)
+            assert np.all(np.diff(li) >= 0), "local expert order within a destination"
+            assert np.all(np.diff(sel)[np.diff(li) == 0] == 1), "rows of one expert keep their order"
+        ex.append(x)
+    for g in range(G):
+        assert ex[g].n_recv == plan.quota[g]
+        for s in range(G):
+            assert ex[g].recv_rows[s] == ex[s].send_rows[g]
+            blk = ex[g].recv_block_offsets[s]
+            assert blk[-1] - blk[0] == ex[s].send_rows[g]
+
+
+def _balanced_worker(rank, world, port, E, k, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        T, L = 40 + 23 * rank, 6
+        idx = _routing(rank, T, E, k, "zipf")
+        z = np.random.default_rng(7 + rank).standard_normal((T, L)).astype(np.float32)
+        counts_local, offsets, perm_token, inv_perm = oracle.permute(idx, E)
+        z_perm = torch.from_numpy(z[perm_token])
+        bounds = ep.partition(E, world)
+        counts = ep.gather_counts(offsets)
+        assert np.array_equal(counts[rank], counts_local)
+        plan = ep.balanced_plan(counts, bounds)
+        x = ep.balanced_exchange(plan, counts, offsets, rank)
+        # the layer orders rows with moe_gather_rows on the GPU; torch indexing here
+        z_send = z_perm[torch.from_numpy(x.send_idx)]
+        z_recv = torch.empty(x.n_recv, L)
+        dist.all_to_all_single(z_recv, z_send, output_split_sizes=x.recv_rows, input_split_sizes=x.send_rows)
+        assert x.n_recv == plan.quota[rank], "every rank runs its quota"
+        local = plan.local_experts(rank)
+        label = np.full(x.n_recv, -1)
+        for s in range(world):
+            b = x.recv_block_offsets[s]
+            for i, e in enumerate(local):
+                label[b[i]:b[i + 1]] = e
+        assert (label >= 0).all()
+        # the received rows are exactly the rows the plan assigns here
+        everyone = [None] * world
+        dist.all_gather_object(everyone, (z_perm.numpy(), offsets))
+        dest = _row_destinations(plan, counts)
+        want = np.concatenate([everyone[s][0][np.nonzero(dest[s] == rank)[0]] for s in range(world)])
+        got_sorted = np.sort(z_recv.numpy(), axis=0)
+        assert np.array_equal(got_sorted, np.sort(want, axis=0)), "received rows"
+        # stand-in experts y = z * (e + 1); the results return to their senders
+        y_recv = z_recv * torch.from_numpy((label + 1).astype(np.float32))[:, None]
+        y_back = torch.empty(len(x.send_idx), L)
+        dist.all_to_all_single(y_back, y_recv, output_split_sizes=x.send_rows, input_split_sizes=x.recv_rows)
+        y_perm = torch.empty_like(y_back)
+        y_perm[torch.from_numpy(x.send_idx)] = y_back
+        expert_of_pos = np.repeat(np.arange(E), counts_local)
+        assert np.array_equal(y_perm.numpy(), z_perm.numpy() * (expert_of_pos + 1).astype(np.float32)[:, None])
+        # redundant copies: every rank receives the slices of the experts it runs without owning them
+        lo, hi = bounds[rank], bounds[rank + 1]
+        home = {"Wg": torch.arange(lo, hi, dtype=torch.float32)[:, None, None].repeat(1, 2, 3),
+                "So_tiled": (torch.arange(lo, hi, dtype=torch.int64)[:, None].repeat(1, 5) % 251).to(torch.uint8)}
+        copies = ep.exchange_replica_weights(plan, home)
+        reps = plan.replicas[rank]
+        assert copies["Wg"].shape == (len(reps), 2, 3) and copies["So_tiled"].shape == (len(reps), 5)
+        for i, e in enumerate(reps):
+            assert torch.all(copies["Wg"][i] == e) and torch.all(copies["So_tiled"][i] == e % 251)
+        out[rank] = (x.n_recv, len(reps))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,E,k", [(2, 13, 3), (3, 10, 2), (4, 9, 3)])
+def test_gloo_balanced_exchange(world, E, k):
+    """The balanced exchange end to end on gloo ranks with Zipf-skewed
+    routing: per-rank loads equal, rows and results travel correctly, and
+    the redundant experts' weight slices arrive from their owners."""
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_balanced_worker, args=(world, _free_port(), E, k, out), nprocs=world, join=True)
+    loads = [out[r][0] for r in range(world)]
+    assert max(loads) - min(loads) <= 1
+    assert sum(out[r][1] for r in range(world)) > 0, "the skew makes some rank run a redundant copy"
