@@ -316,6 +316,37 @@ def exchange_replica_weights(plan: BalancedPlan, home: dict, group=None) -> dict
     return out
 
 
+def balanced_step(z_perm: torch.Tensor, offsets: np.ndarray, bounds: np.ndarray, home: dict, run_experts, gather,
+                  group=None):
+    """One balanced exchange around this rank's expert computation.
+
+    z_perm [n, L]: this rank's expert-major token rows, offsets [E + 1] their
+    CSR offsets; home: name -> [n_home, ...] per-expert weight slices of this
+    rank's experts (sent to the ranks that run copies).  gather(src, idx) ->
+    src[idx] on idx int32 rows (the layer: moe_gather_rows);
+    run_experts(z_recv, exchange, plan, copies) -> fp32 outputs [n_recv, L]
+    for the received rows, copies being this rank's redundant experts' weight
+    slices.  Returns (y_perm [n, L] fp32 in expert-major order, plan,
+    exchange)."""
+    rank = dist.get_rank(group)
+    counts = gather_counts(offsets, group)
+    plan = balanced_plan(counts, bounds)
+    ex = balanced_exchange(plan, counts, offsets, rank)
+    copies = exchange_replica_weights(plan, home, group)
+    dev, n_send = z_perm.device, len(ex.send_idx)
+    z_send = gather(z_perm, torch.from_numpy(ex.send_idx.astype(np.int32)).to(dev))
+    z_recv = torch.empty((ex.n_recv,) + tuple(z_perm.shape[1:]), dtype=z_perm.dtype, device=dev)
+    dist.all_to_all_single(z_recv, z_send, output_split_sizes=ex.recv_rows, input_split_sizes=ex.send_rows,
+                           group=group)
+    y_recv = run_experts(z_recv, ex, plan, copies)
+    y_back = torch.empty((n_send,) + tuple(y_recv.shape[1:]), dtype=y_recv.dtype, device=dev)
+    dist.all_to_all_single(y_back, y_recv, output_split_sizes=ex.send_rows, input_split_sizes=ex.recv_rows,
+                           group=group)
+    inv = np.empty(n_send, np.int64)
+    inv[ex.send_idx] = np.arange(n_send)
+    return gather(y_back, torch.from_numpy(inv.astype(np.int32)).to(dev)), plan, ex
+
+
 class ExpertParallelMoeLayer:
     """One rank's share of an expert-parallel layer.
 
@@ -418,41 +449,31 @@ class ExpertParallelMoeLayer:
     def _balanced_experts(self, d: Dims, offsets: np.ndarray, z_perm: torch.Tensor, stream) -> torch.Tensor:
         """The balanced exchange: y_perm [T k, L] fp32 in expert-major order."""
         dev, L = z_perm.device, d.L
-        counts = gather_counts(offsets, self.group)
-        plan = balanced_plan(counts, self.bounds)
+
+        def gather(src: torch.Tensor, idx: torch.Tensor) -> torch.Tensor:
+            dst = torch.empty((len(idx),) + tuple(src.shape[1:]), dtype=src.dtype, device=dev)
+            check(moe_gather_rows(src, src.shape[0], src[0].numel() * src.element_size(), idx, len(idx), dst,
+                                  stream))
+            return dst
+
+        def run_experts(z_recv: torch.Tensor, ex: BalancedExchange, plan: BalancedPlan, copies: dict):
+            n_local = self.e_local + len(plan.replicas[self.rank])
+            if n_local - self.e_local > self._cap:
+                self._grow(max(n_local - self.e_local, 2 * self._cap))
+            for n, t in copies.items():
+                self._buf[n][self.e_local:n_local].copy_(t)
+            y_recv = torch.empty(ex.n_recv, L, dtype=torch.float32, device=dev)
+            if ex.n_recv > 0:
+                ld = replace(d, E=n_local)
+                blocks = torch.from_numpy(ex.recv_block_offsets.astype(np.int32)).to(dev)
+                ws = torch.empty(moe_expert_ffn_blocks_workspace_size(ld, ex.n_recv, self.G), dtype=torch.uint8,
+                                 device=dev)
+                check(moe_expert_ffn_blocks(ld, self._local_weights(n_local), z_recv, ex.n_recv, blocks, self.G,
+                                            y_recv, ws, None, stream))
+            return y_recv
+
+        y_perm, plan, _ = balanced_step(z_perm, offsets, self.bounds, self._home, run_experts, gather, self.group)
         self.last_plan = plan
-        ex = balanced_exchange(plan, counts, offsets, self.rank)
-        reps = plan.replicas[self.rank]
-        n_local = self.e_local + len(reps)
-        copies = exchange_replica_weights(plan, self._home, self.group)
-        if len(reps) > self._cap:
-            self._grow(max(len(reps), 2 * self._cap))
-        for n, t in copies.items():
-            self._buf[n][self.e_local:n_local].copy_(t)
-        # rows ordered by destination, dispatched, run, returned, put back
-        n_send = len(ex.send_idx)
-        idx = torch.from_numpy(ex.send_idx.astype(np.int32)).to(dev)
-        z_send = torch.empty_like(z_perm)
-        check(moe_gather_rows(z_perm, z_perm.shape[0], L * z_perm.element_size(), idx, n_send, z_send, stream))
-        z_recv = torch.empty(ex.n_recv, L, dtype=z_perm.dtype, device=dev)
-        dist.all_to_all_single(z_recv, z_send, output_split_sizes=ex.recv_rows, input_split_sizes=ex.send_rows,
-                               group=self.group)
-        y_recv = torch.empty(ex.n_recv, L, dtype=torch.float32, device=dev)
-        if ex.n_recv > 0:
-            ld = replace(d, E=n_local)
-            blocks = torch.from_numpy(ex.recv_block_offsets.astype(np.int32)).to(dev)
-            ws = torch.empty(moe_expert_ffn_blocks_workspace_size(ld, ex.n_recv, self.G), dtype=torch.uint8,
-                             device=dev)
-            check(moe_expert_ffn_blocks(ld, self._local_weights(n_local), z_recv, ex.n_recv, blocks, self.G, y_recv,
-                                        ws, None, stream))
-        y_back = torch.empty(n_send, L, dtype=torch.float32, device=dev)
-        dist.all_to_all_single(y_back, y_recv, output_split_sizes=ex.send_rows, input_split_sizes=ex.recv_rows,
-                               group=self.group)
-        inv = np.empty(n_send, np.int64)
-        inv[ex.send_idx] = np.arange(n_send)
-        inv_t = torch.from_numpy(inv.astype(np.int32)).to(dev)
-        y_perm = torch.empty(n_send, L, dtype=torch.float32, device=dev)
-        check(moe_gather_rows(y_back, n_send, L * 4, inv_t, n_send, y_perm, stream))
         return y_perm
 
     __call__ = forward

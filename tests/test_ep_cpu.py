@@ -221,47 +221,45 @@ def _balanced_worker(rank, world, port, E, k, out):
         counts_local, offsets, perm_token, inv_perm = oracle.permute(idx, E)
         z_perm = torch.from_numpy(z[perm_token])
         bounds = ep.partition(E, world)
-        counts = ep.gather_counts(offsets)
-        assert np.array_equal(counts[rank], counts_local)
-        plan = ep.balanced_plan(counts, bounds)
-        x = ep.balanced_exchange(plan, counts, offsets, rank)
-        # the layer orders rows with moe_gather_rows on the GPU; torch indexing here
-        z_send = z_perm[torch.from_numpy(x.send_idx)]
-        z_recv = torch.empty(x.n_recv, L)
-        dist.all_to_all_single(z_recv, z_send, output_split_sizes=x.recv_rows, input_split_sizes=x.send_rows)
-        assert x.n_recv == plan.quota[rank], "every rank runs its quota"
-        local = plan.local_experts(rank)
-        label = np.full(x.n_recv, -1)
-        for s in range(world):
-            b = x.recv_block_offsets[s]
-            for i, e in enumerate(local):
-                label[b[i]:b[i + 1]] = e
-        assert (label >= 0).all()
-        # the received rows are exactly the rows the plan assigns here
         everyone = [None] * world
-        dist.all_gather_object(everyone, (z_perm.numpy(), offsets))
-        dest = _row_destinations(plan, counts)
-        want = np.concatenate([everyone[s][0][np.nonzero(dest[s] == rank)[0]] for s in range(world)])
-        got_sorted = np.sort(z_recv.numpy(), axis=0)
-        assert np.array_equal(got_sorted, np.sort(want, axis=0)), "received rows"
-        # stand-in experts y = z * (e + 1); the results return to their senders
-        y_recv = z_recv * torch.from_numpy((label + 1).astype(np.float32))[:, None]
-        y_back = torch.empty(len(x.send_idx), L)
-        dist.all_to_all_single(y_back, y_recv, output_split_sizes=x.send_rows, input_split_sizes=x.recv_rows)
-        y_perm = torch.empty_like(y_back)
-        y_perm[torch.from_numpy(x.send_idx)] = y_back
-        expert_of_pos = np.repeat(np.arange(E), counts_local)
-        assert np.array_equal(y_perm.numpy(), z_perm.numpy() * (expert_of_pos + 1).astype(np.float32)[:, None])
-        # redundant copies: every rank receives the slices of the experts it runs without owning them
+        dist.all_gather_object(everyone, (z_perm.numpy(), counts_local))
+        counts = np.stack([c for _, c in everyone])
         lo, hi = bounds[rank], bounds[rank + 1]
+        # stand-in weight slices: every element of expert e's slice is e
         home = {"Wg": torch.arange(lo, hi, dtype=torch.float32)[:, None, None].repeat(1, 2, 3),
                 "So_tiled": (torch.arange(lo, hi, dtype=torch.int64)[:, None].repeat(1, 5) % 251).to(torch.uint8)}
-        copies = ep.exchange_replica_weights(plan, home)
-        reps = plan.replicas[rank]
-        assert copies["Wg"].shape == (len(reps), 2, 3) and copies["So_tiled"].shape == (len(reps), 5)
-        for i, e in enumerate(reps):
-            assert torch.all(copies["Wg"][i] == e) and torch.all(copies["So_tiled"][i] == e % 251)
-        out[rank] = (x.n_recv, len(reps))
+        seen = {}
+
+        def run_experts(z_recv, x, plan, copies):
+            # stand-in experts y = z * (e + 1), e the global id of each received row's expert
+            local = plan.local_experts(rank)
+            label = np.full(x.n_recv, -1)
+            for s in range(world):
+                b = x.recv_block_offsets[s]
+                for i, e in enumerate(local):
+                    label[b[i]:b[i + 1]] = e
+            assert (label >= 0).all()
+            reps = plan.replicas[rank]
+            assert copies["Wg"].shape == (len(reps), 2, 3) and copies["So_tiled"].shape == (len(reps), 5)
+            for i, e in enumerate(reps):
+                assert torch.all(copies["Wg"][i] == e) and torch.all(copies["So_tiled"][i] == e % 251)
+            seen["z_recv"], seen["reps"] = z_recv.clone(), len(reps)
+            return z_recv * torch.from_numpy((label + 1).astype(np.float32))[:, None]
+
+        # the layer's own step, with torch indexing for the gather the layer
+        # runs as moe_gather_rows on the GPU
+        y_perm, plan, x = ep.balanced_step(z_perm, offsets, bounds, home, run_experts,
+                                           lambda src, i: src[i.long()])
+        assert np.array_equal(plan.quota, ep.balanced_plan(counts, bounds).quota)
+        assert x.n_recv == plan.quota[rank], "every rank runs its quota"
+        # the received rows are exactly the rows the plan assigns here
+        dest = _row_destinations(plan, counts)
+        want = np.concatenate([everyone[s][0][np.nonzero(dest[s] == rank)[0]] for s in range(world)])
+        assert np.array_equal(np.sort(seen["z_recv"].numpy(), axis=0), np.sort(want, axis=0)), "received rows"
+        # the results are back in this rank's expert-major order
+        expert_of_pos = np.repeat(np.arange(E), counts_local)
+        assert np.array_equal(y_perm.numpy(), z_perm.numpy() * (expert_of_pos + 1).astype(np.float32)[:, None])
+        out[rank] = (x.n_recv, seen["reps"])
     finally:
         dist.destroy_process_group()
 
