@@ -298,6 +298,9 @@ def exchange_replica_weights(plan: BalancedPlan, home: dict, group=None) -> dict
     G = len(plan.quota)
     lo = int(plan.bounds[rank])
     out = {}
+    if not any(plan.replicas):
+        # every rank computes the same plan, so all skip the collectives together
+        return {name: t[:0] for name, t in home.items()}
     for name, t in home.items():
         per = t[0].numel() * t.element_size()
         flat = t.reshape(t.shape[0], -1).view(torch.uint8) if t.dtype != torch.uint8 else t.reshape(t.shape[0], -1)
@@ -347,6 +350,41 @@ def balanced_step(z_perm: torch.Tensor, offsets: np.ndarray, bounds: np.ndarray,
     return gather(y_back, torch.from_numpy(inv.astype(np.int32)).to(dev)), plan, ex
 
 
+class ExpertSlots:
+    """A rank's routed weights for the balanced mode: per tensor name one
+    buffer [n_home + capacity, ...] holding the rank's own expert slices
+    first and, behind them, the step's redundant copies, so that the local
+    expert set (own experts, then copies) is one contiguous prefix."""
+
+    def __init__(self, home: dict, capacity: int):
+        self.home = home
+        self.n_home = next(iter(home.values())).shape[0]
+        self.buf: dict = {}
+        self.capacity = 0
+        self.grow(capacity)
+
+    def grow(self, capacity: int) -> None:
+        for n, t in self.home.items():
+            b = torch.empty((self.n_home + capacity,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+            b[: self.n_home].copy_(t)
+            self.buf[n] = b
+        self.capacity = capacity
+
+    def place(self, copies: dict) -> int:
+        """Writes the step's copies behind the own experts (growing the
+        buffers if needed); returns the local expert count."""
+        n_rep = next(iter(copies.values())).shape[0] if copies else 0
+        if n_rep > self.capacity:
+            self.grow(max(n_rep, 2 * self.capacity))
+        for n, t in copies.items():
+            self.buf[n][self.n_home:self.n_home + n_rep].copy_(t)
+        return self.n_home + n_rep
+
+    def local(self, n_local: int) -> dict:
+        """name -> the first n_local expert slices (views, no copy)."""
+        return {n: b[:n_local] for n, b in self.buf.items()}
+
+
 class ExpertParallelMoeLayer:
     """One rank's share of an expert-parallel layer.
 
@@ -388,20 +426,10 @@ class ExpertParallelMoeLayer:
                 ["Sgv_tiled", "So_tiled"] if dims.routed in BLOCK_SCALED else [])
             self._home = {n: self.weights[n].reshape((self.e_local, -1) if n.endswith("_tiled") else
                                                      tuple(self.weights[n].shape)) for n in names}
-            self._buf = {}
-            self._grow(self.e_local)
-
-    def _grow(self, cap: int) -> None:
-        """Routed-weight buffers for this rank's experts and up to cap
-        redundant copies."""
-        for n, t in self._home.items():
-            b = torch.empty((self.e_local + cap,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
-            b[: self.e_local].copy_(t)
-            self._buf[n] = b
-        self._cap = cap
+            self._slots = ExpertSlots(self._home, self.e_local)
 
     def _local_weights(self, n_local: int):
-        w = {n: (b[:n_local].reshape(-1) if n.endswith("_tiled") else b[:n_local]) for n, b in self._buf.items()}
+        w = {n: (t.reshape(-1) if n.endswith("_tiled") else t) for n, t in self._slots.local(n_local).items()}
         return make_weights(**w)
 
     def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
@@ -457,11 +485,8 @@ class ExpertParallelMoeLayer:
             return dst
 
         def run_experts(z_recv: torch.Tensor, ex: BalancedExchange, plan: BalancedPlan, copies: dict):
-            n_local = self.e_local + len(plan.replicas[self.rank])
-            if n_local - self.e_local > self._cap:
-                self._grow(max(n_local - self.e_local, 2 * self._cap))
-            for n, t in copies.items():
-                self._buf[n][self.e_local:n_local].copy_(t)
+            n_local = self._slots.place(copies)
+            assert n_local == len(plan.local_experts(self.rank))
             y_recv = torch.empty(ex.n_recv, L, dtype=torch.float32, device=dev)
             if ex.n_recv > 0:
                 ld = replace(d, E=n_local)

@@ -195,6 +195,18 @@ def test_block_scaled_path_validates(routed):
         assert q(None, 0, 64, None, None, 0) == moe.MOE_OK               # nothing to do
 
 
+def test_gather_rows_validates_on_the_host():
+    """moe_gather_rows checks its arguments before any launch."""
+    assert moe.moe_gather_rows(FAKE, 4, 32, FAKE, 0, FAKE, 0) == moe.MOE_OK            # nothing to do
+    assert moe.moe_gather_rows(None, 0, 32, None, 0, None, 0) == moe.MOE_OK
+    assert moe.moe_gather_rows(FAKE, 4, 24, FAKE, 2, FAKE, 0) == moe.MOE_ERR_INVALID_ARG  # row not 16-byte multiple
+    assert moe.moe_gather_rows(FAKE, 4, 0, FAKE, 2, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_gather_rows(FAKE, 4, 32, FAKE, -1, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_gather_rows(FAKE, -1, 32, FAKE, 2, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_gather_rows(FAKE, 4, 32, None, 2, FAKE, 0) == moe.MOE_ERR_INVALID_ARG   # no index array
+    assert moe.moe_gather_rows(FAKE + 8, 4, 32, FAKE, 2, FAKE, 0) == moe.MOE_ERR_INVALID_ARG  # misaligned
+
+
 def test_structs_keep_their_tensors_alive():
     """make_weights / make_aux / make_grads hold the tensors whose addresses
     they carry, so a tensor built for the call is not freed (and its memory

@@ -275,3 +275,46 @@ def test_gloo_balanced_exchange(world, E, k):
     loads = [out[r][0] for r in range(world)]
     assert max(loads) - min(loads) <= 1
     assert sum(out[r][1] for r in range(world)) > 0, "the skew makes some rank run a redundant copy"
+
+
+def test_expert_slots_place_copies_behind_own_experts():
+    """The balanced layer's weight buffers: own slices first, the step's
+    copies behind them, growing when a step needs more copies than fit; the
+    local views are prefixes (no copy) and the own slices never change."""
+    home = {"Wg": torch.arange(3, dtype=torch.float32)[:, None, None].repeat(1, 2, 4),
+            "So_tiled": torch.arange(3, dtype=torch.uint8)[:, None].repeat(1, 7)}
+    slots = ep.ExpertSlots(home, capacity=1)
+    assert slots.place({n: t[:0] for n, t in home.items()}) == 3
+    assert torch.equal(slots.local(3)["Wg"], home["Wg"])
+    copies = {"Wg": torch.full((2, 2, 4), 9.0), "So_tiled": torch.full((2, 7), 9, dtype=torch.uint8)}
+    assert slots.place(copies) == 5 and slots.capacity >= 2            # grown
+    loc = slots.local(5)
+    assert torch.equal(loc["Wg"][:3], home["Wg"]) and torch.all(loc["Wg"][3:] == 9)
+    assert torch.all(loc["So_tiled"][3:] == 9) and torch.equal(loc["So_tiled"][:3], home["So_tiled"])
+    assert loc["Wg"].data_ptr() == slots.buf["Wg"].data_ptr()         # a view of the buffer
+    one = {"Wg": torch.full((1, 2, 4), 4.0), "So_tiled": torch.full((1, 7), 4, dtype=torch.uint8)}
+    assert slots.place(one) == 4 and torch.all(slots.local(4)["Wg"][3] == 4)
+    assert torch.equal(slots.local(3)["Wg"], home["Wg"])
+
+
+def _no_copy_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        counts = np.array([[3, 1, 2, 2], [1, 3, 2, 2]])  # every rank already at its quota (8 rows)
+        plan = ep.balanced_plan(counts, ep.partition(4, world))
+        assert not any(plan.replicas)
+        home = {"Wg": torch.zeros(2, 3)}
+        copies = ep.exchange_replica_weights(plan, home)
+        out[rank] = tuple(copies["Wg"].shape)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_no_copies_no_weight_exchange():
+    """A plan without copies returns empty copy sets on every rank (the ranks
+    skip the weight collectives together)."""
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_no_copy_worker, args=(2, _free_port(), out), nprocs=2, join=True)
+    assert out[0] == out[1] == (0, 3)
