@@ -386,18 +386,45 @@ def measure_e2e(layer, x, y, cfg, args, world: int) -> float:
     return ms
 
 
-def near_ties_from_scores(layer, x, cfg) -> int:
-    """Tokens of the whole batch whose device-side selection margin (k-th minus
-    (k+1)-th largest fp32 key s + b) is below NEAR_TIE: where a device and the
-    fp64 oracle may legitimately choose different experts.  Outside any timed
-    region; the scores come from the layer itself (aux output)."""
-    if cfg.k >= cfg.E:
-        return 0
+def routing_of_batch(layer, x, cfg) -> tuple[int, np.ndarray]:
+    """(near-tie tokens, the device's expert choice [T, k]) of the whole batch.
+    Near ties: tokens whose device-side selection margin (k-th minus (k+1)-th
+    largest fp32 key s + b) is below NEAR_TIE, where a device and the fp64
+    oracle may legitimately choose different experts.  Outside any timed
+    region; scores and choice come from the layer itself (aux outputs)."""
     s = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=x.device)
-    layer.forward(x, aux={"scores": s})
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=x.device)
+    layer.forward(x, aux={"scores": s, "topk_idx": idx})
+    idx_np = idx.cpu().numpy().astype(np.int64)
+    if cfg.k >= cfg.E:
+        return 0, idx_np
     key = s + layer.weights["bias"][None, :]
     top = torch.topk(key, cfg.k + 1, dim=1).values
-    return int(((top[:, cfg.k - 1] - top[:, cfg.k]) < NEAR_TIE).sum())
+    return int(((top[:, cfg.k - 1] - top[:, cfg.k]) < NEAR_TIE).sum()), idx_np
+
+
+def ep_balance(idx: np.ndarray, E: int, G: int = 8) -> dict:
+    """The balanced expert-parallel plan (expert_parallel.balanced_plan) on
+    this batch's routing, its tokens cut into G contiguous chunks taken as G
+    ranks' batches: the largest rank load over the mean with experts split
+    over the ranks by the static partition (every row to its expert's owner)
+    and with the balanced plan, and the redundant expert copies that plan
+    runs.  A host computation outside the timed region; nothing is timed."""
+    from sparse_moe_layer_renormalised_b200 import expert_parallel as ep
+
+    chunks = np.array_split(np.arange(idx.shape[0]), G)
+    counts = np.stack([np.bincount(idx[c].reshape(-1), minlength=E) for c in chunks]).astype(np.int64)
+    bounds = ep.partition(E, G)
+    plan = ep.balanced_plan(counts, bounds)
+    C = counts.sum(axis=0)
+    mean = float(C.sum()) / G
+    static = np.array([C[bounds[g]:bounds[g + 1]].sum() for g in range(G)])
+    return {"ranks": G, "rows": int(C.sum()),
+            "static_max_over_mean": round(float(static.max()) / mean, 4),
+            "balanced_max_over_mean": round(float(plan.quota.max()) / mean, 4),
+            "copies": int(sum(len(r) for r in plan.replicas)),
+            "max_copies_per_rank": int(max(len(r) for r in plan.replicas)),
+            "how": "the batch's tokens in G contiguous chunks as the ranks' batches; host planning only"}
 
 
 def oracle_sample(cfg, layer, x, n_tokens: int, seed_offset: int = 0) -> tuple[dict, dict]:
@@ -498,7 +525,9 @@ def workload_line(cfg, layer, x, args, world, rank, local_rank, peaks, headline:
         },
     }
     if world == 1:
-        out["near_tie_tokens"] = near_ties_from_scores(layer, x, cfg)
+        out["near_tie_tokens"], idx = routing_of_batch(layer, x, cfg)
+        if cfg.E >= 8:
+            out["ep_balance"] = ep_balance(idx, cfg.E)
         if not args.no_oracle:
             parity, cpu = oracle_sample(cfg, layer, x, args.cpu_tokens)
             out["parity"] = parity

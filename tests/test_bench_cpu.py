@@ -66,3 +66,45 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_ep_balance_statistic():
+    """The balanced plan's per-rank load on a skewed routing: the static
+    partition's largest rank is well above the mean, the balanced plan's at
+    most one row above it, and the copies are counted."""
+    rng = np.random.default_rng(3)
+    E, k, T = 64, 4, 2000
+    w = (np.arange(E) + 1.0) ** -1.0
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=w / w.sum()) for _ in range(T)])
+    st = bench.ep_balance(idx, E, G=8)
+    assert st["rows"] == T * k and st["ranks"] == 8
+    assert st["static_max_over_mean"] > 1.5                       # the hot experts sit on rank 0
+    assert st["balanced_max_over_mean"] <= 1.0 + 8 / (T * k) + 1e-9
+    assert st["copies"] >= 1 and st["max_copies_per_rank"] >= 1
+
+
+def test_routing_of_batch_logic_on_cpu():
+    """routing_of_batch's host logic with a stand-in layer that fills the
+    same aux outputs as MoeLayer.forward (scores, topk_idx): the near-tie
+    count and the choice it returns."""
+    import torch
+
+    class FakeLayer:
+        def __init__(self, scores, bias, idx):
+            self.s, self.idx = scores, idx
+            self.weights = {"bias": bias}
+
+        def forward(self, x, aux):
+            aux["scores"].copy_(self.s)
+            aux["topk_idx"].copy_(self.idx)
+
+    cfg = gen.CONFIGS["tiny"]
+    g = torch.Generator().manual_seed(4)
+    s = torch.rand(cfg.T, cfg.E, generator=g)
+    s[0, :cfg.k + 1] = 0.9                      # token 0: the k-th and (k+1)-th keys tie
+    bias = torch.zeros(cfg.E)
+    idx = torch.topk(s, cfg.k, dim=1).indices.to(torch.int32)
+    n_tie, got = bench.routing_of_batch(FakeLayer(s, bias, idx), torch.zeros(1), cfg)
+    assert n_tie >= 1 and got.dtype == np.int64 and np.array_equal(got, idx.numpy())
+    st = bench.ep_balance(got, cfg.E)
+    assert st["rows"] == cfg.T * cfg.k
