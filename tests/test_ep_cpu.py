@@ -318,3 +318,112 @@ def test_no_copies_no_weight_exchange():
     out = mgr.dict()
     mp.spawn(_no_copy_worker, args=(2, _free_port(), out), nprocs=2, join=True)
     assert out[0] == out[1] == (0, 3)
+
+
+# ------------------------------------------------------------------------------ the layer's own step on gloo
+def _fake_library(layer, cfg, wd):
+    """fp64 oracle stand-ins for the library entries the expert-parallel layer
+    calls, with the library's argument lists, so that the layer's own step runs
+    on CPU ranks.  The routed experts read the layer's own local weight set
+    (its experts, then its redundant copies), which is what the test checks."""
+    F64 = torch.float64
+    rnd = oracle.storage_round(cfg.act)
+    state = {}
+
+    def router_topk(d, x, Wr, bias, scores, from_scores, idx, p, stream=None):
+        s = oracle.router_scores(x.to(F64), wd["Wr"])
+        i, pp, _ = oracle.select_experts(s, wd["bias"], d.k)
+        scores.copy_(s)
+        idx.copy_(i)
+        p.copy_(pp)
+        return 0
+
+    def latent_shared(d, w, x, z, h_s, stream=None):
+        xf = x.to(F64)
+        z.copy_(rnd(xf @ wd["Wdown"].T))
+        state["y_shared"] = oracle.shared_experts(xf, wd["Wsg"], wd["Wsv"], wd["Wso"], cfg.situ_c, rnd)
+        return 0
+
+    def permute(d, idx, z, offsets, perm_token, inv_perm, z_perm, ws, ws_bytes=None, stream=None):
+        _, off, pt, ip = oracle.permute(idx.numpy().astype(np.int64), d.E)
+        offsets.copy_(torch.from_numpy(off))
+        perm_token.copy_(torch.from_numpy(pt))
+        inv_perm.copy_(torch.from_numpy(ip))
+        z_perm.copy_(z[torch.from_numpy(pt).long()])
+        return 0
+
+    def gather_rows(src, src_rows, row_bytes, idx, n, dst, stream=None):
+        dst.copy_(src[idx.long()])
+        return 0
+
+    def expert_ffn_blocks(d, w, x_rows, n_rows, blocks, n_blocks, y_rows, ws, ws_bytes=None, stream=None):
+        loc = layer._slots.local(d.E) if layer.balance else {n: layer.weights[n] for n in ("Wg", "Wv", "Wo")}
+        b = blocks.numpy().reshape(n_blocks, d.E + 1)
+        for s in range(n_blocks):
+            for i in range(d.E):
+                lo, hi = int(b[s, i]), int(b[s, i + 1])
+                if lo < hi:
+                    y_rows[lo:hi] = oracle.expert_forward(x_rows[lo:hi].to(F64), loc["Wg"][i].to(F64),
+                                                          loc["Wv"][i].to(F64), loc["Wo"][i].to(F64), cfg.situ_c,
+                                                          rnd).to(y_rows.dtype)
+        return 0
+
+    def combine(d, y_perm, inv_perm, p, gamma, u_out, n_out, stream=None):
+        T, k = p.shape
+        u = oracle.combine(y_perm.to(F64)[inv_perm.long()].reshape(T, k, -1), p.to(F64))
+        n_out.copy_(rnd(oracle.rms_norm(u, wd["gamma"], cfg.rms_eps)))
+        return 0
+
+    def output(d, w, h_s, n, y, stream=None):
+        y.copy_(state["y_shared"] + n.to(F64) @ wd["Wup"].T)
+        return 0
+
+    return {"moe_router_topk": router_topk, "moe_latent_shared": latent_shared, "moe_permute": permute,
+            "moe_gather_rows": gather_rows, "moe_expert_ffn_blocks": expert_ffn_blocks, "moe_combine": combine,
+            "moe_output": output}
+
+
+def _layer_worker(rank, world, port, balance, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import gen
+        from oracle import inputs as oin
+        from sparse_moe_layer_renormalised_b200 import Dims
+
+        T_r = 24
+        cfg = gen.CONFIGS["tiny"].with_(T=T_r * world)
+        wd = oin.all_weights(cfg)                       # fp64, the generator's fp32 values
+        bounds = ep.partition(cfg.E, world)
+        lo, hi = int(bounds[rank]), int(bounds[rank + 1])
+        w = {n: wd[n].to(torch.float32) for n in ("Wr", "bias", "Wdown", "Wup", "gamma", "Wsg", "Wsv", "Wso")}
+        w.update({n: wd[n][lo:hi].to(torch.float32).contiguous() for n in ("Wg", "Wv", "Wo")})
+        dims = Dims(T=T_r, H=cfg.H, L=cfg.L, E=cfg.E, k=cfg.k, I=cfg.I, S=cfg.S, Is=cfg.Is, act="f32", routed="f32",
+                    y_out="f32", situ_c=cfg.situ_c, rms_eps=cfg.rms_eps)
+        layer = ep.ExpertParallelMoeLayer(dims, w, balance=balance)
+        for name, f in _fake_library(layer, cfg, wd).items():
+            setattr(ep, name, f)
+        x = oin.x_rows(cfg, np.arange(rank * T_r, (rank + 1) * T_r))
+        y = layer(x.to(torch.float32))
+        ref = oracle.layer_forward(cfg, wd, x)["y"]
+        err = float((y.to(torch.float64) - ref).abs().max() / ref.pow(2).mean().sqrt())
+        copies = len(layer.last_plan.replicas[rank]) if balance else 0
+        out[rank] = (err, copies)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,balance", [(2, True), (3, True), (3, False)])
+def test_gloo_layer_step_matches_the_oracle(world, balance):
+    """The expert-parallel layer's own forward step on gloo ranks, each with
+    its own tokens and only its own experts' weights, the library entries
+    replaced by fp64 oracle stand-ins: every rank's y equals the oracle layer
+    on its tokens (fp32 storage between the steps), in the balanced mode with
+    redundant copies whose weights came from other ranks."""
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_layer_worker, args=(world, _free_port(), balance, out), nprocs=world, join=True)
+    for r in range(world):
+        assert out[r][0] <= 1e-5, (r, out[r])
+    if balance:
+        assert sum(out[r][1] for r in range(world)) > 0, "some rank ran a redundant copy"
