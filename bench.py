@@ -15,7 +15,9 @@ The default run measures five K3-shape workloads, one after the other:
             all-4-bit block-scaled MMA             -> "mxfp4-a4" sub-object
 (H=7168, L=3584, 896 experts top-16, I=3072, 2 shared experts, Is=3072).
 Each line carries its own device time, stage times, roofline, end-to-end
-number, near-tie count and an oracle sample (parity and CPU baseline).
+number, near-tie count, an oracle sample (parity and CPU baseline) and the
+balanced expert-parallel plan of its batch on 8 ranks (ep_balance, host
+planning only).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--no-extra-lines]
   python bench.py --impl reference ...     # the CPU oracle on a bounded sample
