@@ -289,59 +289,76 @@ def gather_counts(offsets: np.ndarray, group=None) -> np.ndarray:
     return torch.stack(out).cpu().numpy()
 
 
-def exchange_replica_weights(plan: BalancedPlan, home: dict, group=None) -> dict:
-    """Sends every redundant expert's weights from its owner to the ranks
-    that run it this step.  home: name -> [n_home, ...] tensor of this rank's
-    experts (one slice per expert); returns name -> [len(replicas[rank]), ...]
-    with the slices of this rank's redundant experts in ascending id order."""
+def exchange_expert_slices(want: list, bounds: np.ndarray, home: dict, group=None) -> dict:
+    """Sends expert weight slices from their owners to the ranks that ask for
+    them.  want[g]: ascending ids of the experts rank g needs (none of its
+    own), the same list on every rank; home: name -> [n_home, ...] tensor of
+    this rank's experts, one slice per expert.  Returns name -> [len(want[rank]),
+    ...], the requested slices in ascending id order.  When nobody asks for
+    anything every rank returns empty tensors without a collective."""
     rank = dist.get_rank(group)
-    G = len(plan.quota)
-    lo = int(plan.bounds[rank])
-    out = {}
-    if not any(plan.replicas):
-        # every rank computes the same plan, so all skip the collectives together
+    G = len(bounds) - 1
+    lo = int(bounds[rank])
+    if not any(want):
         return {name: t[:0] for name, t in home.items()}
+    out = {}
     for name, t in home.items():
         per = t[0].numel() * t.element_size()
         flat = t.reshape(t.shape[0], -1).view(torch.uint8) if t.dtype != torch.uint8 else t.reshape(t.shape[0], -1)
         send, send_sizes = [], []
         for g in range(G):
-            mine = [e - lo for e in plan.replicas[g] if plan.bounds[rank] <= e < plan.bounds[rank + 1]]
+            mine = [e - lo for e in want[g] if bounds[rank] <= e < bounds[rank + 1]]
             send += [flat[i] for i in mine]
             send_sizes.append(per * len(mine))
-        recv_sizes = [per * sum(1 for e in plan.replicas[rank] if plan.bounds[s] <= e < plan.bounds[s + 1])
-                      for s in range(G)]
+        recv_sizes = [per * sum(1 for e in want[rank] if bounds[s] <= e < bounds[s + 1]) for s in range(G)]
         sbuf = torch.cat(send) if send else torch.zeros(0, dtype=torch.uint8, device=t.device)
         rbuf = torch.empty(sum(recv_sizes), dtype=torch.uint8, device=t.device)
         dist.all_to_all_single(rbuf, sbuf.contiguous(), output_split_sizes=recv_sizes, input_split_sizes=send_sizes,
                                group=group)
-        out[name] = rbuf.view(t.dtype).reshape((len(plan.replicas[rank]),) + tuple(t.shape[1:]))
+        out[name] = rbuf.view(t.dtype).reshape((len(want[rank]),) + tuple(t.shape[1:]))
     return out
 
 
+def exchange_replica_weights(plan: BalancedPlan, home: dict, group=None) -> dict:
+    """Every redundant expert's weights from its owner to the ranks that run
+    it this step: name -> [len(replicas[rank]), ...] in ascending id order."""
+    return exchange_expert_slices(plan.replicas, plan.bounds, home, group)
+
+
+def missing_copies(plan: BalancedPlan, held: list | None) -> list:
+    """Per rank, the redundant experts of the plan whose weights it does not
+    hold yet (held[g]: the copies rank g kept from earlier steps)."""
+    if held is None:
+        return [list(r) for r in plan.replicas]
+    return [[e for e in plan.replicas[g] if e not in set(held[g])] for g in range(len(plan.quota))]
+
+
 def balanced_step(z_perm: torch.Tensor, offsets: np.ndarray, bounds: np.ndarray, home: dict, run_experts, gather,
-                  group=None):
+                  group=None, held: list | None = None):
     """One balanced exchange around this rank's expert computation.
 
     z_perm [n, L]: this rank's expert-major token rows, offsets [E + 1] their
     CSR offsets; home: name -> [n_home, ...] per-expert weight slices of this
-    rank's experts (sent to the ranks that run copies).  gather(src, idx) ->
-    src[idx] on idx int32 rows (the layer: moe_gather_rows);
-    run_experts(z_recv, exchange, plan, copies) -> fp32 outputs [n_recv, L]
-    for the received rows, copies being this rank's redundant experts' weight
-    slices.  Returns (y_perm [n, L] fp32 in expert-major order, plan,
+    rank's experts (sent to the ranks that run copies); held (optional, the
+    same on every rank): per rank the copies it kept from earlier steps,
+    which are not sent again.  gather(src, idx) -> src[idx] on idx int32 rows
+    (the layer: moe_gather_rows); run_experts(z_recv, exchange, plan, copies,
+    copy_ids) -> fp32 outputs [n_recv, L] for the received rows, copies being
+    the weight slices of this rank's redundant experts copy_ids (those it did
+    not hold).  Returns (y_perm [n, L] fp32 in expert-major order, plan,
     exchange)."""
     rank = dist.get_rank(group)
     counts = gather_counts(offsets, group)
     plan = balanced_plan(counts, bounds)
     ex = balanced_exchange(plan, counts, offsets, rank)
-    copies = exchange_replica_weights(plan, home, group)
+    want = missing_copies(plan, held)
+    copies = exchange_expert_slices(want, plan.bounds, home, group)
     dev, n_send = z_perm.device, len(ex.send_idx)
     z_send = gather(z_perm, torch.from_numpy(ex.send_idx.astype(np.int32)).to(dev))
     z_recv = torch.empty((ex.n_recv,) + tuple(z_perm.shape[1:]), dtype=z_perm.dtype, device=dev)
     dist.all_to_all_single(z_recv, z_send, output_split_sizes=ex.recv_rows, input_split_sizes=ex.send_rows,
                            group=group)
-    y_recv = run_experts(z_recv, ex, plan, copies)
+    y_recv = run_experts(z_recv, ex, plan, copies, want[rank])
     y_back = torch.empty((n_send,) + tuple(y_recv.shape[1:]), dtype=y_recv.dtype, device=dev)
     dist.all_to_all_single(y_back, y_recv, output_split_sizes=ex.send_rows, input_split_sizes=ex.recv_rows,
                            group=group)
@@ -353,36 +370,59 @@ def balanced_step(z_perm: torch.Tensor, offsets: np.ndarray, bounds: np.ndarray,
 class ExpertSlots:
     """A rank's routed weights for the balanced mode: per tensor name one
     buffer [n_home + capacity, ...] holding the rank's own expert slices
-    first and, behind them, the step's redundant copies, so that the local
-    expert set (own experts, then copies) is one contiguous prefix."""
+    first and, behind them, its redundant copies in ascending id order
+    (`held`), so that the local expert set (own experts, then copies) is one
+    contiguous prefix.  Copies stay from one step to the next; a step whose
+    plan repeats a copy does not receive it again."""
 
     def __init__(self, home: dict, capacity: int):
         self.home = home
         self.n_home = next(iter(home.values())).shape[0]
         self.buf: dict = {}
+        self.held: list = []
         self.capacity = 0
         self.grow(capacity)
 
     def grow(self, capacity: int) -> None:
+        """Room for `capacity` copies; the own slices and the held copies move along."""
+        keep = self.n_home + len(self.held)
         for n, t in self.home.items():
             b = torch.empty((self.n_home + capacity,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
-            b[: self.n_home].copy_(t)
+            if n in self.buf:
+                b[:keep].copy_(self.buf[n][:keep])
+            else:
+                b[: self.n_home].copy_(t)
             self.buf[n] = b
         self.capacity = capacity
 
-    def place(self, copies: dict) -> int:
-        """Writes the step's copies behind the own experts (growing the
-        buffers if needed); returns the local expert count."""
-        n_rep = next(iter(copies.values())).shape[0] if copies else 0
+    def place(self, copies: dict, ids: list, replicas: list) -> int:
+        """Arranges this step's copies, `replicas` (ascending ids), behind the
+        own experts: `copies` holds the slices of `ids` (the copies not held
+        yet, ascending), the rest come from the held copies.  Returns the local
+        expert count."""
+        n_rep = len(replicas)
         if n_rep > self.capacity:
             self.grow(max(n_rep, 2 * self.capacity))
+        h = len(self.held)
+        old = {e: i for i, e in enumerate(self.held)}
+        new = {e: h + i for i, e in enumerate(ids)}
+        if any(e not in old and e not in new for e in replicas):
+            raise ValueError("a redundant copy is neither held nor received")
+        src = [new[e] if e in new else old[e] for e in replicas]
         for n, t in copies.items():
-            self.buf[n][self.n_home:self.n_home + n_rep].copy_(t)
+            pool = torch.cat([self.buf[n][self.n_home:self.n_home + h], t])  # a fresh tensor: no aliasing
+            idx = torch.tensor(src, dtype=torch.long, device=pool.device)
+            self.buf[n][self.n_home:self.n_home + n_rep].copy_(pool.index_select(0, idx))
+        self.held = list(replicas)
         return self.n_home + n_rep
 
     def local(self, n_local: int) -> dict:
         """name -> the first n_local expert slices (views, no copy)."""
         return {n: b[:n_local] for n, b in self.buf.items()}
+
+    def forget(self) -> None:
+        """Drops the held copies (after the owners' weights changed)."""
+        self.held = []
 
 
 class ExpertParallelMoeLayer:
@@ -427,6 +467,7 @@ class ExpertParallelMoeLayer:
             self._home = {n: self.weights[n].reshape((self.e_local, -1) if n.endswith("_tiled") else
                                                      tuple(self.weights[n].shape)) for n in names}
             self._slots = ExpertSlots(self._home, self.e_local)
+            self._held = None  # per rank, the copies kept from the last step (the same list on every rank)
 
     def _local_weights(self, n_local: int):
         w = {n: (t.reshape(-1) if n.endswith("_tiled") else t) for n, t in self._slots.local(n_local).items()}
@@ -484,8 +525,8 @@ class ExpertParallelMoeLayer:
                                   stream))
             return dst
 
-        def run_experts(z_recv: torch.Tensor, ex: BalancedExchange, plan: BalancedPlan, copies: dict):
-            n_local = self._slots.place(copies)
+        def run_experts(z_recv: torch.Tensor, ex: BalancedExchange, plan: BalancedPlan, copies: dict, ids: list):
+            n_local = self._slots.place(copies, ids, plan.replicas[self.rank])
             assert n_local == len(plan.local_experts(self.rank))
             y_recv = torch.empty(ex.n_recv, L, dtype=torch.float32, device=dev)
             if ex.n_recv > 0:
@@ -497,8 +538,17 @@ class ExpertParallelMoeLayer:
                                             y_recv, ws, None, stream))
             return y_recv
 
-        y_perm, plan, _ = balanced_step(z_perm, offsets, self.bounds, self._home, run_experts, gather, self.group)
+        y_perm, plan, _ = balanced_step(z_perm, offsets, self.bounds, self._home, run_experts, gather, self.group,
+                                        held=self._held)
         self.last_plan = plan
+        self._held = [list(r) for r in plan.replicas]
         return y_perm
+
+    def forget_copies(self) -> None:
+        """Call on every rank after the routed weights changed: the redundant
+        copies kept from earlier steps are dropped and sent again when needed."""
+        if self.balance:
+            self._held = None
+            self._slots.forget()
 
     __call__ = forward

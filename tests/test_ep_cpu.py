@@ -230,7 +230,7 @@ def _balanced_worker(rank, world, port, E, k, out):
                 "So_tiled": (torch.arange(lo, hi, dtype=torch.int64)[:, None].repeat(1, 5) % 251).to(torch.uint8)}
         seen = {}
 
-        def run_experts(z_recv, x, plan, copies):
+        def run_experts(z_recv, x, plan, copies, ids):
             # stand-in experts y = z * (e + 1), e the global id of each received row's expert
             local = plan.local_experts(rank)
             label = np.full(x.n_recv, -1)
@@ -240,6 +240,7 @@ def _balanced_worker(rank, world, port, E, k, out):
                     label[b[i]:b[i + 1]] = e
             assert (label >= 0).all()
             reps = plan.replicas[rank]
+            assert ids == reps, "without held copies every copy arrives"
             assert copies["Wg"].shape == (len(reps), 2, 3) and copies["So_tiled"].shape == (len(reps), 5)
             for i, e in enumerate(reps):
                 assert torch.all(copies["Wg"][i] == e) and torch.all(copies["So_tiled"][i] == e % 251)
@@ -279,22 +280,40 @@ def test_gloo_balanced_exchange(world, E, k):
 
 def test_expert_slots_place_copies_behind_own_experts():
     """The balanced layer's weight buffers: own slices first, the step's
-    copies behind them, growing when a step needs more copies than fit; the
-    local views are prefixes (no copy) and the own slices never change."""
-    home = {"Wg": torch.arange(3, dtype=torch.float32)[:, None, None].repeat(1, 2, 4),
-            "So_tiled": torch.arange(3, dtype=torch.uint8)[:, None].repeat(1, 7)}
+    copies behind them in ascending id order, growing when a step needs more
+    copies than fit; copies held from the previous step are reused (only
+    new ones arrive), the own slices never change, and the local views are
+    prefixes of the buffers."""
+    def sl(ids):
+        return {"Wg": torch.tensor(ids, dtype=torch.float32)[:, None, None].repeat(1, 2, 4),
+                "So_tiled": (torch.tensor(ids, dtype=torch.int64)[:, None].repeat(1, 7) % 251).to(torch.uint8)}
+
+    home = sl([0, 1, 2])
     slots = ep.ExpertSlots(home, capacity=1)
-    assert slots.place({n: t[:0] for n, t in home.items()}) == 3
+    assert slots.place(sl([]), [], []) == 3
     assert torch.equal(slots.local(3)["Wg"], home["Wg"])
-    copies = {"Wg": torch.full((2, 2, 4), 9.0), "So_tiled": torch.full((2, 7), 9, dtype=torch.uint8)}
-    assert slots.place(copies) == 5 and slots.capacity >= 2            # grown
-    loc = slots.local(5)
-    assert torch.equal(loc["Wg"][:3], home["Wg"]) and torch.all(loc["Wg"][3:] == 9)
-    assert torch.all(loc["So_tiled"][3:] == 9) and torch.equal(loc["So_tiled"][:3], home["So_tiled"])
-    assert loc["Wg"].data_ptr() == slots.buf["Wg"].data_ptr()         # a view of the buffer
-    one = {"Wg": torch.full((1, 2, 4), 4.0), "So_tiled": torch.full((1, 7), 4, dtype=torch.uint8)}
-    assert slots.place(one) == 4 and torch.all(slots.local(4)["Wg"][3] == 4)
-    assert torch.equal(slots.local(3)["Wg"], home["Wg"])
+
+    def check(replicas):
+        loc = slots.local(3 + len(replicas))
+        assert torch.equal(loc["Wg"][:3], home["Wg"]) and torch.equal(loc["So_tiled"][:3], home["So_tiled"])
+        for i, e in enumerate(replicas):
+            assert torch.all(loc["Wg"][3 + i] == e) and torch.all(loc["So_tiled"][3 + i] == e % 251)
+        assert slots.held == replicas
+
+    assert slots.place(sl([9, 40]), [9, 40], [9, 40]) == 5 and slots.capacity >= 2  # grown
+    check([9, 40])
+    assert slots.local(5)["Wg"].data_ptr() == slots.buf["Wg"].data_ptr()           # a view of the buffer
+    # next step: 9 and 40 are held; only 17 and 300 arrive; the order is by id
+    assert slots.place(sl([17, 300]), [17, 300], [9, 17, 40, 300]) == 7
+    check([9, 17, 40, 300])
+    # a step that drops copies and reuses one
+    assert slots.place(sl([]), [], [40]) == 4
+    check([40])
+    with pytest.raises(ValueError):
+        slots.place(sl([]), [], [40, 41])      # 41 neither held nor received
+    slots.forget()
+    assert slots.held == [] and slots.place(sl([5]), [5], [5]) == 4
+    check([5])
 
 
 def _no_copy_worker(rank, world, port, out):
@@ -392,7 +411,7 @@ def _layer_worker(rank, world, port, balance, out):
         from sparse_moe_layer_renormalised_b200 import Dims
 
         T_r = 24
-        cfg = gen.CONFIGS["tiny"].with_(T=T_r * world)
+        cfg = gen.CONFIGS["tiny"].with_(T=2 * T_r * world)
         wd = oin.all_weights(cfg)                       # fp64, the generator's fp32 values
         bounds = ep.partition(cfg.E, world)
         lo, hi = int(bounds[rank]), int(bounds[rank + 1])
@@ -403,12 +422,27 @@ def _layer_worker(rank, world, port, balance, out):
         layer = ep.ExpertParallelMoeLayer(dims, w, balance=balance)
         for name, f in _fake_library(layer, cfg, wd).items():
             setattr(ep, name, f)
-        x = oin.x_rows(cfg, np.arange(rank * T_r, (rank + 1) * T_r))
-        y = layer(x.to(torch.float32))
-        ref = oracle.layer_forward(cfg, wd, x)["y"]
-        err = float((y.to(torch.float64) - ref).abs().max() / ref.pow(2).mean().sqrt())
-        copies = len(layer.last_plan.replicas[rank]) if balance else 0
-        out[rank] = (err, copies)
+        sent = []  # the copies requested from their owners, per step
+        orig = ep.exchange_expert_slices
+
+        def recorded(want, *a, **kw):
+            sent.append([list(v) for v in want])
+            return orig(want, *a, **kw)
+
+        ep.exchange_expert_slices = recorded
+        # three steps: a batch, the same batch again (its copies are all held),
+        # then another batch (only the copies not held travel)
+        errs, copies = [], []
+        for b in (0, 0, 1):
+            x = oin.x_rows(cfg, np.arange((b * world + rank) * T_r, (b * world + rank + 1) * T_r))
+            y = layer(x.to(torch.float32))
+            ref = oracle.layer_forward(cfg, wd, x)["y"]
+            errs.append(float((y.to(torch.float64) - ref).abs().max() / ref.pow(2).mean().sqrt()))
+            copies.append(len(layer.last_plan.replicas[rank]) if balance else 0)
+        if balance:
+            assert not any(sent[1]), "a repeated plan sends no weights"
+            assert all(set(sent[2][g]) <= set(layer.last_plan.replicas[g]) for g in range(world))
+        out[rank] = (max(errs), sum(copies))
     finally:
         dist.destroy_process_group()
 
