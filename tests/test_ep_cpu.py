@@ -447,7 +447,7 @@ def _layer_worker(rank, world, port, balance, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,balance", [(2, True), (3, True), (3, False)])
+@pytest.mark.parametrize("world,balance", [(1, True), (2, True), (3, True), (3, False)])
 def test_gloo_layer_step_matches_the_oracle(world, balance):
     """The expert-parallel layer's own forward step on gloo ranks, each with
     its own tokens and only its own experts' weights, the library entries
@@ -459,7 +459,7 @@ def test_gloo_layer_step_matches_the_oracle(world, balance):
     mp.spawn(_layer_worker, args=(world, _free_port(), balance, out), nprocs=world, join=True)
     for r in range(world):
         assert out[r][0] <= 1e-5, (r, out[r])
-    if balance:
+    if balance and world > 1:
         assert sum(out[r][1] for r in range(world)) > 0, "some rank ran a redundant copy"
 
 
