@@ -232,19 +232,21 @@ class BalancedExchange:
     n_recv: int
 
 
-def _pieces(plan: BalancedPlan, counts: np.ndarray, s: int):
-    """(destination, local expert index there, first row of the piece within
-    the sender's expert-major rows of that expert, rows) for sender s."""
-    local = {g: {int(e): i for i, e in enumerate(plan.local_experts(g))} for g in range(len(plan.quota))}
-    before = counts[:s].sum(axis=0)  # rows of each expert from earlier senders
-    out = []
-    for e in np.nonzero(counts[s])[0]:
-        lo, hi = int(before[e]), int(before[e] + counts[s, e])
-        for g, st, n in plan.segments[e]:
-            a, b = max(lo, st), min(hi, st + n)
-            if a < b:
-                out.append((g, local[g][int(e)], int(e), a - lo, b - a))
-    return out
+def _segment_table(plan: BalancedPlan):
+    """The plan's segments as arrays (expert, rank, start, rows) and each
+    segment's local expert index on its rank (own experts first, then copies
+    in ascending id order)."""
+    seg = [(e, g, st, n) for e, lst in enumerate(plan.segments) for g, st, n in lst]
+    if not seg:
+        z = np.zeros(0, np.int64)
+        return z, z, z, z, z
+    e, g, st, n = (np.array(c, np.int64) for c in zip(*seg))
+    n_home = np.diff(plan.bounds)
+    local = e - plan.bounds[g]
+    own = (local >= 0) & (local < n_home[g])
+    for i in np.nonzero(~own)[0]:
+        local[i] = n_home[g[i]] + plan.replicas[g[i]].index(int(e[i]))
+    return e, g, st, n, local
 
 
 def balanced_exchange(plan: BalancedPlan, counts: np.ndarray, offsets: np.ndarray, rank: int) -> BalancedExchange:
@@ -256,28 +258,34 @@ def balanced_exchange(plan: BalancedPlan, counts: np.ndarray, offsets: np.ndarra
     counts = np.asarray(counts, np.int64)
     G = len(plan.quota)
     n_local = len(plan.local_experts(rank))
-    by_dest = [[] for _ in range(G)]
-    for g, li, e, first, n in _pieces(plan, counts, rank):
-        by_dest[g].append((li, int(offsets[e]) + first, n))
-    idx, send_rows = [], []
-    for g in range(G):
-        pieces = sorted(by_dest[g])
-        send_rows.append(sum(n for _, _, n in pieces))
-        idx += [np.arange(st, st + n, dtype=np.int64) for _, st, n in pieces]
-    send_idx = np.concatenate(idx) if idx else np.zeros(0, np.int64)
-    blocks = np.zeros((G, n_local + 1), np.int64)
-    start = 0
+    e, g, st, n, local = _segment_table(plan)
+    # rows of each expert from earlier senders: sender s's rows of expert e
+    # are positions [before[s, e], before[s, e] + counts[s, e]) of e's rows
+    before = np.cumsum(counts, axis=0) - counts
+    lo = before[:, e]
+    hi = lo + counts[:, e]
+    a = np.maximum(lo, st[None, :])
+    overlap = np.maximum(np.minimum(hi, (st + n)[None, :]) - a, 0)  # [senders, segments]
+    # this rank's sends: pieces ordered by (destination, its local expert)
+    mine = np.nonzero(overlap[rank] > 0)[0]
+    order = mine[np.lexsort((local[mine], g[mine]))]
+    starts = np.asarray(offsets, np.int64)[e[order]] + (a[rank, order] - lo[rank, order])
+    lens = overlap[rank, order]
+    total = int(lens.sum())
+    first = np.cumsum(lens) - lens
+    send_idx = np.repeat(starts - first, lens) + np.arange(total, dtype=np.int64)
+    send_rows = np.bincount(g[order], weights=lens, minlength=G).astype(np.int64).tolist()
+    # this rank's receives: per source, rows per local expert
+    here = np.nonzero(g == rank)[0]
+    per = np.zeros((G, n_local), np.int64)
     for s in range(G):
-        per = np.zeros(n_local, np.int64)
-        for g, li, _, _, n in _pieces(plan, counts, s):
-            if g == rank:
-                per[li] += n
-        blocks[s, 0] = start
-        blocks[s, 1:] = start + np.cumsum(per)
-        start = int(blocks[s, -1])
-    return BalancedExchange(send_idx=send_idx, send_rows=send_rows,
-                            recv_rows=[int(blocks[s, -1] - blocks[s, 0]) for s in range(G)],
-                            recv_block_offsets=blocks, n_recv=start)
+        np.add.at(per[s], local[here], overlap[s, here])
+    blocks = np.zeros((G, n_local + 1), np.int64)
+    tot = per.sum(axis=1)
+    blocks[:, 0] = np.cumsum(tot) - tot
+    blocks[:, 1:] = blocks[:, :1] + np.cumsum(per, axis=1)
+    return BalancedExchange(send_idx=send_idx, send_rows=[int(v) for v in send_rows],
+                            recv_rows=[int(v) for v in tot], recv_block_offsets=blocks, n_recv=int(tot.sum()))
 
 
 def gather_counts(offsets: np.ndarray, group=None) -> np.ndarray:
