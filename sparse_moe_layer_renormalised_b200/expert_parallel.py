@@ -189,17 +189,19 @@ def balanced_plan(counts: np.ndarray, bounds: np.ndarray) -> BalancedPlan:
     deficit = np.maximum(-excess, 0)
     receivers = [g for g in range(G) if deficit[g] > 0]
     keep = C.copy()                     # rows the owner keeps
-    given: list = [[] for _ in range(len(C))]  # per expert: (rank, rows) handed over, in order
+    given: dict = {}                    # expert -> [(rank, rows)] handed over, in order
     ri = 0
     for d in range(G):
         need = int(excess[d])
         if need <= 0:
             continue
-        for e in sorted(range(bounds[d], bounds[d + 1]), key=lambda e: (-C[e], e)):
+        ids = np.arange(bounds[d], bounds[d + 1])
+        for e in ids[np.lexsort((ids, -C[ids]))]:  # hottest first, ties to the lower id
+            e = int(e)
             while need > 0 and keep[e] > 0:
                 r = receivers[ri]
                 n = int(min(need, keep[e], deficit[r]))
-                given[e].append((r, n))
+                given.setdefault(e, []).append((r, n))
                 keep[e] -= n
                 need -= n
                 deficit[r] -= n
@@ -208,15 +210,14 @@ def balanced_plan(counts: np.ndarray, bounds: np.ndarray) -> BalancedPlan:
             if need == 0:
                 break
     owner = np.searchsorted(bounds, np.arange(len(C)), side="right") - 1
-    segments, replicas = [], [[] for _ in range(G)]
-    for e in range(len(C)):
-        seg = [(int(owner[e]), 0, int(keep[e]))] if keep[e] > 0 else []
+    segments = [[(int(o), 0, int(c))] if c > 0 else [] for o, c in zip(owner.tolist(), keep.tolist())]
+    replicas = [[] for _ in range(G)]
+    for e, lst in given.items():
         start = int(keep[e])
-        for r, n in given[e]:
-            seg.append((r, start, n))
+        for r, n in lst:
+            segments[e].append((r, start, n))
             replicas[r].append(e)
             start += n
-        segments.append(seg)
     return BalancedPlan(bounds=np.asarray(bounds, np.int64), quota=quota, segments=segments,
                         replicas=[sorted(set(x)) for x in replicas])
 
