@@ -7,7 +7,7 @@
 //
 // Same work decomposition and operand swap as gemm_expert.cuh (weight rows are
 // the MMA's M on a 2-CTA pair, M = 256; token rows its N), with these
-// differences:
+// differences (as written for MXFP8 inputs; MXFP4 inputs below):
 //  * a stage covers K = 256 (two 128-wide halves, 8 MMAs of K = 32).  The MMA
 //    issue is single-threaded and each barrier wait costs it a few hundred
 //    cycles (measured on B200: ~250 cycles per mbarrier check and ~50 per
@@ -33,12 +33,12 @@
 // element in the low nibble), which kind::mxf4 reads as they are: a 128-byte
 // wide box (plain byte TMA, 128-byte swizzle) holds K = 256, and a stage
 // covers K = 512 in two such slices, 8 MMAs of K = 64, each taking two scale
-// bytes (j = 0 or 2) of one 128-wide K chunk's scale columns.  K = 512 per
-// stage halves the per-stage waits, copies and commits of the single-thread
-// roles against K = 256 (measured on B200: at K = 256 the all-4-bit stage
-// took ~1500 cycles with the tensor pipe 21% busy).  Its token box is at most
-// 104 rows per CTA (the tile's half), so that three stages fit; its four
-// chunks' scales take 48 tensor-memory columns per buffer, so two buffers.
+// bytes (j = 0 or 2) of one 128-wide K chunk's scale columns, so that a
+// stage again carries 8 MMAs per wait and commit (measured on B200 at the K3
+// shape, K = 256 and K = 512 stages gave the same time: the data path, not the
+// single-thread roles, bounds this kernel).  Its token box is at most 104
+// rows per CTA (the tile's half), so that three stages fit; its four chunks'
+// scales take 48 tensor-memory columns per buffer, so two buffers.
 // Warp roles: 0 TMA producer (both CTAs), 1 TMEM owner and MMA issuer (even
 // CTA), 2-5 and 7-10 epilogue (both CTAs), 6 scale copier (even CTA).  The
 // two epilogue sets of four warps (one per tensor-memory lane quarter each)
