@@ -178,7 +178,7 @@ def _e2m1_table():
     return np.array([tab[c] for c in range(16)])
 
 
-def test_e2m1_encode_is_the_nearest_code_ties_to_even(O):
+def _pin_e2m1_encode(encode):
     """Brute force over the OCP table: every value maps to the code whose value
     is nearest (magnitudes beyond 6 to +-6), a tie going to the even code; the
     sign is kept, -0 included.  Midpoints of every neighbour pair are in the
@@ -190,23 +190,27 @@ def test_e2m1_encode_is_the_nearest_code_ties_to_even(O):
     v = np.concatenate([mags, mids, np.nextafter(mids, 0), np.nextafter(mids, 10), rng.uniform(0, 9, 5000),
                         [6.5, 7.0, 100.0, 1e300]])
     v = np.concatenate([v, -v])
-    got = O.e2m1_encode(torch.from_numpy(v))
+    got = encode(torch.from_numpy(v))
     for x, c in zip(v, got):
         a = min(abs(x), 6.0)
         d = np.abs(mags - a)
         best = np.flatnonzero(d == d.min())
         want = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
         assert c == (want | (8 if np.signbit(x) else 0)), (x, c)
-    assert list(O.e2m1_encode(torch.tensor([0.0, -0.0], dtype=F64))) == [0, 8]
-    assert np.array_equal(O.e2m1_encode(torch.from_numpy(tab[np.r_[0:8, 9:16]])), np.r_[0:8, 9:16])
+    assert list(encode(torch.tensor([0.0, -0.0], dtype=F64))) == [0, 8]
+    assert np.array_equal(encode(torch.from_numpy(tab[np.r_[0:8, 9:16]])), np.r_[0:8, 9:16])
 
 
-def test_mx4_scale_rule_closed_forms(O):
+def test_e2m1_encode_is_the_nearest_code_ties_to_even(O):
+    _pin_e2m1_encode(O.e2m1_encode)
+
+
+def _pin_mx4_scale_rule(quantize):
     """OCP MX v1.0 shared scale of an MXFP4 block, s = floor(log2 max|v|) - 2,
     clamped to the E8M0 range; codes of v / 2^s packed two per byte, the even
     element in the low nibble."""
     def q(block):
-        c, s = O.mx4_quantize(torch.tensor([block], dtype=F64))
+        c, s = quantize(torch.tensor([block], dtype=F64))
         return c[0], int(s[0, 0])
 
     c, s = q([1.0] * 32)                      # s = -2: 1 -> 4, code 6
@@ -221,8 +225,72 @@ def test_mx4_scale_rule_closed_forms(O):
     assert s == 227 and c[0] == 0x70
     c, s = q([2.0**-130] + [0.0] * 31)        # clamped at -127: 2^-130 * 2^127 = 0.125 rounds to 0
     assert s == 0 and set(c) == {0}
-    v = torch.tensor([[0.2] * 16 + [5.0] * 16], dtype=F64)  # s = 0: 0.2 -> 0 (nearest of 0, 0.5)
-    assert O.mx4_round(v)[0, 0].item() == 0.0 and O.mx4_round(v)[0, 16].item() == 4.0
+    c, s = q([0.2] * 16 + [5.0] * 16)         # s = 0: 0.2 -> 0 (nearest of 0, 0.5), 5 -> 4 (tie, even code 6)
+    assert s == 127 and set(c[:8]) == {0} and set(c[8:]) == {0x66}
+
+
+def test_mx4_scale_rule_closed_forms(O):
+    _pin_mx4_scale_rule(O.mx4_quantize)
+
+
+# Plausible slips, planted in copies of the oracle's encoders on the CPU: each
+# must fail the pins above.
+def _e2m1_mutant(kind):
+    def encode(v):
+        v = torch.as_tensor(v).to(F64)
+        neg = torch.signbit(v)
+        a = torch.clamp(v.abs(), max=4.0 if kind == "saturate_at_4" else 6.0)
+        _, ex = torch.frexp(a)
+        q = torch.clamp(ex.to(torch.int64) - 1, min=0)
+        x = torch.ldexp(a, (1 - q).to(torch.int64))
+        units = torch.floor(x + 0.5) if kind == "ties_away" else torch.round(x)
+        if kind == "subnormal_spacing":  # below 1 the step taken as 1 instead of 0.5
+            units = torch.where(q == 0, 2 * torch.round(x / 2), units)
+        carry = (q >= 1) & (units >= 4)
+        q = torch.where(carry, q + 1, q)
+        units = torch.where(carry, units / 2, units).to(torch.int64)
+        code = torch.where(q == 0, units, ((q + 1) << 1) | (units - 2))
+        if kind != "sign_dropped":
+            code = torch.where(neg, code | 8, code)
+        return code.to(torch.uint8).numpy()
+    return encode
+
+
+def _mx4_mutant(kind):
+    def quantize(v):
+        v = torch.as_tensor(v).to(F64)
+        R, K = v.shape
+        blocks = v.reshape(R, K // 32, 32)
+        amax = blocks.abs().amax(dim=2)
+        _, ex = torch.frexp(amax)
+        emax = {"emax_1": 1, "emax_3": 3}.get(kind, 2)
+        fl = ex.to(torch.int64) - 1
+        if kind == "round_log2":
+            fl = torch.round(torch.log2(torch.where(amax > 0, amax, torch.ones_like(amax)))).to(torch.int64)
+        s = torch.clamp(fl - emax, min=-127, max=127)
+        s = torch.where(amax == 0, torch.full_like(s, 0 if kind == "zero_block_scale_1" else -127), s)
+        nib = oracle.torch_ref.e2m1_encode(torch.ldexp(blocks, (-s)[:, :, None].expand(R, K // 32, 32)).reshape(R, K))
+        lo, hi = (nib[:, 1::2], nib[:, 0::2]) if kind == "nibbles_swapped" else (nib[:, 0::2], nib[:, 1::2])
+        return (lo | (hi << 4)).astype(np.uint8), (s + 127).to(torch.uint8).numpy()
+    return quantize
+
+
+@pytest.mark.parametrize("kind", ["ties_away", "saturate_at_4", "subnormal_spacing", "sign_dropped"])
+def test_e2m1_pin_catches_a_planted_slip(kind):
+    with pytest.raises(AssertionError):
+        _pin_e2m1_encode(_e2m1_mutant(kind))
+
+
+@pytest.mark.parametrize("kind", ["emax_1", "emax_3", "round_log2", "zero_block_scale_1", "nibbles_swapped"])
+def test_mx4_pin_catches_a_planted_slip(kind):
+    with pytest.raises(AssertionError):
+        _pin_mx4_scale_rule(_mx4_mutant(kind))
+
+
+def test_unmutated_copies_pass_the_pins():
+    """The copies the slips are planted in are faithful without a slip."""
+    _pin_e2m1_encode(_e2m1_mutant("none"))
+    _pin_mx4_scale_rule(_mx4_mutant("none"))
 
 
 def test_mx4_round_is_the_nearest_block_value_and_idempotent(O):
