@@ -529,7 +529,10 @@ def workload_line(cfg, layer, x, args, world, rank, local_rank, peaks, headline:
     if world == 1:
         out["near_tie_tokens"], idx = routing_of_batch(layer, x, cfg)
         if cfg.E >= 8:
-            out["ep_balance"] = ep_balance(idx, cfg.E)
+            try:  # an informational host statistic: it never costs the measured line
+                out["ep_balance"] = ep_balance(idx, cfg.E)
+            except Exception as exc:  # noqa: BLE001
+                out["ep_balance"] = {"error": f"{type(exc).__name__}: {exc}"}
         if not args.no_oracle:
             parity, cpu = oracle_sample(cfg, layer, x, args.cpu_tokens)
             out["parity"] = parity
