@@ -6,6 +6,7 @@ import re
 
 import pytest
 
+import gen
 import sparse_moe_layer_renormalised_b200 as moe
 from conftest import ROOT
 
@@ -226,3 +227,17 @@ def test_structs_keep_their_tensors_alive():
         del s
         gc.collect()
         assert ref() is None
+
+
+@pytest.mark.parametrize("name", sorted(gen.CONFIGS))
+def test_every_workload_is_valid_and_supported(name):
+    """Every workload of gen/configs.py passes the library's host-side dims
+    rules (valid and implemented), so its workspace size is positive; the
+    block-scaled ones also size their tiled weight scales."""
+    cfg = gen.CONFIGS[name]
+    d = moe.Dims(T=cfg.T, H=cfg.H, L=cfg.L, E=cfg.E, k=cfg.k, I=cfg.I, S=cfg.S, Is=cfg.Is, act=cfg.act,
+                 routed=cfg.routed, y_out="f32", situ_c=cfg.situ_c, rms_eps=cfg.rms_eps)
+    assert moe.moe_workspace_size(d) > 0
+    if cfg.routed in moe.BLOCK_SCALED:
+        st, gu, dn = moe.moe_mx_tiled_scales_size(d)
+        assert st == moe.MOE_OK and gu == cfg.E * cfg.I * cfg.L // 16 and dn == cfg.E * cfg.L * cfg.I // 32
